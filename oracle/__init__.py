@@ -1,0 +1,192 @@
+"""fp64 CPU oracle for kernelised linear attention -- TEST INFRASTRUCTURE.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never touches it, and it shares no code with them.
+
+Thin ctypes wrappers around ``lt_oracle.c``.  Every function takes CPU arrays
+(numpy, or torch CPU tensors) holding the exact values given to the GPU
+(float32, bfloat16 or float64), widens them to fp64 and returns fp64 numpy
+arrays.  Layouts are token-major: dense ``[B][N][H][d]``, packed
+``[N_total][H][d]`` with ``cu_seqlens``.  The mathematics and the page each
+function follows are documented in ``lt_oracle.c``.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_F32, _BF16, _F64 = 0, 1, 2
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        vp, dp, ip = ctypes.c_void_p, ctypes.POINTER(ctypes.c_double), ctypes.c_int
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        fwd_args = [vp, vp, vp, ip, dp, ip, ip, ip, ip, ip, ip, ip, ctypes.c_double, i32p]
+        lib.lt_oracle_fwd_quadratic.argtypes = fwd_args
+        lib.lt_oracle_fwd_recurrent.argtypes = fwd_args
+        lib.lt_oracle_fwd_rows.argtypes = [vp, vp, vp, ip, ip, ip, ip, ip, ip, ip, ip,
+                                           ctypes.c_double, i32p, i64p, ip, dp]
+        lib.lt_oracle_noncausal_numerator.argtypes = [vp, vp, vp, ip, dp, ip, ip, ip, ip, ip,
+                                                      ip, i32p, ip]
+        lib.lt_oracle_decode_step.argtypes = [vp, vp, vp, ip, dp, dp, dp, ip, ip, ip, ip, ip,
+                                              ctypes.c_double]
+        lib.lt_oracle_phi.argtypes = [ctypes.c_double]
+        lib.lt_oracle_phi.restype = ctypes.c_double
+        lib.lt_oracle_num_threads.restype = ctypes.c_int
+        for name in ("lt_oracle_fwd_quadratic", "lt_oracle_fwd_recurrent", "lt_oracle_fwd_rows",
+                     "lt_oracle_noncausal_numerator", "lt_oracle_decode_step"):
+            getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _raw(x):
+    """Return (contiguous numpy array holding the raw bits, type code)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous()
+            if x.dtype == torch.bfloat16:
+                return x.view(torch.int16).numpy().view(np.uint16), _BF16
+            if x.dtype == torch.float32:
+                return x.numpy(), _F32
+            if x.dtype == torch.float64:
+                return x.numpy(), _F64
+            raise TypeError("unsupported dtype %s" % x.dtype)
+    except ImportError:
+        pass
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float32:
+        return x, _F32
+    if x.dtype == np.float64:
+        return x, _F64
+    raise TypeError("unsupported dtype %s" % x.dtype)
+
+
+def _same_type(*arrs):
+    raws = [_raw(a) for a in arrs]
+    types = {t for _, t in raws}
+    if len(types) != 1:
+        raise TypeError("q, k, v must share one dtype")
+    return [r for r, _ in raws], types.pop()
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _cu(cu_seqlens):
+    if cu_seqlens is None:
+        return None, None
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    return cu, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def _geometry(q, k, v, cu_seqlens):
+    """(B, Hq, Hkv, N, d, dv, out_shape) from token-major shapes."""
+    if cu_seqlens is None:
+        B, N, Hq, d = q.shape
+        Hkv, dv = k.shape[2], v.shape[3]
+        return B, Hq, Hkv, N, d, dv, (B, N, Hq, dv)
+    N, Hq, d = q.shape
+    Hkv, dv = k.shape[1], v.shape[2]
+    B = len(cu_seqlens) - 1
+    return B, Hq, Hkv, N, d, dv, (N, Hq, dv)
+
+
+def phi(x: float) -> float:
+    """phi(x) = ELU(x) + 1 (alpha = 1), in fp64."""
+    return _load().lt_oracle_phi(float(x))
+
+
+def num_threads() -> int:
+    return _load().lt_oracle_num_threads()
+
+
+def _fwd(fn, q, k, v, causal, eps, cu_seqlens):
+    (rq, rk, rv), t = _same_type(q, k, v)
+    B, Hq, Hkv, N, d, dv, oshape = _geometry(rq, rk, rv, cu_seqlens)
+    out = np.zeros(oshape, dtype=np.float64)
+    cu, cup = _cu(cu_seqlens)
+    rc = fn(_ptr(rq), _ptr(rk), _ptr(rv), t, _dptr(out), B, Hq, Hkv, N, d, dv,
+            int(bool(causal)), float(eps), cup)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
+
+
+def fwd_quadratic(q, k, v, causal=True, eps=1e-6, cu_seqlens=None):
+    """Masked quadratic form: O_i = sum_j a_ij V_j / (sum_j a_ij + eps)."""
+    return _fwd(_load().lt_oracle_fwd_quadratic, q, k, v, causal, eps, cu_seqlens)
+
+
+def fwd_recurrent(q, k, v, causal=True, eps=1e-6, cu_seqlens=None):
+    """Recurrent (RNN) form over the fixed-size state (S, z)."""
+    return _fwd(_load().lt_oracle_fwd_recurrent, q, k, v, causal, eps, cu_seqlens)
+
+
+def fwd_rows(q, k, v, rows, causal=True, eps=1e-6, cu_seqlens=None):
+    """Selected output rows by the quadratic definition.
+
+    ``rows``: integer array of shape [R, 3] holding (sequence, position
+    within the sequence, query head).  Returns fp64 [R, dv].
+    """
+    (rq, rk, rv), t = _same_type(q, k, v)
+    B, Hq, Hkv, N, d, dv, _ = _geometry(rq, rk, rv, cu_seqlens)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    out = np.zeros((rows.shape[0], dv), dtype=np.float64)
+    cu, cup = _cu(cu_seqlens)
+    rc = _load().lt_oracle_fwd_rows(_ptr(rq), _ptr(rk), _ptr(rv), t, B, Hq, Hkv, N, d, dv,
+                                    int(bool(causal)), float(eps), cup,
+                                    rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                    rows.shape[0], _dptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected a row index")
+    return out
+
+
+def noncausal_numerator(q, k, v, order, cu_seqlens=None):
+    """Unnormalised phi(Q)(phi(K)^T V); order 0 = scores first, 1 = KV first."""
+    (rq, rk, rv), t = _same_type(q, k, v)
+    B, Hq, Hkv, N, d, dv, oshape = _geometry(rq, rk, rv, cu_seqlens)
+    out = np.zeros(oshape, dtype=np.float64)
+    cu, cup = _cu(cu_seqlens)
+    rc = _load().lt_oracle_noncausal_numerator(_ptr(rq), _ptr(rk), _ptr(rv), t, _dptr(out),
+                                               B, Hq, Hkv, N, d, dv, cup, int(order))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
+
+
+def decode_step(q, k, v, S, z, eps=1e-6):
+    """One recurrent decode step.
+
+    q [B][Hq][d], k [B][Hkv][d], v [B][Hkv][dv]; S [B][Hkv][d][dv] and
+    z [B][Hkv][d] are fp64 numpy arrays updated in place.  Returns
+    out [B][Hq][dv] in fp64.
+    """
+    (rq, rk, rv), t = _same_type(q, k, v)
+    B, Hq, d = rq.shape
+    Hkv, dv = rk.shape[1], rv.shape[2]
+    if S.dtype != np.float64 or z.dtype != np.float64 or not S.flags.c_contiguous \
+            or not z.flags.c_contiguous:
+        raise TypeError("S and z must be C-contiguous float64 arrays")
+    out = np.zeros((B, Hq, dv), dtype=np.float64)
+    rc = _load().lt_oracle_decode_step(_ptr(rq), _ptr(rk), _ptr(rv), t, _dptr(S), _dptr(z),
+                                       _dptr(out), B, Hq, Hkv, d, dv, float(eps))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out

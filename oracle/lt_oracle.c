@@ -1,0 +1,348 @@
+/*
+ * lt_oracle.c -- plain fp64 CPU oracle for kernelised (linear) attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file or the library built from it; only the test suite, the
+ * package's smoke check and the benchmark's CPU-baseline leg use it.  It
+ * shares no code, header, table or constant with the CUDA library.
+ *
+ * What it computes (sources, by page and section):
+ *   - "lineartile 1.0.0" (PyPI page), section "How It Works": the feature map
+ *     phi(x) = ELU(x) + 1 and the reordered non-causal product
+ *     phi(Q) (phi(K)^T V), i.e. compute phi(K)^T V first.
+ *   - same page, section "Reference": the method is the linear attention of
+ *     "Transformers are RNNs" (Katharopoulos et al., 2020): causal output
+ *         O_i = phi(Q_i) S_i / (phi(Q_i) . z_i + eps),
+ *         S_i = sum_{j<=i} phi(K_j)^T V_j,   z_i = sum_{j<=i} phi(K_j),
+ *     which can be evaluated either as a masked quadratic form or as a
+ *     recurrence over a fixed-size state (the "RNN view").
+ *   - same page, section "Features": variable sequence length (packed
+ *     sequences, no padding), grouped-query attention, KV-cache reuse
+ *     (for linear attention the cache is the fixed-size (S, z) state).
+ *   - "Why Stream Wins at Ultra-Long Context", section 4.2: the forward
+ *     linear recurrence h_t = h_{t-1} a_t + b_t, here with a_t = 1 and
+ *     b_t = phi(K_t)^T V_t.
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   ELU alpha = 1; no 1/sqrt(d) score scale inside the method; eps is added
+ *   to the denominator only; the causal sum is inclusive (j <= i); the
+ *   non-causal mode returns the same normalised form with the sum over all
+ *   j; query head h uses KV head floor(h * H_kv / H_q); token-major layouts
+ *   [B][N][H][d] (dense) and [N_total][H][d] (packed, cu_seqlens).
+ *
+ * Every input is widened exactly to double before any arithmetic: bf16 and
+ * fp32 values are exactly representable in fp64, so the oracle sees the very
+ * values the GPU sees.  All arithmetic is fp64.
+ *
+ * Pins (tests in tests/test_oracle_pins.py): a hand-worked 2x2 example,
+ * agreement of the two independent forms, associativity of the non-causal
+ * product, closed forms (constant keys -> prefix mean of V), invariants
+ * (denominator > 0, implied weights sum to 1 - eps/den), GQA == explicit KV
+ * replication, packed == independent per-sequence calls, decode chaining ==
+ * quadratic causal form.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* element type codes for the raw input buffers */
+#define ORC_F32 0
+#define ORC_BF16 1
+#define ORC_F64 2
+
+/* Read element idx of a raw buffer of the given type, widened to double. */
+static double load_elem(const void *p, int64_t idx, int type) {
+    if (type == ORC_F64) return ((const double *)p)[idx];
+    if (type == ORC_F32) return (double)((const float *)p)[idx];
+    /* bf16: the 16 stored bits are the high half of an IEEE binary32 */
+    uint32_t bits = (uint32_t)((const uint16_t *)p)[idx] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* phi(x) = ELU(x) + 1 with alpha = 1: x + 1 for x > 0, exp(x) for x <= 0. */
+double lt_oracle_phi(double x) { return x > 0.0 ? x + 1.0 : exp(x); }
+
+int lt_oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Sequence geometry: start token (in the packed/dense token index space of
+ * one batch row) and length.  Dense mode: every sequence has N tokens and
+ * lives in its own batch row; packed mode: one batch row, offsets from
+ * cu_seqlens. */
+static void seq_range(int s, int N, const int32_t *cu, int64_t *base_tok, int64_t *len) {
+    if (cu) {
+        *base_tok = cu[s];
+        *len = (int64_t)cu[s + 1] - cu[s];
+    } else {
+        *base_tok = (int64_t)s * N;
+        *len = N;
+    }
+}
+
+/* Flat offset of element c of row (token t, head h) in a token-major tensor
+ * whose rows have H heads of width w.  t is the global token index
+ * (b*N + n in dense mode, the packed index in packed mode). */
+static int64_t off(int64_t t, int h, int H, int w, int c) {
+    return ((t * H + h) * (int64_t)w) + c;
+}
+
+static int check_args(int B, int Hq, int Hkv, int N, int d, int dv, double eps) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || dv <= 0) return 1;
+    if (Hq % Hkv != 0) return 1;
+    if (!(eps >= 0.0)) return 1;
+    return 0;
+}
+
+/*
+ * Form 1: the masked quadratic form, straight from the definition.
+ * For each sequence, query head h (KV head g = h*Hkv/Hq) and query i:
+ *     a_ij = phi(Q_i) . phi(K_j)       for j <= i (all j when causal == 0)
+ *     O_i  = (sum_j a_ij V_j) / (sum_j a_ij + eps)
+ * O(n^2) per sequence: use only for small n.
+ */
+int lt_oracle_fwd_quadratic(const void *q, const void *k, const void *v, int in_type,
+                            double *out, int B, int Hq, int Hkv, int N, int d, int dv,
+                            int causal, double eps, const int32_t *cu_seqlens) {
+    if (check_args(B, Hq, Hkv, N, d, dv, eps)) return 1;
+    const int G = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int s = 0; s < B; ++s) {
+        for (int h = 0; h < Hq; ++h) {
+            const int g = h / G;
+            int64_t t0, n;
+            seq_range(s, N, cu_seqlens, &t0, &n);
+            double *pq = malloc(sizeof(double) * d);
+            double *pk = malloc(sizeof(double) * d);
+            double *num = malloc(sizeof(double) * dv);
+            for (int64_t i = 0; i < n; ++i) {
+                for (int c = 0; c < d; ++c) pq[c] = lt_oracle_phi(load_elem(q, off(t0 + i, h, Hq, d, c), in_type));
+                for (int c = 0; c < dv; ++c) num[c] = 0.0;
+                double den = 0.0;
+                const int64_t jend = causal ? i + 1 : n;
+                for (int64_t j = 0; j < jend; ++j) {
+                    for (int c = 0; c < d; ++c) pk[c] = lt_oracle_phi(load_elem(k, off(t0 + j, g, Hkv, d, c), in_type));
+                    double a = 0.0;
+                    for (int c = 0; c < d; ++c) a += pq[c] * pk[c];
+                    for (int c = 0; c < dv; ++c) num[c] += a * load_elem(v, off(t0 + j, g, Hkv, dv, c), in_type);
+                    den += a;
+                }
+                for (int c = 0; c < dv; ++c) out[off(t0 + i, h, Hq, dv, c)] = num[c] / (den + eps);
+            }
+            free(pq);
+            free(pk);
+            free(num);
+        }
+    }
+    return 0;
+}
+
+/*
+ * Form 2: the recurrence over the fixed-size state (the RNN view).
+ *     S <- 0 (d x dv), z <- 0 (d)
+ *     for i = 0..n-1:  S += phi(K_i)^T V_i;  z += phi(K_i);
+ *                      O_i = phi(Q_i) S / (phi(Q_i) . z + eps)
+ * Non-causal: run the state update over the whole sequence first, then
+ * evaluate every O_i with the final (S, z).
+ */
+int lt_oracle_fwd_recurrent(const void *q, const void *k, const void *v, int in_type,
+                            double *out, int B, int Hq, int Hkv, int N, int d, int dv,
+                            int causal, double eps, const int32_t *cu_seqlens) {
+    if (check_args(B, Hq, Hkv, N, d, dv, eps)) return 1;
+    const int G = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int s = 0; s < B; ++s) {
+        for (int h = 0; h < Hq; ++h) {
+            const int g = h / G;
+            int64_t t0, n;
+            seq_range(s, N, cu_seqlens, &t0, &n);
+            double *S = calloc((size_t)d * dv, sizeof(double));
+            double *z = calloc((size_t)d, sizeof(double));
+            double *pq = malloc(sizeof(double) * d);
+            double *pk = malloc(sizeof(double) * d);
+            double *vv = malloc(sizeof(double) * dv);
+            if (!causal) {
+                for (int64_t i = 0; i < n; ++i) {
+                    for (int c = 0; c < d; ++c) pk[c] = lt_oracle_phi(load_elem(k, off(t0 + i, g, Hkv, d, c), in_type));
+                    for (int c = 0; c < dv; ++c) vv[c] = load_elem(v, off(t0 + i, g, Hkv, dv, c), in_type);
+                    for (int a = 0; a < d; ++a) {
+                        for (int c = 0; c < dv; ++c) S[a * dv + c] += pk[a] * vv[c];
+                        z[a] += pk[a];
+                    }
+                }
+            }
+            for (int64_t i = 0; i < n; ++i) {
+                if (causal) {
+                    for (int c = 0; c < d; ++c) pk[c] = lt_oracle_phi(load_elem(k, off(t0 + i, g, Hkv, d, c), in_type));
+                    for (int c = 0; c < dv; ++c) vv[c] = load_elem(v, off(t0 + i, g, Hkv, dv, c), in_type);
+                    for (int a = 0; a < d; ++a) {
+                        for (int c = 0; c < dv; ++c) S[a * dv + c] += pk[a] * vv[c];
+                        z[a] += pk[a];
+                    }
+                }
+                for (int c = 0; c < d; ++c) pq[c] = lt_oracle_phi(load_elem(q, off(t0 + i, h, Hq, d, c), in_type));
+                double den = eps;
+                for (int a = 0; a < d; ++a) den += pq[a] * z[a];
+                for (int c = 0; c < dv; ++c) {
+                    double num = 0.0;
+                    for (int a = 0; a < d; ++a) num += pq[a] * S[a * dv + c];
+                    out[off(t0 + i, h, Hq, dv, c)] = num / den;
+                }
+            }
+            free(S);
+            free(z);
+            free(pq);
+            free(pk);
+            free(vv);
+        }
+    }
+    return 0;
+}
+
+/*
+ * Selected output rows by the quadratic definition, for checking outputs of
+ * very long sequences without evaluating every row.  rows holds nrows
+ * triples (sequence s, position i within the sequence, query head h);
+ * out_rows receives nrows x dv values.  Cost per row: O(i * (d + dv)).
+ */
+int lt_oracle_fwd_rows(const void *q, const void *k, const void *v, int in_type,
+                       int B, int Hq, int Hkv, int N, int d, int dv, int causal, double eps,
+                       const int32_t *cu_seqlens, const int64_t *rows, int nrows, double *out_rows) {
+    if (check_args(B, Hq, Hkv, N, d, dv, eps)) return 1;
+    const int G = Hq / Hkv;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int r = 0; r < nrows; ++r) {
+        const int s = (int)rows[3 * r + 0];
+        const int64_t i = rows[3 * r + 1];
+        const int h = (int)rows[3 * r + 2];
+        int64_t t0, n;
+        if (s < 0 || s >= B || h < 0 || h >= Hq) { bad = 1; continue; }
+        seq_range(s, N, cu_seqlens, &t0, &n);
+        if (i < 0 || i >= n) { bad = 1; continue; }
+        const int g = h / G;
+        double *pq = malloc(sizeof(double) * d);
+        double *num = calloc((size_t)dv, sizeof(double));
+        for (int c = 0; c < d; ++c) pq[c] = lt_oracle_phi(load_elem(q, off(t0 + i, h, Hq, d, c), in_type));
+        double den = 0.0;
+        const int64_t jend = causal ? i + 1 : n;
+        for (int64_t j = 0; j < jend; ++j) {
+            double a = 0.0;
+            for (int c = 0; c < d; ++c) a += pq[c] * lt_oracle_phi(load_elem(k, off(t0 + j, g, Hkv, d, c), in_type));
+            for (int c = 0; c < dv; ++c) num[c] += a * load_elem(v, off(t0 + j, g, Hkv, dv, c), in_type);
+            den += a;
+        }
+        for (int c = 0; c < dv; ++c) out_rows[(int64_t)r * dv + c] = num[c] / (den + eps);
+        free(pq);
+        free(num);
+    }
+    return bad;
+}
+
+/*
+ * The unnormalised non-causal product of the "How It Works" section,
+ * evaluated in either association order:
+ *   order 0:  (phi(Q) phi(K)^T) V      -- scores first, O(n^2)
+ *   order 1:  phi(Q) (phi(K)^T V)      -- key/value product first, O(n)
+ * Mathematically identical; used to pin associativity.  Dense or packed.
+ */
+int lt_oracle_noncausal_numerator(const void *q, const void *k, const void *v, int in_type,
+                                  double *out, int B, int Hq, int Hkv, int N, int d, int dv,
+                                  const int32_t *cu_seqlens, int order) {
+    if (check_args(B, Hq, Hkv, N, d, dv, 0.0)) return 1;
+    const int G = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int s = 0; s < B; ++s) {
+        for (int h = 0; h < Hq; ++h) {
+            const int g = h / G;
+            int64_t t0, n;
+            seq_range(s, N, cu_seqlens, &t0, &n);
+            double *pq = malloc(sizeof(double) * d);
+            double *pk = malloc(sizeof(double) * d);
+            double *KV = calloc((size_t)d * dv, sizeof(double));
+            if (order == 1) {
+                for (int64_t j = 0; j < n; ++j) {
+                    for (int c = 0; c < d; ++c) pk[c] = lt_oracle_phi(load_elem(k, off(t0 + j, g, Hkv, d, c), in_type));
+                    for (int a = 0; a < d; ++a)
+                        for (int c = 0; c < dv; ++c)
+                            KV[a * dv + c] += pk[a] * load_elem(v, off(t0 + j, g, Hkv, dv, c), in_type);
+                }
+            }
+            for (int64_t i = 0; i < n; ++i) {
+                for (int c = 0; c < d; ++c) pq[c] = lt_oracle_phi(load_elem(q, off(t0 + i, h, Hq, d, c), in_type));
+                for (int c = 0; c < dv; ++c) {
+                    double acc = 0.0;
+                    if (order == 1) {
+                        for (int a = 0; a < d; ++a) acc += pq[a] * KV[a * dv + c];
+                    }
+                    out[off(t0 + i, h, Hq, dv, c)] = acc;
+                }
+                if (order == 0) {
+                    for (int64_t j = 0; j < n; ++j) {
+                        double a = 0.0;
+                        for (int c = 0; c < d; ++c) a += pq[c] * lt_oracle_phi(load_elem(k, off(t0 + j, g, Hkv, d, c), in_type));
+                        for (int c = 0; c < dv; ++c)
+                            out[off(t0 + i, h, Hq, dv, c)] += a * load_elem(v, off(t0 + j, g, Hkv, dv, c), in_type);
+                    }
+                }
+            }
+            free(pq);
+            free(pk);
+            free(KV);
+        }
+    }
+    return 0;
+}
+
+/*
+ * One recurrent decode step (the fixed-size state standing in for a KV
+ * cache).  For each batch row b and KV head g:
+ *     S[b][g] += phi(k)^T v,  z[b][g] += phi(k)        (update first: j <= i)
+ * then for every query head h of the group:
+ *     out[b][h] = phi(q[b][h]) S[b][g] / (phi(q[b][h]) . z[b][g] + eps)
+ * q [B][Hq][d], k [B][Hkv][d], v [B][Hkv][dv] (raw, in_type);
+ * S [B][Hkv][d][dv], z [B][Hkv][d] fp64 in/out; out [B][Hq][dv] fp64.
+ */
+int lt_oracle_decode_step(const void *q, const void *k, const void *v, int in_type,
+                          double *S, double *z, double *out, int B, int Hq, int Hkv, int d,
+                          int dv, double eps) {
+    if (check_args(B, Hq, Hkv, 1, d, dv, eps)) return 1;
+    const int G = Hq / Hkv;
+    for (int b = 0; b < B; ++b) {
+        for (int g = 0; g < Hkv; ++g) {
+            double *Sg = S + ((int64_t)b * Hkv + g) * d * dv;
+            double *zg = z + ((int64_t)b * Hkv + g) * d;
+            for (int a = 0; a < d; ++a) {
+                const double pk = lt_oracle_phi(load_elem(k, ((int64_t)b * Hkv + g) * d + a, in_type));
+                for (int c = 0; c < dv; ++c)
+                    Sg[a * dv + c] += pk * load_elem(v, ((int64_t)b * Hkv + g) * dv + c, in_type);
+                zg[a] += pk;
+            }
+        }
+        for (int h = 0; h < Hq; ++h) {
+            const int g = h / G;
+            const double *Sg = S + ((int64_t)b * Hkv + g) * d * dv;
+            const double *zg = z + ((int64_t)b * Hkv + g) * d;
+            double den = eps;
+            for (int a = 0; a < d; ++a)
+                den += lt_oracle_phi(load_elem(q, ((int64_t)b * Hq + h) * d + a, in_type)) * zg[a];
+            for (int c = 0; c < dv; ++c) {
+                double num = 0.0;
+                for (int a = 0; a < d; ++a)
+                    num += lt_oracle_phi(load_elem(q, ((int64_t)b * Hq + h) * d + a, in_type)) * Sg[a * dv + c];
+                out[((int64_t)b * Hq + h) * dv + c] = num / den;
+            }
+        }
+    }
+    return 0;
+}

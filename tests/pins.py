@@ -1,0 +1,265 @@
+"""Pins for the fp64 oracle: checks against facts the pages and the
+mathematics fix, independent of the oracle's own code.
+
+Each ``pin_*`` function raises AssertionError when the oracle (as currently
+loaded in the ``oracle`` package) violates the fact.  They are run directly
+by ``test_oracle_pins.py`` and against deliberately broken copies of the
+oracle by ``test_oracle_mutants.py`` (every planted mistake must trip at
+least one pin).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rand(shape, seed, scale=1.0):
+    g = np.random.default_rng(seed)
+    return g.standard_normal(shape) * scale
+
+
+def pin_phi_is_elu_plus_one():
+    """phi(x) = ELU(x) + 1 (alpha = 1), checked against torch's ELU."""
+    xs = np.concatenate([np.linspace(-30, 30, 601), [-1e-12, 0.0, 1e-12, -800.0]])
+    ref = torch.nn.functional.elu(torch.tensor(xs, dtype=torch.float64), alpha=1.0) + 1.0
+    got = np.array([oracle.phi(x) for x in xs])
+    # torch forms ELU+1 as expm1(x) + 1, whose absolute rounding is ~1e-16
+    assert np.allclose(got, ref.numpy(), rtol=1e-14, atol=2e-16), "phi != ELU+1"
+    assert oracle.phi(0.0) == 1.0 and oracle.phi(1.0) == 2.0
+    assert abs(oracle.phi(-math.log(2.0)) - 0.5) < 1e-16
+
+
+def _hand_2x2_inputs(g):
+    q = np.array(g["q"], dtype=np.float64).reshape(1, 2, 1, 2)
+    k = np.array([[1.0, 0.0], [0.0, -math.log(2.0)]]).reshape(1, 2, 1, 2)
+    v = np.array(g["v"], dtype=np.float64).reshape(1, 2, 1, 2)
+    return q, k, v
+
+
+def pin_hand_2x2():
+    """Hand-worked 2x2 example (tests/golden/hand_2x2.json)."""
+    g = _load("hand_2x2.json")
+    q, k, v = _hand_2x2_inputs(g)
+    for fn in (oracle.fwd_quadratic, oracle.fwd_recurrent):
+        got = fn(q, k, v, causal=True, eps=0.0)[0, :, 0]
+        assert np.allclose(got, g["causal_eps0"], rtol=0, atol=1e-15), (fn.__name__, got)
+        got = fn(q, k, v, causal=False, eps=0.0)[0, :, 0]
+        assert np.allclose(got, g["noncausal_eps0"], rtol=0, atol=1e-15), (fn.__name__, got)
+        got = fn(q, k, v, causal=True, eps=1e-6)[0, :, 0]
+        assert np.allclose(got, g["causal_eps1e-6"], rtol=0, atol=1e-15), (fn.__name__, got)
+    for order in (0, 1):
+        got = oracle.noncausal_numerator(q, k, v, order)[0, :, 0]
+        assert np.allclose(got, g["noncausal_numerator"], rtol=0, atol=1e-15), (order, got)
+    rows = np.array([[0, 0, 0], [0, 1, 0]])
+    got = oracle.fwd_rows(q, k, v, rows, causal=True, eps=0.0)
+    assert np.allclose(got, g["causal_eps0"], rtol=0, atol=1e-15)
+
+
+def hand_3tok_inputs(d=64, dv=64, dtype=torch.float32):
+    """The exact 3-token example embedded in d feature dims (padding -9984)."""
+    g = _load("hand_3tok_exact.json")
+    q = torch.full((1, 3, 1, d), g["pad_value"], dtype=torch.float64)
+    k = torch.full((1, 3, 1, d), g["pad_value"], dtype=torch.float64)
+    q[0, :, 0, :2] = torch.tensor(g["q_active"], dtype=torch.float64)
+    k[0, :, 0, :2] = torch.tensor(g["k_active"], dtype=torch.float64)
+    v = torch.zeros((1, 3, 1, dv), dtype=torch.float64)
+    for j in range(3):
+        v[0, j, 0, j] = 1.0
+    return q.to(dtype), k.to(dtype), v.to(dtype), g
+
+
+def pin_hand_3tok():
+    """Exact 3-token example with underflowing padding dims, fp32 and bf16 inputs."""
+    for dt in (torch.float32, torch.bfloat16):
+        q, k, v, g = hand_3tok_inputs(dtype=dt)
+        for fn in (oracle.fwd_quadratic, oracle.fwd_recurrent):
+            got = fn(q, k, v, causal=True, eps=0.0)[0, :, 0]
+            assert np.allclose(got[:, :3], g["causal_eps0_first3cols"], rtol=0, atol=1e-15)
+            assert np.all(got[:, 3:] == 0.0)
+            got = fn(q, k, v, causal=False, eps=0.0)[0, :, 0]
+            assert np.allclose(got[:, :3], g["noncausal_eps0_first3cols"], rtol=0, atol=1e-15)
+
+
+TWO_FORM_CASES = [
+    # (B, Hq, Hkv, N, d, dv, causal)
+    (1, 1, 1, 1, 1, 1, True),
+    (1, 1, 1, 7, 2, 3, True),
+    (2, 2, 1, 33, 3, 8, True),
+    (1, 4, 2, 65, 8, 2, False),
+    (2, 8, 2, 40, 64, 64, True),
+    (1, 2, 2, 19, 64, 128, False),
+]
+
+
+def pin_two_forms_agree():
+    """Quadratic and recurrent forms agree to 1e-12 relative (tiny inputs)."""
+    for i, (B, Hq, Hkv, N, d, dv, causal) in enumerate(TWO_FORM_CASES):
+        q = _rand((B, N, Hq, d), 10 + i)
+        k = _rand((B, N, Hkv, d), 20 + i)
+        v = _rand((B, N, Hkv, dv), 30 + i)
+        a = oracle.fwd_quadratic(q, k, v, causal=causal, eps=1e-6)
+        b = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
+        scale = max(1e-300, np.abs(a).max())
+        assert np.abs(a - b).max() <= 1e-12 * scale, (i, np.abs(a - b).max(), scale)
+
+
+def pin_associativity():
+    """(phi(Q) phi(K)^T) V == phi(Q) (phi(K)^T V); and the normalised
+    non-causal output equals numerator / numerator-with-V-all-ones."""
+    q = _rand((2, 23, 4, 5), 1)
+    k = _rand((2, 23, 2, 5), 2)
+    v = _rand((2, 23, 2, 6), 3)
+    n0 = oracle.noncausal_numerator(q, k, v, 0)
+    n1 = oracle.noncausal_numerator(q, k, v, 1)
+    assert np.abs(n0 - n1).max() <= 1e-12 * np.abs(n0).max()
+    den = oracle.noncausal_numerator(q, k, np.ones_like(v), 1)
+    o = oracle.fwd_recurrent(q, k, v, causal=False, eps=0.0)
+    assert np.abs(o - n0 / den).max() <= 1e-12 * np.abs(o).max()
+
+
+def pin_constant_keys_give_prefix_mean():
+    """All keys equal => every score in a row is equal => with eps = 0 the
+    causal output is the running mean of V and the non-causal one the mean."""
+    B, N, H, d, dv = 1, 17, 2, 4, 3
+    q = _rand((B, N, H, d), 4)
+    k = np.broadcast_to(_rand((1, 1, H, d), 5), (B, N, H, d)).copy()
+    v = _rand((B, N, H, dv), 6)
+    prefix_mean = np.cumsum(v, axis=1) / np.arange(1, N + 1).reshape(1, N, 1, 1)
+    for fn in (oracle.fwd_quadratic, oracle.fwd_recurrent):
+        o = fn(q, k, v, causal=True, eps=0.0)
+        assert np.abs(o - prefix_mean).max() <= 1e-13
+        o = fn(q, k, v, causal=False, eps=0.0)
+        assert np.abs(o - v.mean(axis=1, keepdims=True)).max() <= 1e-13
+
+
+def pin_first_row_is_v0():
+    """Causal row 0 sees only token 0: O_0 = V_0 * a/(a + eps)."""
+    q = _rand((2, 9, 3, 4), 7)
+    k = _rand((2, 9, 3, 4), 8)
+    v = _rand((2, 9, 3, 5), 9)
+    for fn in (oracle.fwd_quadratic, oracle.fwd_recurrent):
+        o = fn(q, k, v, causal=True, eps=0.0)
+        assert np.abs(o[:, 0] - v[:, 0]).max() <= 1e-14
+
+
+def pin_weights_sum_to_one_minus_eps_over_den():
+    """With V = 1 every output equals sum(a)/(sum(a)+eps): exactly 1 at eps=0,
+    in (0, 1) for eps > 0 and decreasing in eps; den > 0 always."""
+    q = _rand((1, 31, 2, 6), 11, 3.0)
+    k = _rand((1, 31, 2, 6), 12, 3.0)
+    ones = np.ones((1, 31, 2, 4))
+    for causal in (True, False):
+        for fn in (oracle.fwd_quadratic, oracle.fwd_recurrent):
+            o0 = fn(q, k, ones, causal=causal, eps=0.0)
+            assert np.abs(o0 - 1.0).max() <= 1e-14
+            o1 = fn(q, k, ones, causal=causal, eps=1e-3)
+            o2 = fn(q, k, ones, causal=causal, eps=1e-1)
+            assert np.all(o1 < 1.0) and np.all(o2 > 0.0) and np.all(o2 < o1)
+    # den from the V=1 output: 1 - O = eps/den  => den = eps/(1-O) > 0
+    o = oracle.fwd_recurrent(q, k, ones, causal=True, eps=1e-2)
+    assert np.all(1e-2 / (1.0 - o) > 0)
+
+
+def pin_convex_hull():
+    """At eps = 0 each causal output is a convex combination of V_0..V_i."""
+    q = _rand((1, 40, 2, 8), 13)
+    k = _rand((1, 40, 2, 8), 14)
+    v = _rand((1, 40, 2, 5), 15)
+    o = oracle.fwd_quadratic(q, k, v, causal=True, eps=0.0)
+    lo = np.minimum.accumulate(v, axis=1)
+    hi = np.maximum.accumulate(v, axis=1)
+    assert np.all(o >= lo - 1e-13) and np.all(o <= hi + 1e-13)
+
+
+def pin_gqa_equals_replication():
+    """H_kv < H_q equals explicit replication of each KV head over its group
+    of G = H_q/H_kv consecutive query heads."""
+    B, N, Hq, Hkv, d, dv = 2, 21, 8, 2, 4, 3
+    q = _rand((B, N, Hq, d), 16)
+    k = _rand((B, N, Hkv, d), 17)
+    v = _rand((B, N, Hkv, dv), 18)
+    G = Hq // Hkv
+    kr = np.repeat(k, G, axis=2)
+    vr = np.repeat(v, G, axis=2)
+    for causal in (True, False):
+        a = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
+        b = oracle.fwd_quadratic(q, kr, vr, causal=causal, eps=1e-6)
+        assert np.abs(a - b).max() <= 1e-12 * np.abs(b).max()
+
+
+def pin_packed_equals_independent():
+    """Packed sequences (cu_seqlens) equal independent dense calls."""
+    lens = [5, 1, 0, 12, 7]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T, Hq, Hkv, d, dv = int(cu[-1]), 4, 2, 3, 5
+    q = _rand((T, Hq, d), 19)
+    k = _rand((T, Hkv, d), 20)
+    v = _rand((T, Hkv, dv), 21)
+    for causal in (True, False):
+        for fn in (oracle.fwd_quadratic, oracle.fwd_recurrent):
+            packed = fn(q, k, v, causal=causal, eps=1e-6, cu_seqlens=cu)
+            for s, n in enumerate(lens):
+                if n == 0:
+                    continue
+                a, b = cu[s], cu[s + 1]
+                dense = oracle.fwd_quadratic(q[None, a:b], k[None, a:b], v[None, a:b],
+                                             causal=causal, eps=1e-6)[0]
+                assert np.abs(packed[a:b] - dense).max() <= 1e-12 * max(1.0, np.abs(dense).max())
+
+
+def pin_decode_chain_equals_causal():
+    """N decode steps from a zero state reproduce the causal forward row by row."""
+    B, N, Hq, Hkv, d, dv = 3, 11, 4, 2, 5, 6
+    q = _rand((B, N, Hq, d), 22)
+    k = _rand((B, N, Hkv, d), 23)
+    v = _rand((B, N, Hkv, dv), 24)
+    ref = oracle.fwd_quadratic(q, k, v, causal=True, eps=1e-6)
+    S = np.zeros((B, Hkv, d, dv))
+    z = np.zeros((B, Hkv, d))
+    for t in range(N):
+        o = oracle.decode_step(np.ascontiguousarray(q[:, t]), np.ascontiguousarray(k[:, t]),
+                               np.ascontiguousarray(v[:, t]), S, z, eps=1e-6)
+        assert np.abs(o - ref[:, t]).max() <= 1e-12 * max(1.0, np.abs(ref[:, t]).max())
+
+
+def pin_value_scaling_and_key_permutation():
+    """O(Q, K, cV) = c O(Q, K, V); non-causal output is invariant to a joint
+    permutation of the key/value tokens (queries held fixed)."""
+    q = _rand((1, 15, 2, 4), 25)
+    k = _rand((1, 15, 2, 4), 26)
+    v = _rand((1, 15, 2, 3), 27)
+    a = oracle.fwd_recurrent(q, k, v, causal=True, eps=1e-6)
+    b = oracle.fwd_recurrent(q, k, -2.5 * v, causal=True, eps=1e-6)
+    assert np.abs(b + 2.5 * a).max() <= 1e-12 * np.abs(b).max()
+    perm = np.random.default_rng(0).permutation(15)
+    o = oracle.noncausal_numerator(q, k, v, 0)
+    op = oracle.noncausal_numerator(q, k[:, perm], v[:, perm], 0)
+    assert np.abs(o - op).max() <= 1e-12 * np.abs(o).max()
+
+
+ALL_PINS = [
+    pin_phi_is_elu_plus_one,
+    pin_hand_2x2,
+    pin_hand_3tok,
+    pin_two_forms_agree,
+    pin_associativity,
+    pin_constant_keys_give_prefix_mean,
+    pin_first_row_is_v0,
+    pin_weights_sum_to_one_minus_eps_over_den,
+    pin_convex_hull,
+    pin_gqa_equals_replication,
+    pin_packed_equals_independent,
+    pin_decode_chain_equals_causal,
+    pin_value_scaling_and_key_permutation,
+]

@@ -1,0 +1,59 @@
+"""Power of the oracle pins: plant a plausible mistake in a copy of the
+oracle's C source, build it, and require that at least one pin fails.
+
+The mistakes are planted only in a temporary copy of the oracle, on the CPU.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle import build as obuild
+import pins
+
+MUTANTS = [
+    ("phi without the +1", "return x > 0.0 ? x + 1.0 : exp(x);", "return x > 0.0 ? x : exp(x);"),
+    ("phi with exp(-x)", "return x > 0.0 ? x + 1.0 : exp(x);", "return x > 0.0 ? x + 1.0 : exp(-x);"),
+    ("exclusive causal sum", "causal ? i + 1 : n", "causal ? i : n"),
+    ("eps dropped", "(den + eps)", "(den)"),
+    ("eps dropped (recurrent)", "double den = eps;", "double den = 0.0;"),
+    ("GQA head mapping h % Hkv", "const int g = h / G;", "const int g = h % Hkv;"),
+    ("normaliser accumulates phi(k)^2", "z[a] += pk[a];", "z[a] += pk[a] * pk[a];"),
+    ("bf16 widened with wrong shift", "<< 16;", "<< 15;"),
+    ("non-causal state never filled", "if (!causal) {", "if (0) {"),
+    ("packed sequences lose their last token", "*len = (int64_t)cu[s + 1] - cu[s];",
+     "*len = (int64_t)cu[s + 1] - cu[s] - (cu[s + 1] > cu[s]);"),
+    ("decode reads state before update", "zg[a] += pk;", "zg[a] += 0.0 * pk;"),
+    ("numerator sums V of the query row", "num[c] += a * load_elem(v, off(t0 + j,",
+     "num[c] += a * load_elem(v, off(t0 + i,"),
+]
+
+
+def _build_mutant(tmp_path, idx, old, new):
+    with open(obuild.SRC) as f:
+        src = f.read()
+    assert old in src, "mutation target not found: %r" % old
+    src = src.replace(old, new)
+    c = tmp_path / ("mutant%d.c" % idx)
+    so = tmp_path / ("mutant%d.so" % idx)
+    c.write_text(src)
+    subprocess.run(["gcc", "-std=c11", "-O1", "-fopenmp", "-fPIC", "-shared", "-o", str(so),
+                    str(c), "-lm"], check=True)
+    return str(so)
+
+
+@pytest.mark.parametrize("idx", range(len(MUTANTS)), ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, monkeypatch, idx):
+    name, old, new = MUTANTS[idx]
+    path = _build_mutant(tmp_path, idx, old, new)
+    monkeypatch.setattr(oracle, "_lib", None)
+    monkeypatch.setattr(obuild, "build", lambda force=False: path)
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin()
+        except AssertionError:
+            failed.append(pin.__name__)
+    monkeypatch.setattr(oracle, "_lib", None)
+    assert failed, "no pin caught the planted mistake: %s" % name
