@@ -1,0 +1,144 @@
+"""ctypes binding of liblt.so (the C ABI in include/lt_linear_attn.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch supplies device memory and the current stream.  Importing
+this module loads the library; a missing library is an error (there is no
+fallback path).
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblt.so")
+
+LT_OK, LT_ERR_INVALID_ARG, LT_ERR_UNSUPPORTED, LT_ERR_CUDA = 0, 1, 2, 3
+LT_ERR_DEVICE_TIMEOUT, LT_ERR_DEVICE_BAD_SEQLENS = 4, 5
+LT_F32, LT_BF16 = 0, 1
+
+# every entry point declared in include/lt_linear_attn.h
+EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_decode_step", "lt_status_string",
+            "lt_get_last_device_error", "lt_abi_version")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("liblt.so is not built (run `python -m "
+                      "causal_linear_attention_chunked_b200.build`)")
+lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+lib.lt_linear_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _vp,
+                                   _i]
+lib.lt_linear_attn_fwd.restype = _i
+lib.lt_linear_attn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f,
+                                           _vp, _i]
+lib.lt_linear_attn_decode_step.restype = _i
+lib.lt_status_string.argtypes = [_i]
+lib.lt_status_string.restype = ctypes.c_char_p
+lib.lt_get_last_device_error.argtypes = [_vp]
+lib.lt_get_last_device_error.restype = _i
+lib.lt_abi_version.restype = _i
+
+
+class LtError(RuntimeError):
+    def __init__(self, status):
+        self.status = status
+        super().__init__(lib.lt_status_string(status).decode())
+
+
+def _check(status):
+    if status != LT_OK:
+        raise LtError(status)
+
+
+def _dtype_code(t):
+    if t == torch.bfloat16:
+        return LT_BF16
+    if t == torch.float32:
+        return LT_F32
+    raise TypeError("unsupported dtype %s (bfloat16 or float32)" % t)
+
+
+def _stream_handle(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def linear_attn_fwd(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, out=None, stream=None):
+    """O = linear attention of (q, k, v); see include/lt_linear_attn.h.
+
+    Dense: q [B, N, H_q, d], k [B, N, H_kv, d], v [B, N, H_kv, dv].
+    Packed: q [N, H_q, d] ... with cu_seqlens (int32, device, B+1 entries).
+    Returns out with q's dtype, shape [..., H_q, dv].
+    """
+    if cu_seqlens is None:
+        B, N, Hq, d = q.shape
+        Hkv, dv = k.shape[2], v.shape[3]
+        oshape = (B, N, Hq, dv)
+    else:
+        N, Hq, d = q.shape
+        Hkv, dv = k.shape[1], v.shape[2]
+        B = cu_seqlens.numel() - 1
+        oshape = (N, Hq, dv)
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
+            raise TypeError("cu_seqlens must be a contiguous int32 tensor")
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+    if out is None:
+        out = torch.empty(oshape, dtype=q.dtype, device=q.device)
+    _check(lib.lt_linear_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, Hq, Hkv, N, d, dv,
+                                  int(bool(causal)), float(eps), _ptr(cu_seqlens),
+                                  _stream_handle(stream, q.device), _dtype_code(q.dtype)))
+    return out
+
+
+def linear_attn_decode_step(q, k, v, S, z, eps=1e-6, out=None, stream=None):
+    """One recurrent step; S [B, H_kv, d, dv] and z [B, H_kv, d] (fp32) are
+    updated in place.  q [B, H_q, d], k [B, H_kv, d], v [B, H_kv, dv]."""
+    B, Hq, d = q.shape
+    Hkv, dv = k.shape[1], v.shape[2]
+    for t in (q, k, v, S, z):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    if S.dtype != torch.float32 or z.dtype != torch.float32:
+        raise TypeError("S and z must be float32")
+    if out is None:
+        out = torch.empty((B, Hq, dv), dtype=q.dtype, device=q.device)
+    _check(lib.lt_linear_attn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(S), _ptr(z), _ptr(out),
+                                          B, Hq, Hkv, d, dv, float(eps),
+                                          _stream_handle(stream, q.device),
+                                          _dtype_code(q.dtype)))
+    return out
+
+
+def get_last_device_error(stream=None):
+    """Synchronise the stream; return the device error status and clear it."""
+    dev = torch.cuda.current_device()
+    return lib.lt_get_last_device_error(_stream_handle(stream, dev))
+
+
+def linear_attn_fwd_host(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, device="cuda",
+                         stream=None, out_host=None):
+    """End-to-end call on HOST tensors: copy the inputs (pinned host memory
+    recommended) to the device, run the forward pass, copy the result back.
+    All copies and the kernel are enqueued on one stream; returns the host
+    output once it has arrived."""
+    dev = torch.device(device)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    with torch.cuda.stream(s):
+        qd = q.to(dev, non_blocking=True)
+        kd = k.to(dev, non_blocking=True)
+        vd = v.to(dev, non_blocking=True)
+        cud = cu_seqlens.to(dev, non_blocking=True) if cu_seqlens is not None else None
+        od = linear_attn_fwd(qd, kd, vd, causal=causal, eps=eps, cu_seqlens=cud, stream=s)
+        if out_host is None:
+            out_host = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
+        out_host.copy_(od, non_blocking=True)
+    s.synchronize()
+    return out_host

@@ -1,0 +1,722 @@
+// fwd_bf16_sm100.cu -- chunked kernelised linear attention, bf16 I/O with
+// fp32 accumulation, on the sm_100a tensor cores (tcgen05 + TMA + TMEM).
+//
+// Method (lineartile 1.0.0, "How It Works" and "Reference" sections; the
+// causal form is the linear attention of Katharopoulos et al. 2020):
+//     O_i = phi(Q_i) S_i / (phi(Q_i) . z_i + eps),
+//     S_i = sum_{j<=i} phi(K_j)^T V_j,  z_i = sum_{j<=i} phi(K_j),
+//     phi(x) = ELU(x) + 1.
+// Chunked evaluation ("Why Stream Wins at Ultra-Long Context", section 5.3:
+// chunk-local work plus an inter-chunk carry): for a chunk c of C tokens,
+//     num_c = mask(phi(Q_c) phi(K_c)^T) V_c + phi(Q_c) S_<c
+//     den_c = mask(phi(Q_c) phi(K_c)^T) 1   + phi(Q_c) z_<c
+//     [S|z]_<c+1 = [S|z]_<c + phi(K_c)^T [V_c | 1].
+// The three products are dense contractions and run on the tensor cores.
+// The carried state [S|z] lives in TMEM as an fp32 accumulator; each chunk
+// it is read once, rounded to bf16 and staged in shared memory as the B
+// operand of phi(Q_c) [S|z]_<c.
+//
+// One CTA owns one (sequence, KV head) pair and walks its chunks in order;
+// every query head of the KV head's group is served from the same K/V tiles
+// and the same state.  Warp roles (320 threads):
+//   warps 0-3  transform warpgroup: phi applied in place to the TMA-loaded
+//              K and Q tiles, tail rows zeroed; causal mask of the score
+//              tile, conversion to bf16, staging as the A operand of P V.
+//   warps 4-7  state/epilogue warpgroup: TMEM state -> bf16 operand;
+//              TMEM accumulator -> normalised bf16 rows -> global memory.
+//   warp 8     TMA producer.
+//   warp 9     TMEM allocator and single-thread MMA issuer.
+// Non-causal mode (phi(Q)(phi(K)^T V) normalised the same way): first the
+// state over all chunks (K, V only), then every output row as
+// phi(Q_i) [S|z]_n (Q only).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lt_internal.h"
+#include "lt_ptx.cuh"
+
+namespace lt {
+namespace {
+
+constexpr int kChunk = 128;          // tokens per chunk (MMA M for the row tiles)
+constexpr int kRowBytes = 128;       // one swizzle atom row: 64 bf16
+constexpr int kBox = kChunk * kRowBytes;  // one 64-column box of a chunk tile
+constexpr int kThreads = 320;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+
+template <int D, int DV>
+struct Cfg {
+  static constexpr int QT = kChunk * D * 2;
+  static constexpr int KT = kChunk * D * 2;
+  static constexpr int VT = kChunk * DV * 2;
+  static constexpr int PBT = kChunk * kChunk * 2;
+  static constexpr int SOPT = (DV / 64 + 1) * D * kRowBytes;  // [S | z 0..] operand
+  static constexpr int ONEST = kChunk * kRowBytes;
+  static constexpr bool kBig = (D == 128);
+  static constexpr int NQ = (D == 64 && DV == 64) ? 3 : 2;
+  static constexpr int NKV = (D == 128) ? 1 : 2;
+  static constexpr int NPB = (DV == 128) ? 1 : 2;
+  static constexpr int NSOP = (D == 128) ? 1 : 2;
+  static constexpr int ACCW = DV + 16;  // numerator columns + normaliser block
+  static constexpr int NP = (D == 64 && DV == 128) ? 1 : (DV == 64 ? 2 : 1);
+  static constexpr int NA = (DV == 64) ? 2 : 1;
+  static constexpr int TM_P = 0;
+  static constexpr int TM_ACC = NP * kChunk;
+  static constexpr int TM_S = TM_ACC + NA * ACCW;
+  static constexpr int TM_COLS = 512;
+  static_assert(TM_S + ACCW <= TM_COLS, "TMEM budget");
+  // shared memory layout (all tiles 1024-byte aligned)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + NQ * QT;
+  static constexpr int OFF_V = OFF_K + NKV * KT;
+  static constexpr int OFF_PB = OFF_V + NKV * VT;
+  static constexpr int OFF_SOP = OFF_PB + NPB * PBT;
+  static constexpr int OFF_ONES = OFF_SOP + NSOP * SOPT;
+  static constexpr int OFF_BAR = OFF_ONES + ONEST;
+  static constexpr int NBARS = 4 * NQ + 3 * NKV + 2 * NP + 2 * NPB + 2 * NSOP + 2 + 2 * NA + 1;
+  static constexpr int SMEM = OFF_BAR + NBARS * 8 + 16 + 1024;  // + tmem slot + align slack
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+struct Bars {
+  uint64_t *q_full, *q_empty, *q_xf, *q_spare;
+  uint64_t *kv_full, *kv_empty, *kv_xf;
+  uint64_t *p_full, *p_empty;
+  uint64_t *pb_full, *pb_empty;
+  uint64_t *sop_full, *sop_empty;
+  uint64_t *s_full, *s_empty;
+  uint64_t *acc_full, *acc_empty;
+  uint64_t *drain;
+};
+
+template <int D, int DV>
+__device__ __forceinline__ Bars carve_bars(uint8_t* base) {
+  using K = Cfg<D, DV>;
+  uint64_t* b = reinterpret_cast<uint64_t*>(base);
+  Bars r;
+  r.q_full = b; b += K::NQ;
+  r.q_empty = b; b += K::NQ;
+  r.q_xf = b; b += K::NQ;
+  r.q_spare = b; b += K::NQ;
+  r.kv_full = b; b += K::NKV;
+  r.kv_empty = b; b += K::NKV;
+  r.kv_xf = b; b += K::NKV;
+  r.p_full = b; b += K::NP;
+  r.p_empty = b; b += K::NP;
+  r.pb_full = b; b += K::NPB;
+  r.pb_empty = b; b += K::NPB;
+  r.sop_full = b; b += K::NSOP;
+  r.sop_empty = b; b += K::NSOP;
+  r.s_full = b; b += 1;
+  r.s_empty = b; b += 1;
+  r.acc_full = b; b += K::NA;
+  r.acc_empty = b; b += K::NA;
+  r.drain = b; b += 1;
+  return r;
+}
+
+// phi in place over a [kChunk x (NBOX*64)] bf16 tile (rows of 128-byte
+// boxes, swizzled; phi is elementwise so the swizzle does not matter).
+// Rows >= valid are zeroed.  128 threads.
+template <int NBOX>
+__device__ __forceinline__ void xf_tile(uint8_t* tile, int valid, bool apply_phi, int tid) {
+  constexpr int kChunks = kChunk * NBOX * 8;  // 16-byte pieces
+#pragma unroll 4
+  for (int ch = tid; ch < kChunks; ch += 128) {
+    const int rem = ch % (kChunk * 8);
+    const int row = rem >> 3;
+    uint4* p = reinterpret_cast<uint4*>(tile + (ch / (kChunk * 8)) * kBox + rem * 16);
+    uint4 v = *p;
+    if (row >= valid) {
+      v = make_uint4(0u, 0u, 0u, 0u);
+    } else if (apply_phi) {
+      uint32_t* u = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = unpack_bf16x2(u[e]);
+        u[e] = pack_bf16x2(phi_f(f.x), phi_f(f.y));
+      }
+    } else {
+      continue;
+    }
+    *p = v;
+  }
+}
+
+// Byte offset of the 16-byte piece holding columns [8*jj, 8*jj+8) of row
+// `row` inside a 128-byte-swizzled 64-column box (1024-byte aligned).
+__device__ __forceinline__ uint32_t sw128_off(int row, int jj) {
+  return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((jj ^ (row & 7)) << 4));
+}
+
+struct FwdArgs {
+  __nv_bfloat16* out;
+  const int32_t* cu_seqlens;
+  int B, Hq, Hkv, N, G, causal;
+  float eps;
+  int total_tokens;
+  int* err;
+};
+
+template <int D, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+    lt_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+  using K = Cfg<D, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ volatile int s_abort;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int g = blockIdx.x;  // KV head
+  const int s = blockIdx.y;  // sequence (batch row or packed sequence)
+
+  // sequence geometry
+  int t0, n;
+  if (a.cu_seqlens) {
+    const int lo = a.cu_seqlens[s], hi = a.cu_seqlens[s + 1];
+    if (lo < 0 || hi < lo || hi > a.total_tokens) {
+      if (tid == 0) report_error(a.err, kDevErrBadSeqlens);
+      return;
+    }
+    t0 = lo;
+    n = hi - lo;
+  } else {
+    t0 = s * a.N;
+    n = a.N;
+  }
+  if (n <= 0) return;
+  const int nc = (n + kChunk - 1) / kChunk;
+  const int G = a.G;
+  const int n_items = nc * G;
+
+  uint8_t* sQ = smem + K::OFF_Q;
+  uint8_t* sK = smem + K::OFF_K;
+  uint8_t* sV = smem + K::OFF_V;
+  uint8_t* sPB = smem + K::OFF_PB;
+  uint8_t* sSOP = smem + K::OFF_SOP;
+  uint8_t* sONES = smem + K::OFF_ONES;
+  Bars bars = carve_bars<D, DV>(smem + K::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + K::OFF_BAR + K::NBARS * 8);
+
+  if (tid == 0) {
+    s_abort = 0;
+    for (int i = 0; i < K::NQ; ++i) {
+      mbar_init(&bars.q_full[i], 1);
+      mbar_init(&bars.q_empty[i], 1);
+      mbar_init(&bars.q_xf[i], 1);
+      mbar_init(&bars.q_spare[i], 1);
+    }
+    for (int i = 0; i < K::NKV; ++i) {
+      mbar_init(&bars.kv_full[i], 1);
+      mbar_init(&bars.kv_empty[i], 1);
+      mbar_init(&bars.kv_xf[i], 1);
+    }
+    for (int i = 0; i < K::NP; ++i) {
+      mbar_init(&bars.p_full[i], 1);
+      mbar_init(&bars.p_empty[i], 1);
+    }
+    for (int i = 0; i < K::NPB; ++i) {
+      mbar_init(&bars.pb_full[i], 1);
+      mbar_init(&bars.pb_empty[i], 1);
+    }
+    for (int i = 0; i < K::NSOP; ++i) {
+      mbar_init(&bars.sop_full[i], 1);
+      mbar_init(&bars.sop_empty[i], 1);
+    }
+    mbar_init(bars.s_full, 1);
+    mbar_init(bars.s_empty, 1);
+    for (int i = 0; i < K::NA; ++i) {
+      mbar_init(&bars.acc_full[i], 1);
+      mbar_init(&bars.acc_empty[i], 1);
+    }
+    mbar_init(bars.drain, 1);
+    fence_mbar_init();
+  }
+  // The [1 | 0 ... 0] block: the extra B operand whose products give the
+  // normaliser (phi(K)^T 1 and the row sums of the masked scores).  Row r
+  // holds bf16 1.0 in logical column 0, zeros elsewhere (128-byte swizzle).
+  for (int ch = tid; ch < kChunk * 8; ch += kThreads) {
+    const int row = ch >> 3, phys = ch & 7;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (phys == (row & 7)) v.x = 0x3F80u;  // logical piece 0 lands at (0 ^ row%8)
+    *reinterpret_cast<uint4*>(sONES + row * kRowBytes + phys * 16) = v;
+  }
+  fence_proxy_async_smem();
+  if (warp == 9) tmem_alloc(tmem_slot, K::TM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* abort_flag = &s_abort;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      int q_issued = 0, kv_issued = 0;
+      bool ok = true;
+      auto load_kv = [&](int c) -> bool {
+        const int st = c % K::NKV;
+        if (!mbar_wait(&bars.kv_empty[st], ((c / K::NKV) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+          return false;
+        mbar_arrive_expect_tx(&bars.kv_full[st], K::KT + K::VT);
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_3d(sK + st * K::KT + bx * kBox, &tm_k, &bars.kv_full[st], bx * 64, g,
+                      t0 + c * kChunk);
+        for (int bx = 0; bx < DV / 64; ++bx)
+          tma_load_3d(sV + st * K::VT + bx * kBox, &tm_v, &bars.kv_full[st], bx * 64, g,
+                      t0 + c * kChunk);
+        ++kv_issued;
+        return true;
+      };
+      auto load_q = [&](int i) -> bool {
+        const int st = i % K::NQ;
+        const int c = i / G, h = i % G;
+        if (!mbar_wait(&bars.q_empty[st], ((i / K::NQ) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+          return false;
+        mbar_arrive_expect_tx(&bars.q_full[st], K::QT);
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_3d(sQ + st * K::QT + bx * kBox, &tm_q, &bars.q_full[st], bx * 64,
+                      g * G + h, t0 + c * kChunk);
+        ++q_issued;
+        return true;
+      };
+      if (a.causal) {
+        for (int i = 0; i < n_items && ok; ++i) {
+          if (i % G == 0) ok = load_kv(i / G);
+          if (ok) ok = load_q(i);
+        }
+      } else {
+        for (int c = 0; c < nc && ok; ++c) ok = load_kv(c);
+        for (int i = 0; i < n_items && ok; ++i) ok = load_q(i);
+      }
+      if (!ok) {
+        // drain: wait (bounded, ignoring the abort flag) for copies in flight
+        int dummy = 0;
+        for (int c = (kv_issued > K::NKV ? kv_issued - K::NKV : 0); c < kv_issued; ++c)
+          mbar_wait(&bars.kv_full[c % K::NKV], (c / K::NKV) & 1, &dummy, nullptr, kWaitLimitNs);
+        for (int i = (q_issued > K::NQ ? q_issued - K::NQ : 0); i < q_issued; ++i)
+          mbar_wait(&bars.q_full[i % K::NQ], (i / K::NQ) & 1, &dummy, nullptr, kWaitLimitNs);
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_P = idesc_bf16_f32(kChunk, kChunk, 0, 0);
+      constexpr uint32_t ID_SV = idesc_bf16_f32(D, DV, 1, 1);
+      constexpr uint32_t ID_S1 = idesc_bf16_f32(D, 16, 1, 1);
+      constexpr uint32_t ID_PV = idesc_bf16_f32(kChunk, DV, 0, 1);
+      constexpr uint32_t ID_P1 = idesc_bf16_f32(kChunk, 16, 0, 1);
+      constexpr uint32_t ID_QS = idesc_bf16_f32(kChunk, DV + 16, 0, 1);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      const uint32_t sPBa = smem_u32(sPB), sSOPa = smem_u32(sSOP), sONESa = smem_u32(sONES);
+      const uint32_t t_s = tmem + K::TM_S;
+      bool ok = true;
+
+      // S_acc (+)= phi(K_c)^T [V_c | 1]
+      auto issue_state = [&](int c, bool accumulate) {
+        const int st = c % K::NKV;
+        const uint32_t kb = sKa + st * K::KT, vb = sVa + st * K::VT;
+        for (int kk = 0; kk < kChunk / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(kb + kk * 2048, kBox, 1024);
+          umma_f16_ss(t_s, ad, smem_desc_sw128(vb + kk * 2048, kBox, 1024), ID_SV,
+                      (accumulate || kk > 0) ? 1u : 0u);
+          umma_f16_ss(t_s + DV, ad, smem_desc_sw128(sONESa + kk * 2048, kBox, 1024), ID_S1,
+                      (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      // Acc (+)= phi(Q) [S|z]  (B operand staged by the state warpgroup)
+      auto issue_qs = [&](uint32_t t_acc, uint32_t qb, uint32_t sopb, bool accumulate) {
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(qb + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sopb + kk * 2048, D * kRowBytes, 1024);
+          umma_f16_ss(t_acc, ad, bd, ID_QS, (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      if (a.causal) {
+        auto issue_acc = [&](int j) -> bool {
+          const int c = j / G, h = j % G;
+          const int pbs = j % K::NPB, as = j % K::NA, qs = j % K::NQ;
+          if (!mbar_wait(&bars.pb_full[pbs], (j / K::NPB) & 1, abort_flag, a.err, kWaitLimitNs))
+            return false;
+          if (h == 0 && !mbar_wait(&bars.sop_full[c % K::NSOP], (c / K::NSOP) & 1, abort_flag,
+                                   a.err, kWaitLimitNs))
+            return false;
+          if (!mbar_wait(&bars.acc_empty[as], ((j / K::NA) & 1) ^ 1, abort_flag, a.err,
+                         kWaitLimitNs))
+            return false;
+          tc_fence_after();
+          const uint32_t t_acc = tmem + K::TM_ACC + as * K::ACCW;
+          const uint32_t pb = sPBa + pbs * K::PBT;
+          const uint32_t vb = sVa + (c % K::NKV) * K::VT;
+          for (int kk = 0; kk < kChunk / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(pb + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024);
+            umma_f16_ss(t_acc, ad, smem_desc_sw128(vb + kk * 2048, kBox, 1024), ID_PV,
+                        kk > 0 ? 1u : 0u);
+            umma_f16_ss(t_acc + DV, ad, smem_desc_sw128(sONESa + kk * 2048, kBox, 1024), ID_P1,
+                        kk > 0 ? 1u : 0u);
+          }
+          issue_qs(t_acc, sQa + qs * K::QT, sSOPa + (c % K::NSOP) * K::SOPT, true);
+          umma_commit(&bars.acc_full[as]);
+          umma_commit(&bars.pb_empty[pbs]);
+          umma_commit(&bars.q_empty[qs]);
+          if (h == G - 1) {
+            umma_commit(&bars.kv_empty[c % K::NKV]);
+            umma_commit(&bars.sop_empty[c % K::NSOP]);
+          }
+          return true;
+        };
+        for (int i = 0; i < n_items && ok; ++i) {
+          const int c = i / G;
+          // single K/V stage: the previous chunk's last accumulator MMA must
+          // be issued (it releases the stage) before waiting for new tiles
+          const bool flush_first = (K::NKV == 1) && (i % G == 0) && i > 0;
+          if (flush_first) {
+            ok = issue_acc(i - 1);
+            if (!ok) break;
+          }
+          if (i % G == 0) {
+            const int st = c % K::NKV;
+            ok = mbar_wait(&bars.kv_xf[st], (c / K::NKV) & 1, abort_flag, a.err, kWaitLimitNs) &&
+                 mbar_wait(bars.s_empty, c & 1, abort_flag, a.err, kWaitLimitNs);
+            if (!ok) break;
+            tc_fence_after();
+            issue_state(c, c > 0);
+            umma_commit(bars.s_full);
+          }
+          const int qs = i % K::NQ, ps = i % K::NP;
+          ok = mbar_wait(&bars.q_xf[qs], (i / K::NQ) & 1, abort_flag, a.err, kWaitLimitNs) &&
+               mbar_wait(&bars.p_empty[ps], ((i / K::NP) & 1) ^ 1, abort_flag, a.err,
+                         kWaitLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+          {
+            const uint32_t t_p = tmem + K::TM_P + ps * kChunk;
+            const uint32_t qb = sQa + qs * K::QT, kb = sKa + (c % K::NKV) * K::KT;
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t o = (kk >> 2) * kBox + (kk & 3) * 32;
+              umma_f16_ss(t_p, smem_desc_sw128(qb + o, 16, 1024),
+                          smem_desc_sw128(kb + o, 16, 1024), ID_P, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars.p_full[ps]);
+          }
+          if (i > 0 && !flush_first) ok = issue_acc(i - 1);
+        }
+        if (ok && n_items > 0) ok = issue_acc(n_items - 1);
+      } else {
+        for (int c = 0; c < nc && ok; ++c) {
+          const int st = c % K::NKV;
+          ok = mbar_wait(&bars.kv_xf[st], (c / K::NKV) & 1, abort_flag, a.err, kWaitLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+          issue_state(c, c > 0);
+          umma_commit(&bars.kv_empty[st]);
+        }
+        if (ok) umma_commit(bars.s_full);
+        if (ok) ok = mbar_wait(&bars.sop_full[0], 0, abort_flag, a.err, kWaitLimitNs);
+        for (int i = 0; i < n_items && ok; ++i) {
+          const int qs = i % K::NQ, as = i % K::NA;
+          ok = mbar_wait(&bars.q_xf[qs], (i / K::NQ) & 1, abort_flag, a.err, kWaitLimitNs) &&
+               mbar_wait(&bars.acc_empty[as], ((i / K::NA) & 1) ^ 1, abort_flag, a.err,
+                         kWaitLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qs(tmem + K::TM_ACC + as * K::ACCW, sQa + qs * K::QT, sSOPa, false);
+          umma_commit(&bars.acc_full[as]);
+          umma_commit(&bars.q_empty[qs]);
+        }
+      }
+      // drain the tensor pipe before TMEM is released
+      umma_commit(bars.drain);
+      int dummy = 0;
+      mbar_wait(bars.drain, 0, &dummy, nullptr, kWaitLimitNs);
+    }
+  } else if (warp < 4) {
+    // ----------------------------------------------- transform warpgroup
+    const int x = tid;  // 0..127 == TMEM lane == chunk row
+    bool ok = true;
+    auto xf_kv = [&](int c) -> bool {
+      const int st = c % K::NKV;
+      if (!mbar_wait(&bars.kv_full[st], (c / K::NKV) & 1, abort_flag, a.err, kWaitLimitNs))
+        return false;
+      const int valid = min(kChunk, n - c * kChunk);
+      xf_tile<D / 64>(sK + st * K::KT, valid, true, x);
+      if (valid < kChunk) xf_tile<DV / 64>(sV + st * K::VT, valid, false, x);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (x == 0) mbar_arrive(&bars.kv_xf[st]);
+      return true;
+    };
+    auto xf_q = [&](int i) -> bool {
+      const int st = i % K::NQ;
+      if (!mbar_wait(&bars.q_full[st], (i / K::NQ) & 1, abort_flag, a.err, kWaitLimitNs))
+        return false;
+      xf_tile<D / 64>(sQ + st * K::QT, kChunk, true, x);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (x == 0) mbar_arrive(&bars.q_xf[st]);
+      return true;
+    };
+    // mask + convert the score tile of item j into the bf16 A operand
+    auto mask_p = [&](int j) -> bool {
+      const int ps = j % K::NP, pbs = j % K::NPB;
+      if (!mbar_wait(&bars.p_full[ps], (j / K::NP) & 1, abort_flag, a.err, kWaitLimitNs))
+        return false;
+      if (!mbar_wait(&bars.pb_empty[pbs], ((j / K::NPB) & 1) ^ 1, abort_flag, a.err,
+                     kWaitLimitNs))
+        return false;
+      tc_fence_after();
+      const uint32_t t_p = tmem + K::TM_P + ps * kChunk + ((uint32_t)(warp * 32) << 16);
+      uint8_t* pb = sPB + pbs * K::PBT;
+      const int row = x;
+#pragma unroll 1
+      for (int b = 0; b < kChunk / 32; ++b) {
+        uint4 w[4];
+        if (b <= warp) {  // warp-uniform: blocks right of the diagonal are all zero
+          float r[32];
+          tmem_ld32(t_p + b * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (b * 32 + e > row) r[e] = 0.0f;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            w[q4] = make_uint4(pack_bf16x2(r[q4 * 8 + 0], r[q4 * 8 + 1]),
+                               pack_bf16x2(r[q4 * 8 + 2], r[q4 * 8 + 3]),
+                               pack_bf16x2(r[q4 * 8 + 4], r[q4 * 8 + 5]),
+                               pack_bf16x2(r[q4 * 8 + 6], r[q4 * 8 + 7]));
+        } else {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) w[q4] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        const int kb = b >> 1;  // 64-key block
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int jj = (b & 1) * 4 + q4;
+          *reinterpret_cast<uint4*>(pb + kb * kBox + sw128_off(row, jj)) = w[q4];
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (x == 0) {
+        mbar_arrive(&bars.p_empty[ps]);
+        mbar_arrive(&bars.pb_full[pbs]);
+      }
+      return true;
+    };
+    if (a.causal) {
+      for (int i = 0; i < n_items && ok; ++i) {
+        // With a single K/V stage the next chunk's tiles arrive only after
+        // the previous chunk's last score tile has been consumed.
+        const bool flush_first = (K::NKV == 1) && (i % G == 0) && i > 0;
+        if (flush_first) ok = mask_p(i - 1);
+        if (ok && i % G == 0) ok = xf_kv(i / G);
+        if (ok) ok = xf_q(i);
+        if (ok && i > 0 && !flush_first) ok = mask_p(i - 1);
+      }
+      if (ok && n_items > 0) ok = mask_p(n_items - 1);
+    } else {
+      for (int c = 0; c < nc && ok; ++c) ok = xf_kv(c);
+      for (int i = 0; i < n_items && ok; ++i) ok = xf_q(i);
+    }
+  } else {
+    // ----------------------------------------- state / epilogue warpgroup
+    const int x = tid - 128;          // 0..127
+    const int sp = warp & 3;          // TMEM sub-partition of this warp
+    const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+    bool ok = true;
+    // Stage [S|z] (fp32 TMEM, or zero) as the bf16 MN-major B operand.
+    // For D == 64 the state tile is an M=64 accumulator: rows 16*sp + l
+    // live in lanes l < 16 of sub-partition sp.
+    // use: how many times this Sop buffer was staged before (phase parity)
+    auto stage_state = [&](int buf, int use, bool zero, int s_parity) -> bool {
+      const bool has_row = (D == 128) || (lane < 16);
+      const int row = (D == 128) ? x : (sp * 16 + lane);
+      float r[DV + 16];
+      if (!zero) {
+        if (!mbar_wait(bars.s_full, s_parity, abort_flag, a.err, kWaitLimitNs)) return false;
+        tc_fence_after();
+        const uint32_t t_s = tmem + K::TM_S + lane_base;
+#pragma unroll
+        for (int cb = 0; cb < DV / 32; ++cb) {
+          float t32[32];
+          tmem_ld32(t_s + cb * 32, t32);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[cb * 32 + e] = t32[e];
+        }
+        float t16[16];
+        tmem_ld16(t_s + DV, t16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) r[DV + e] = t16[e];
+        tc_fence_before();
+      } else {
+#pragma unroll
+        for (int e = 0; e < DV + 16; ++e) r[e] = 0.0f;
+      }
+      named_bar_sync(2, 128);
+      if (x == 0) mbar_arrive(bars.s_empty);
+      if (!mbar_wait(&bars.sop_empty[buf], (use & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+        return false;
+      if (has_row) {
+        uint8_t* sop = sSOP + buf * K::SOPT;
+#pragma unroll
+        for (int q8 = 0; q8 < (DV + 16) / 8; ++q8) {
+          const int grp = q8 >> 3, jj = q8 & 7;
+          const uint4 w = make_uint4(pack_bf16x2(r[q8 * 8 + 0], r[q8 * 8 + 1]),
+                                     pack_bf16x2(r[q8 * 8 + 2], r[q8 * 8 + 3]),
+                                     pack_bf16x2(r[q8 * 8 + 4], r[q8 * 8 + 5]),
+                                     pack_bf16x2(r[q8 * 8 + 6], r[q8 * 8 + 7]));
+          *reinterpret_cast<uint4*>(sop + grp * (D * kRowBytes) + sw128_off(row, jj)) = w;
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(2, 128);
+      if (x == 0) mbar_arrive(&bars.sop_full[buf]);
+      return true;
+    };
+    auto epilogue = [&](int j) -> bool {
+      const int c = j / G, h = j % G, as = j % K::NA;
+      if (!mbar_wait(&bars.acc_full[as], (j / K::NA) & 1, abort_flag, a.err, kWaitLimitNs))
+        return false;
+      tc_fence_after();
+      const uint32_t t_acc = tmem + K::TM_ACC + as * K::ACCW + lane_base;
+      float t16[16];
+      tmem_ld16(t_acc + DV, t16);
+      tmem_wait_ld();
+      const float inv = 1.0f / (t16[0] + a.eps);
+      const int valid = min(kChunk, n - c * kChunk);
+      const bool store = x < valid;
+      __nv_bfloat16* orow =
+          a.out + ((size_t)(t0 + c * kChunk + x) * a.Hq + (size_t)(g * G + h)) * DV;
+#pragma unroll 1
+      for (int cb = 0; cb < DV / 32; ++cb) {
+        float r[32];
+        tmem_ld32(t_acc + cb * 32, r);
+        tmem_wait_ld();
+        if (store) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint4 w = make_uint4(pack_bf16x2(r[q4 * 8 + 0] * inv, r[q4 * 8 + 1] * inv),
+                                       pack_bf16x2(r[q4 * 8 + 2] * inv, r[q4 * 8 + 3] * inv),
+                                       pack_bf16x2(r[q4 * 8 + 4] * inv, r[q4 * 8 + 5] * inv),
+                                       pack_bf16x2(r[q4 * 8 + 6] * inv, r[q4 * 8 + 7] * inv));
+            *reinterpret_cast<uint4*>(orow + cb * 32 + q4 * 8) = w;
+          }
+        }
+      }
+      tc_fence_before();
+      named_bar_sync(2, 128);
+      if (x == 0) mbar_arrive(&bars.acc_empty[as]);
+      return true;
+    };
+    if (a.causal) {
+      // [S|z]_<c is staged into buffer c % NSOP.  With two buffers the next
+      // chunk's state is staged before this chunk's epilogues; with one, the
+      // buffer frees only after the chunk's last accumulator MMA, so staging
+      // waits until every earlier epilogue of the chunk has released TMEM.
+      auto stage_next = [&](int c) -> bool {
+        return stage_state((c + 1) % K::NSOP, (c + 1) / K::NSOP, false, c & 1);
+      };
+      ok = stage_state(0, 0, true, 0);
+      for (int c = 0; c < nc && ok; ++c) {
+        const bool early = K::NSOP >= 2;
+        if (early && c + 1 < nc) ok = stage_next(c);
+        for (int h = 0; h < G && ok; ++h) {
+          if (!early && h == G - 1 && c + 1 < nc) ok = stage_next(c);
+          if (ok) ok = epilogue(c * G + h);
+        }
+      }
+    } else {
+      // the state is complete once every chunk has been accumulated
+      ok = stage_state(0, 0, false, 0);
+      for (int i = 0; i < n_items && ok; ++i) ok = epilogue(i);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, K::TM_COLS);
+  }
+}
+
+// ------------------------------------------------------------- host side
+bool make_tmap_3d(CUtensorMap* m, const void* base, int inner, int heads, long long tokens,
+                  int box_inner) {
+  using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static EncodeFn encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return false;
+    encode = reinterpret_cast<EncodeFn>(fn);
+  }
+  const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)heads, (cuuint64_t)tokens};
+  const cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * heads * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)box_inner, 1u, (cuuint32_t)kChunk};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int DV>
+cudaError_t launch_fwd(const FwdLaunch& p, cudaStream_t stream) {
+  using K = Cfg<D, DV>;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
+      !make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64) ||
+      !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64))
+    return cudaErrorInvalidValue;
+  auto kern = lt_fwd_bf16_kernel<D, DV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
+  if (e != cudaSuccess) return e;
+  FwdArgs a;
+  a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
+  a.cu_seqlens = p.cu_seqlens;
+  a.B = p.B;
+  a.Hq = p.Hq;
+  a.Hkv = p.Hkv;
+  a.N = p.N;
+  a.G = p.Hq / p.Hkv;
+  a.causal = p.causal;
+  a.eps = p.eps;
+  a.total_tokens = (int)p.total_tokens;
+  a.err = p.err;
+  dim3 grid(p.Hkv, p.B);
+  kern<<<grid, kThreads, K::SMEM, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_bf16(const FwdLaunch& p, cudaStream_t stream) {
+  if (p.d == 64 && p.dv == 64) return launch_fwd<64, 64>(p, stream);
+  if (p.d == 128 && p.dv == 128) return launch_fwd<128, 128>(p, stream);
+  if (p.d == 64 && p.dv == 128) return launch_fwd<64, 128>(p, stream);
+  if (p.d == 128 && p.dv == 64) return launch_fwd<128, 64>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lt

@@ -1,0 +1,178 @@
+// lt_api.cu -- the C ABI declared in include/lt_linear_attn.h: argument
+// validation on the host, kernel selection, and the per-device error word.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "../../include/lt_linear_attn.h"
+#include "lt_internal.h"
+#include "lt_ptx.cuh"
+
+namespace {
+
+// Kernels record asynchronous errors here (first error wins).
+__device__ int g_device_error;
+
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices];
+std::mutex g_err_mu;
+
+// Device address of the error word on the current device (looked up once
+// per device).
+int* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+bool is_device_ptr(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error state
+    return false;
+  }
+  return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+bool width_ok(int w) { return w == 64 || w == 128; }
+
+}  // namespace
+
+extern "C" {
+
+int lt_abi_version(void) { return 1; }
+
+const char* lt_status_string(lt_status_t s) {
+  switch (s) {
+    case LT_OK: return "LT_OK";
+    case LT_ERR_INVALID_ARG: return "LT_ERR_INVALID_ARG: invalid argument";
+    case LT_ERR_UNSUPPORTED: return "LT_ERR_UNSUPPORTED: unsupported width or dtype";
+    case LT_ERR_CUDA: return "LT_ERR_CUDA: CUDA runtime or launch failure";
+    case LT_ERR_DEVICE_TIMEOUT: return "LT_ERR_DEVICE_TIMEOUT: a kernel gave up a stalled wait";
+    case LT_ERR_DEVICE_BAD_SEQLENS: return "LT_ERR_DEVICE_BAD_SEQLENS: inconsistent cu_seqlens";
+  }
+  return "unknown lt_status_t";
+}
+
+lt_status_t lt_linear_attn_fwd(const void* q, const void* k, const void* v, void* out, int B,
+                               int H_q, int H_kv, int N, int d, int dv, int causal, float eps,
+                               const int32_t* cu_seqlens, lt_stream_t stream,
+                               lt_dtype_t dtype) {
+  if (dtype != LT_F32 && dtype != LT_BF16) return LT_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !out) return LT_ERR_INVALID_ARG;
+  if (B <= 0 || H_q <= 0 || H_kv <= 0 || N <= 0) return LT_ERR_INVALID_ARG;
+  if (H_q % H_kv != 0) return LT_ERR_INVALID_ARG;
+  if (B > 65535) return LT_ERR_INVALID_ARG;  // grid y extent
+  if (causal != 0 && causal != 1) return LT_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !isfinite(eps)) return LT_ERR_INVALID_ARG;
+  if (!width_ok(d) || !width_ok(dv)) return LT_ERR_UNSUPPORTED;
+  const long long tokens = cu_seqlens ? (long long)N : (long long)B * (long long)N;
+  if (tokens >= (1ll << 31)) return LT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return LT_ERR_INVALID_ARG;
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return LT_ERR_INVALID_ARG;
+  if (!is_device_ptr(q) || !is_device_ptr(k) || !is_device_ptr(v) || !is_device_ptr(out) ||
+      (cu_seqlens && !is_device_ptr(cu_seqlens)))
+    return LT_ERR_INVALID_ARG;
+  const size_t es = dtype == LT_BF16 ? 2 : 4;
+  const size_t nq = (size_t)tokens * H_q * d * es, nk = (size_t)tokens * H_kv * d * es;
+  const size_t nv = (size_t)tokens * H_kv * dv * es, no = (size_t)tokens * H_q * dv * es;
+  if (overlaps(out, no, q, nq) || overlaps(out, no, k, nk) || overlaps(out, no, v, nv))
+    return LT_ERR_INVALID_ARG;
+  int* err = device_error_word();
+  if (!err) return LT_ERR_CUDA;
+
+  lt::FwdLaunch p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.out = out;
+  p.cu_seqlens = cu_seqlens;
+  p.B = B;
+  p.Hq = H_q;
+  p.Hkv = H_kv;
+  p.N = N;
+  p.d = d;
+  p.dv = dv;
+  p.causal = causal;
+  p.eps = eps;
+  p.total_tokens = tokens;
+  p.err = err;
+  const cudaError_t e = dtype == LT_BF16 ? lt::launch_fwd_bf16(p, (cudaStream_t)stream)
+                                         : lt::launch_fwd_f32(p, (cudaStream_t)stream);
+  return e == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status_t lt_linear_attn_decode_step(const void* q, const void* k, const void* v, float* S,
+                                       float* z, void* out, int B, int H_q, int H_kv, int d,
+                                       int dv, float eps, lt_stream_t stream,
+                                       lt_dtype_t dtype) {
+  if (dtype != LT_F32 && dtype != LT_BF16) return LT_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !S || !z || !out) return LT_ERR_INVALID_ARG;
+  if (B <= 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return LT_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !isfinite(eps)) return LT_ERR_INVALID_ARG;
+  if (!width_ok(d) || !width_ok(dv)) return LT_ERR_UNSUPPORTED;
+  if (B > 65535) return LT_ERR_INVALID_ARG;
+  if (!aligned16(S) || (reinterpret_cast<uintptr_t>(z) & 3u)) return LT_ERR_INVALID_ARG;
+  if (!is_device_ptr(q) || !is_device_ptr(k) || !is_device_ptr(v) || !is_device_ptr(S) ||
+      !is_device_ptr(z) || !is_device_ptr(out))
+    return LT_ERR_INVALID_ARG;
+  const size_t es = dtype == LT_BF16 ? 2 : 4;
+  const size_t no = (size_t)B * H_q * dv * es;
+  if (overlaps(out, no, q, (size_t)B * H_q * d * es) ||
+      overlaps(out, no, k, (size_t)B * H_kv * d * es) ||
+      overlaps(out, no, v, (size_t)B * H_kv * dv * es) ||
+      overlaps(out, no, S, (size_t)B * H_kv * d * dv * 4) ||
+      overlaps(out, no, z, (size_t)B * H_kv * d * 4) ||
+      overlaps(S, (size_t)B * H_kv * d * dv * 4, z, (size_t)B * H_kv * d * 4))
+    return LT_ERR_INVALID_ARG;
+  lt::DecodeLaunch p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.S = S;
+  p.z = z;
+  p.out = out;
+  p.B = B;
+  p.Hq = H_q;
+  p.Hkv = H_kv;
+  p.d = d;
+  p.dv = dv;
+  p.eps = eps;
+  p.bf16 = dtype == LT_BF16;
+  return lt::launch_decode(p, (cudaStream_t)stream) == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status_t lt_get_last_device_error(lt_stream_t stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return LT_ERR_CUDA;
+  int* err = device_error_word();
+  if (!err) return LT_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpy(&code, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LT_ERR_CUDA;
+  if (code != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return LT_ERR_CUDA;
+  }
+  if (code == lt::kDevErrTimeout) return LT_ERR_DEVICE_TIMEOUT;
+  if (code == lt::kDevErrBadSeqlens) return LT_ERR_DEVICE_BAD_SEQLENS;
+  return code == 0 ? LT_OK : LT_ERR_CUDA;
+}
+
+}  // extern "C"

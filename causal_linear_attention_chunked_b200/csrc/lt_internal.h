@@ -1,0 +1,37 @@
+// lt_internal.h -- launch descriptors shared by the C ABI layer and the
+// kernel translation units (host side only).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lt {
+
+struct FwdLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  const int32_t* cu_seqlens;  // device, B+1 entries, or nullptr (dense)
+  int B, Hq, Hkv, N, d, dv, causal;
+  float eps;
+  long long total_tokens;  // B*N (dense) or N (packed)
+  int* err;                // device error word
+};
+
+struct DecodeLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  float* S;
+  float* z;
+  void* out;
+  int B, Hq, Hkv, d, dv;
+  float eps;
+  int bf16;  // 1: bf16 q/k/v/out, 0: fp32
+};
+
+cudaError_t launch_fwd_bf16(const FwdLaunch& p, cudaStream_t stream);
+cudaError_t launch_fwd_f32(const FwdLaunch& p, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeLaunch& p, cudaStream_t stream);
+
+}  // namespace lt

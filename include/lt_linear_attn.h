@@ -1,0 +1,136 @@
+/*
+ * lt_linear_attn.h -- C ABI of the B200 (sm_100a) kernelised linear
+ * attention library (liblt.so).
+ *
+ * The operation (lineartile 1.0.0, PyPI page, sections "How It Works" and
+ * "Reference"; the causal normalised form is the linear attention of
+ * Katharopoulos et al. 2020 that the page cites):
+ *
+ *     phi(x) = ELU(x) + 1           (alpha = 1: x + 1 for x > 0, e^x else)
+ *     causal:      O_i = phi(Q_i) S_i / (phi(Q_i) . z_i + eps),
+ *                  S_i = sum_{j<=i} phi(K_j)^T V_j,  z_i = sum_{j<=i} phi(K_j)
+ *     non-causal:  the same with S and z summed over the whole sequence,
+ *                  i.e. phi(Q)(phi(K)^T V) ("compute K^T V first")
+ *                  normalised row by row with phi(Q_i) . z + eps.
+ *
+ * No 1/sqrt(d) score scale is applied inside the operation; callers that
+ * want one scale Q (or K) beforehand.  eps is added to the denominator only.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc / cudaMallocAsync
+ *     / managed memory) owned by the caller; the library keeps no reference
+ *     to them after the call returns and allocates nothing.
+ *   - Layouts are token-major and dense (row-major, no padding):
+ *       dense:   q [B][N][H_q][d],  k [B][N][H_kv][d],  v [B][N][H_kv][dv],
+ *                out [B][N][H_q][dv]
+ *       packed:  the same without the B dimension, [N][H][.], where
+ *                N = total tokens = cu_seqlens[B].
+ *   - Grouped-query attention: query head h reads KV head
+ *     floor(h * H_kv / H_q), i.e. contiguous groups of G = H_q / H_kv.
+ *   - Work is enqueued on `stream` and the call returns without waiting
+ *     (asynchronous).  Results are valid once the stream reaches the work.
+ *   - Argument errors are detected on the host before anything is
+ *     enqueued; in that case nothing is written and nothing is launched.
+ *   - Errors found by a kernel (an inconsistent cu_seqlens array, a stalled
+ *     pipeline) are recorded in a per-device error word and reported by
+ *     lt_get_last_device_error().
+ *   - The caller must ensure that output buffers do not overlap inputs.
+ */
+#ifndef LT_LINEAR_ATTN_H
+#define LT_LINEAR_ATTN_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LT_API __attribute__((visibility("default")))
+#else
+#define LT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as the CUDA runtime's cudaStream_t (NULL = legacy default). */
+typedef struct CUstream_st *lt_stream_t;
+
+typedef enum {
+  LT_OK = 0,
+  LT_ERR_INVALID_ARG = 1,     /* null/misaligned/host pointer, bad size or eps */
+  LT_ERR_UNSUPPORTED = 2,     /* d or dv not in {64, 128}, unknown dtype */
+  LT_ERR_CUDA = 3,            /* a CUDA runtime call or launch failed */
+  LT_ERR_DEVICE_TIMEOUT = 4,  /* a kernel gave up on a stalled wait */
+  LT_ERR_DEVICE_BAD_SEQLENS = 5 /* a kernel found cu_seqlens inconsistent */
+} lt_status_t;
+
+typedef enum {
+  LT_F32 = 0,  /* fp32 inputs/outputs, fp32 FMA arithmetic */
+  LT_BF16 = 1  /* bf16 inputs/outputs, tensor cores, fp32 accumulation */
+} lt_dtype_t;
+
+/*
+ * Forward pass of (causal or non-causal) linear attention.
+ *
+ * q, k, v   inputs of element type `dtype`, layouts above; 16-byte aligned.
+ * out       output, same element type, layout [.][N][H_q][dv]; 16-byte
+ *           aligned; must not overlap q, k or v.
+ * B         dense: batch rows; packed: number of sequences.  B >= 1.
+ * H_q, H_kv query and KV heads, H_kv >= 1, H_q a multiple of H_kv.
+ * N         dense: tokens per row; packed: total tokens.  N >= 1 and the
+ *           total token count (B*N dense, N packed) below 2^31.
+ * d, dv     key and value widths, each 64 or 128.
+ * causal    1: prefix sums j <= i (diagonal included); 0: whole sequence.
+ * eps       denominator offset, finite and >= 0 (1e-6 is typical).
+ * cu_seqlens NULL for dense inputs; else a DEVICE int32 array of B+1
+ *           non-decreasing offsets with cu_seqlens[0] = 0 and
+ *           cu_seqlens[B] = N; sequence s is tokens [cu[s], cu[s+1]).
+ *           Empty sequences are allowed.  An inconsistent array is skipped
+ *           by the kernel and reported by lt_get_last_device_error().
+ * stream    CUDA stream to enqueue on.
+ * dtype     LT_BF16 (tensor-core path) or LT_F32 (fp32 FMA path).
+ *
+ * Returns LT_OK when the work was enqueued.
+ */
+LT_API lt_status_t lt_linear_attn_fwd(const void *q, const void *k, const void *v, void *out,
+                               int B, int H_q, int H_kv, int N, int d, int dv, int causal,
+                               float eps, const int32_t *cu_seqlens, lt_stream_t stream,
+                               lt_dtype_t dtype);
+
+/*
+ * One recurrent decode step: the fixed-size state (S, z) plays the role of
+ * a KV cache (lineartile page, "KV Cache Reuse"; recurrent view of the
+ * cited linear attention).  For every batch row b and KV head g:
+ *     S[b][g] += phi(k[b][g])^T v[b][g];   z[b][g] += phi(k[b][g]);
+ * then for every query head h of g's group:
+ *     out[b][h] = phi(q[b][h]) S[b][g] / (phi(q[b][h]) . z[b][g] + eps).
+ * The update comes first, so the new token attends to itself.
+ *
+ * q   [B][H_q][d],  k [B][H_kv][d],  v [B][H_kv][dv]   (element type dtype)
+ * S   [B][H_kv][d][dv] fp32, updated in place (16-byte aligned)
+ * z   [B][H_kv][d]     fp32, updated in place
+ * out [B][H_q][dv]     (element type dtype); must not overlap the inputs.
+ * A zero-initialised (S, z) starts a new sequence; chaining N steps gives
+ * the causal forward pass row by row.
+ */
+LT_API lt_status_t lt_linear_attn_decode_step(const void *q, const void *k, const void *v, float *S,
+                                       float *z, void *out, int B, int H_q, int H_kv, int d,
+                                       int dv, float eps, lt_stream_t stream, lt_dtype_t dtype);
+
+/* Static, human-readable name of a status code. */
+LT_API const char *lt_status_string(lt_status_t status);
+
+/*
+ * Synchronise `stream`, then read and clear the current device's error
+ * word.  Returns LT_OK, LT_ERR_DEVICE_TIMEOUT, LT_ERR_DEVICE_BAD_SEQLENS,
+ * or LT_ERR_CUDA if the synchronisation itself failed.
+ */
+LT_API lt_status_t lt_get_last_device_error(lt_stream_t stream);
+
+/* ABI version of this header: 1. */
+LT_API int lt_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LT_LINEAR_ATTN_H */

@@ -1,0 +1,31 @@
+"""Parity metric shared by the GPU tests.
+
+Row metric (the tolerance reading used throughout): for every output row
+(token, head) take ||O_gpu - O_ref||_inf / ||O_ref||_inf and report the
+maximum over rows.  Elementwise relative error is meaningless for outputs
+near zero (V has mean 0), so each row is measured against its own largest
+entry.  Bars: 1e-4 for fp32 I/O, 2e-2 for bf16 I/O with fp32 accumulation.
+"""
+import numpy as np
+
+TOL_F32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+def row_rel_err(gpu, ref):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    if ref.size == 0:
+        return 0.0
+    g2 = gpu.reshape(-1, gpu.shape[-1])
+    r2 = ref.reshape(-1, ref.shape[-1])
+    assert np.all(np.isfinite(g2)), "non-finite GPU output"
+    den = np.abs(r2).max(axis=1)
+    den = np.maximum(den, 1e-30)
+    return float((np.abs(g2 - r2).max(axis=1) / den).max())
+
+
+def tol_for(dtype):
+    import torch
+    return TOL_F32 if dtype == torch.float32 else TOL_BF16

@@ -1,0 +1,103 @@
+"""The C ABI: the library loads, exports every entry point the header
+declares, and rejects invalid arguments on the host (CPU only: none of these
+calls reaches a CUDA API)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"LT_API\s+[\w\s\*]+?\b(lt_\w+)\s*\(", src)
+    return names
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    assert "lt_linear_attn_fwd" in names and "lt_linear_attn_decode_step" in names
+
+
+def test_library_exports_every_declared_symbol():
+    from causal_linear_attention_chunked_b200 import _binding as b
+    for name in declared_functions():
+        assert hasattr(b.lib, name), name
+    assert set(declared_functions()) == set(b.EXPORTED)
+
+
+def test_abi_version_and_status_strings():
+    from causal_linear_attention_chunked_b200 import _binding as b
+    assert b.lib.lt_abi_version() == 1
+    for code in range(6):
+        assert b.lib.lt_status_string(code).startswith(b"LT_")
+    assert b.lib.lt_status_string(99) == b"unknown lt_status_t"
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every case fails before that
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(q=None), 1),
+    (dict(B=0), 1),
+    (dict(Hq=0), 1),
+    (dict(Hkv=3, Hq=8), 1),
+    (dict(N=0), 1),
+    (dict(causal=2), 1),
+    (dict(eps=-1.0), 1),
+    (dict(eps=float("nan")), 1),
+    (dict(eps=float("inf")), 1),
+    (dict(d=32), 2),
+    (dict(dv=96), 2),
+    (dict(dtype=7), 2),
+    (dict(B=70000), 1),
+    (dict(B=1 << 16, N=1 << 16), 1),
+])
+def test_fwd_rejects_invalid_arguments(case, expect):
+    from causal_linear_attention_chunked_b200 import _binding as b
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, B=1, Hq=8, Hkv=8, N=16, d=64, dv=64, causal=1,
+             eps=1e-6, cu=None, stream=None, dtype=1)
+    a.update(case)
+    st = b.lib.lt_linear_attn_fwd(a["q"], a["k"], a["v"], a["out"], a["B"], a["Hq"], a["Hkv"],
+                                  a["N"], a["d"], a["dv"], a["causal"], a["eps"], a["cu"],
+                                  a["stream"], a["dtype"])
+    assert st == expect
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(S=None), 1),
+    (dict(B=0), 1),
+    (dict(Hkv=3, Hq=8), 1),
+    (dict(eps=-1e-3), 1),
+    (dict(d=48), 2),
+    (dict(dtype=5), 2),
+])
+def test_decode_rejects_invalid_arguments(case, expect):
+    from causal_linear_attention_chunked_b200 import _binding as b
+    a = dict(q=FAKE, k=FAKE, v=FAKE, S=FAKE, z=FAKE, out=FAKE, B=4, Hq=8, Hkv=8, d=64, dv=64,
+             eps=1e-6, stream=None, dtype=1)
+    a.update(case)
+    st = b.lib.lt_linear_attn_decode_step(a["q"], a["k"], a["v"], a["S"], a["z"], a["out"],
+                                          a["B"], a["Hq"], a["Hkv"], a["d"], a["dv"], a["eps"],
+                                          a["stream"], a["dtype"])
+    assert st == expect
+
+
+def test_oracle_and_library_share_no_code():
+    """The oracle sources never include/import the CUDA path and vice versa."""
+    osrc = open(os.path.join(ROOT, "oracle", "lt_oracle.c")).read()
+    assert "#include \"" not in osrc
+    opy = open(os.path.join(ROOT, "oracle", "__init__.py")).read()
+    assert "causal_linear_attention_chunked_b200" not in opy
+    pkg = os.path.join(ROOT, "causal_linear_attention_chunked_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "lt_oracle" not in txt, f

@@ -1,0 +1,134 @@
+"""GPU forward pass against the fp64 oracle, element by element, on seeded
+inputs that span several 128-token chunks and a ragged tail (bf16) or
+several 32-token chunks (fp32).  Every call goes through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import pins
+from parity import row_rel_err, tol_for, TOL_BF16, TOL_F32
+from causal_linear_attention_chunked_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def lt():
+    import causal_linear_attention_chunked_b200 as L
+    return L
+
+
+def run_dense(q, k, v, causal, eps=1e-6):
+    L = lt()
+    out = L.linear_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, eps=eps)
+    torch.cuda.synchronize()
+    assert L.get_last_device_error() == 0
+    return out.float().cpu().numpy()
+
+
+DENSE_CASES = [
+    # (B, Hq, Hkv, N, d, dv, causal)
+    (1, 1, 1, 1, 64, 64, True),
+    (1, 2, 2, 127, 64, 64, True),
+    (2, 2, 2, 128, 64, 64, True),
+    (1, 1, 1, 129, 64, 64, True),
+    (2, 3, 3, 3 * 128 + 5, 64, 64, True),
+    (1, 8, 2, 600, 64, 64, True),
+    (1, 4, 1, 1000, 64, 64, False),
+    (2, 2, 2, 257, 64, 64, False),
+    (1, 4, 4, 300, 128, 128, True),
+    (1, 8, 2, 517, 128, 128, True),
+    (1, 4, 2, 300, 128, 128, False),
+    (1, 2, 2, 300, 64, 128, True),
+    (1, 4, 2, 260, 128, 64, True),
+    (1, 2, 1, 200, 64, 128, False),
+]
+
+
+@pytest.mark.parametrize("case", DENSE_CASES, ids=lambda c: "B%dHq%dHkv%dN%dd%ddv%d%s" % (
+    c[0], c[1], c[2], c[3], c[4], c[5], "c" if c[6] else "nc"))
+def test_bf16_dense_vs_oracle(case):
+    B, Hq, Hkv, N, d, dv, causal = case
+    q, k, v = inputs.make_custom(B, Hq, Hkv, N, d, dv, torch.bfloat16, d ** -0.5, seed=hash(case) % 1000)
+    got = run_dense(q, k, v, causal)
+    ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
+    err = row_rel_err(got, ref)
+    assert err <= TOL_BF16, err
+
+
+@pytest.mark.parametrize("scale", [1.0, 3.0])
+def test_bf16_large_magnitude_inputs(scale):
+    """sigma = 1 and 3: phi underflows for very negative inputs, scores spread."""
+    q, k, v = inputs.make_custom(1, 4, 4, 700, 64, 64, torch.bfloat16, scale, seed=77)
+    for causal in (True, False):
+        got = run_dense(q, k, v, causal)
+        ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
+        assert row_rel_err(got, ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("case", [
+    (1, 1, 1, 256, 64, 64, True),   # the fp32 workload's shape
+    (2, 4, 2, 100, 64, 64, True),
+    (1, 2, 2, 77, 128, 128, False),
+    (1, 2, 1, 65, 64, 128, True),
+])
+def test_f32_vs_oracle(case):
+    B, Hq, Hkv, N, d, dv, causal = case
+    q, k, v = inputs.make_custom(B, Hq, Hkv, N, d, dv, torch.float32, 1.0, seed=N)
+    got = run_dense(q, k, v, causal)
+    ref = oracle.fwd_quadratic(q, k, v, causal=causal, eps=1e-6)
+    assert row_rel_err(got, ref) <= TOL_F32
+
+
+def test_f32_workload_full():
+    w = inputs.WORKLOADS["fp32_b1h1n256d64"]
+    q, k, v, _ = inputs.make(w)
+    got = run_dense(q, k, v, True, w.eps)
+    ref = oracle.fwd_quadratic(q, k, v, causal=True, eps=w.eps)
+    assert row_rel_err(got, ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dd", [(64, 64), (128, 128)])
+def test_hand_example_on_gpu(dtype, dd):
+    """The exact 3-token example of tests/golden/hand_3tok_exact.json."""
+    q, k, v, g = pins.hand_3tok_inputs(d=dd[0], dv=dd[1], dtype=dtype)
+    for causal, key in ((True, "causal_eps0_first3cols"), (False, "noncausal_eps0_first3cols")):
+        got = run_dense(q, k, v, causal, eps=0.0)[0, :, 0]
+        tol = 1e-6 if dtype == torch.float32 else 4e-3
+        assert np.abs(got[:, :3] - np.array(g[key])).max() <= tol
+        assert np.all(got[:, 3:] == 0.0)
+
+
+VARLEN_CASES = [
+    ([1, 127, 128, 129, 300], 2, 2, 64, 64, True),
+    ([0, 5, 0, 260, 1], 4, 2, 64, 64, True),
+    ([200, 0, 131], 4, 4, 64, 64, False),
+    ([130, 7, 257], 8, 2, 128, 128, True),
+    ([64, 300], 2, 1, 128, 128, False),
+]
+
+
+@pytest.mark.parametrize("case", VARLEN_CASES, ids=lambda c: "L%s_Hq%dHkv%d_d%d_%s" % (
+    "-".join(map(str, c[0])), c[1], c[2], c[3], "c" if c[5] else "nc"))
+def test_bf16_packed_vs_oracle(case):
+    lens, Hq, Hkv, d, dv, causal = case
+    w = inputs.Workload("t", len(lens), Hq, Hkv, 0, d, dv, torch.bfloat16, d ** -0.5, causal,
+                        sum(lens))
+    q, k, v, cu = inputs.make(w, lengths=lens)
+    L = lt()
+    out = L.linear_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, eps=1e-6,
+                            cu_seqlens=cu.cuda())
+    assert L.get_last_device_error() == 0
+    ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6, cu_seqlens=cu.numpy())
+    assert row_rel_err(out.float().cpu().numpy(), ref) <= TOL_BF16
+
+
+def test_bf16_deterministic():
+    q, k, v = inputs.make_custom(2, 4, 2, 1111, 64, 64, torch.bfloat16, 0.125, seed=5)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    L = lt()
+    a = L.linear_attn_fwd(q, k, v)
+    b = L.linear_attn_fwd(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
