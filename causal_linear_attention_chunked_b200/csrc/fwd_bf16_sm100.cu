@@ -33,18 +33,17 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "lt_internal.h"
 #include "lt_ptx.cuh"
+#include "fwd_common.cuh"
 
 namespace lt {
 namespace {
 
-constexpr int kChunk = 128;          // tokens per chunk (MMA M for the row tiles)
-constexpr int kRowBytes = 128;       // one swizzle atom row: 64 bf16
-constexpr int kBox = kChunk * kRowBytes;  // one 64-column box of a chunk tile
 constexpr int kThreads = 320;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+using namespace fwd;
 
 template <int D, int DV>
 struct Cfg {
@@ -116,49 +115,6 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
   r.drain = b; b += 1;
   return r;
 }
-
-// phi in place over a [kChunk x (NBOX*64)] bf16 tile (rows of 128-byte
-// boxes, swizzled; phi is elementwise so the swizzle does not matter).
-// Rows >= valid are zeroed.  128 threads.
-template <int NBOX>
-__device__ __forceinline__ void xf_tile(uint8_t* tile, int valid, bool apply_phi, int tid) {
-  constexpr int kChunks = kChunk * NBOX * 8;  // 16-byte pieces
-#pragma unroll 4
-  for (int ch = tid; ch < kChunks; ch += 128) {
-    const int rem = ch % (kChunk * 8);
-    const int row = rem >> 3;
-    uint4* p = reinterpret_cast<uint4*>(tile + (ch / (kChunk * 8)) * kBox + rem * 16);
-    uint4 v = *p;
-    if (row >= valid) {
-      v = make_uint4(0u, 0u, 0u, 0u);
-    } else if (apply_phi) {
-      uint32_t* u = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = unpack_bf16x2(u[e]);
-        u[e] = pack_bf16x2(phi_f(f.x), phi_f(f.y));
-      }
-    } else {
-      continue;
-    }
-    *p = v;
-  }
-}
-
-// Byte offset of the 16-byte piece holding columns [8*jj, 8*jj+8) of row
-// `row` inside a 128-byte-swizzled 64-column box (1024-byte aligned).
-__device__ __forceinline__ uint32_t sw128_off(int row, int jj) {
-  return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((jj ^ (row & 7)) << 4));
-}
-
-struct FwdArgs {
-  __nv_bfloat16* out;
-  const int32_t* cu_seqlens;
-  int B, Hq, Hkv, N, G, causal;
-  float eps;
-  int total_tokens;
-  int* err;
-};
 
 template <int D, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -239,15 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bars.drain, 1);
     fence_mbar_init();
   }
-  // The [1 | 0 ... 0] block: the extra B operand whose products give the
-  // normaliser (phi(K)^T 1 and the row sums of the masked scores).  Row r
-  // holds bf16 1.0 in logical column 0, zeros elsewhere (128-byte swizzle).
-  for (int ch = tid; ch < kChunk * 8; ch += kThreads) {
-    const int row = ch >> 3, phys = ch & 7;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (phys == (row & 7)) v.x = 0x3F80u;  // logical piece 0 lands at (0 ^ row%8)
-    *reinterpret_cast<uint4*>(sONES + row * kRowBytes + phys * 16) = v;
-  }
+  init_ones_block(sONES, tid, kThreads);
   fence_proxy_async_smem();
   if (warp == 9) tmem_alloc(tmem_slot, K::TM_COLS);
   tc_fence_before();
@@ -654,33 +602,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// ------------------------------------------------------------- host side
-bool make_tmap_3d(CUtensorMap* m, const void* base, int inner, int heads, long long tokens,
-                  int box_inner) {
-  using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-  static EncodeFn encode = nullptr;
-  if (!encode) {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !fn)
-      return false;
-    encode = reinterpret_cast<EncodeFn>(fn);
-  }
-  const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)heads, (cuuint64_t)tokens};
-  const cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * heads * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)box_inner, 1u, (cuuint32_t)kChunk};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int DV>
 cudaError_t launch_fwd(const FwdLaunch& p, cudaStream_t stream) {
   using K = Cfg<D, DV>;
@@ -712,6 +633,10 @@ cudaError_t launch_fwd(const FwdLaunch& p, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_fwd_bf16(const FwdLaunch& p, cudaStream_t stream) {
+  // LT_KERNEL=seq selects the sequential kernel for every shape (ablation)
+  const char* force = getenv("LT_KERNEL");
+  const bool seq = force && force[0] == 's' && force[1] == 'e';
+  if (!seq && split_supported(p)) return launch_fwd_bf16_split(p, stream);
   if (p.d == 64 && p.dv == 64) return launch_fwd<64, 64>(p, stream);
   if (p.d == 128 && p.dv == 128) return launch_fwd<128, 128>(p, stream);
   if (p.d == 64 && p.dv == 128) return launch_fwd<64, 128>(p, stream);

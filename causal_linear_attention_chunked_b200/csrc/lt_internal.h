@@ -31,6 +31,10 @@ struct DecodeLaunch {
 };
 
 cudaError_t launch_fwd_bf16(const FwdLaunch& p, cudaStream_t stream);
+// d = dv = 64: sequence split over a thread-block cluster (or one CTA per
+// (sequence, KV head) for packed inputs)
+bool split_supported(const FwdLaunch& p);
+cudaError_t launch_fwd_bf16_split(const FwdLaunch& p, cudaStream_t stream);
 cudaError_t launch_fwd_f32(const FwdLaunch& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeLaunch& p, cudaStream_t stream);
 

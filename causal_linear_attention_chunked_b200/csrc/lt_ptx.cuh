@@ -145,6 +145,19 @@ __device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16.  A is K-major in TMEM:
+// row m in lane m, two consecutive bf16 K elements per 32-bit column (the
+// even element in the low half).
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive (once) on bar when every tcgen05.mma issued so far by this thread
 // has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -169,6 +182,25 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
         "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]),
         "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
       : "r"(taddr));
+}
+
+// 32 lanes x 32 bits, 16 consecutive columns, register -> TMEM.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
@@ -207,6 +239,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The same descriptor with its start address advanced by `bytes` (the
+// start-address field holds addr >> 4 in 14 bits; shared addresses stay
+// below 256 KB, so the add never carries out of the field).
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulator.
 // a_mn / b_mn: 1 when the operand is MN-major, 0 when K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
@@ -230,10 +269,140 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   return __bfloat1622float2(h);
 }
 
+// Feature map on a pair of packed bf16 values:
+//     phi(x) = ELU(x) + 1 = max(x, 0) + exp(min(x, 0))
+// (x > 0: x + e^0 = x + 1; x <= 0: 0 + e^x).  The exponent argument
+// min(x,0)*log2(e) is formed in fp32 and rounded once to bf16 for the
+// packed hardware base-2 exponential (two results per instruction); the sum
+// is rounded to bf16, the precision of the tensor-core operand anyway.
+__device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
+  uint32_t y;
+  asm("{\n\t.reg .b32 zero, neg, pos, t, e;\n\t"
+      ".reg .f32 lo, hi;\n\t"
+      "mov.b32 zero, 0;\n\t"
+      "min.bf16x2 neg, %1, zero;\n\t"
+      "max.bf16x2 pos, %1, zero;\n\t"
+      "shl.b32 lo, neg, 16;\n\t"              // low half -> fp32
+      "and.b32 hi, neg, 0xFFFF0000;\n\t"      // high half -> fp32
+      "mul.f32 lo, lo, 0f3FB8AA3B;\n\t"       // * log2(e)
+      "mul.f32 hi, hi, 0f3FB8AA3B;\n\t"
+      "cvt.rn.bf16x2.f32 t, hi, lo;\n\t"
+      "ex2.approx.ftz.bf16x2 e, t;\n\t"
+      "add.rn.bf16x2 %0, pos, e;\n\t}"
+      : "=r"(y)
+      : "r"(x));
+  return y;
+}
+
 // Feature map of the method: phi(x) = ELU(x) + 1 = x + 1 (x > 0), e^x (x <= 0).
 __device__ __forceinline__ float phi_f(float x) {
   const float e = __expf(fminf(x, 0.0f));
   return x > 0.0f ? x + 1.0f : e;
+}
+
+}  // namespace lt
+
+// ------------------------------------------------------------- clusters
+namespace lt {
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// All threads of all CTAs of the cluster (release/acquire at cluster scope).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_cluster_f4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
+// Asynchronous 16-byte store into the shared memory of a CTA of the
+// cluster; completes 16 transaction bytes on that CTA's mbarrier (both
+// addresses cluster-mapped, same target CTA).
+__device__ __forceinline__ void st_async_f4(uint32_t cluster_addr, float4 v,
+                                            uint32_t cluster_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, "
+      "[%5];" ::"r"(cluster_addr),
+      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(cluster_bar)
+      : "memory");
+}
+
+// Bulk copy (TMA engine) from this CTA's shared memory into the shared
+// memory of a CTA of the cluster, completing `bytes` on that CTA's mbarrier.
+// Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint32_t src_cta,
+                                                     uint32_t bytes, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+      "[%3];" ::"r"(dst_cluster),
+      "r"(src_cta), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_acq_rel_cluster() {
+  asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
+
+// Arrive on an mbarrier of CTA-in-cluster (cluster-mapped address), with
+// release semantics at cluster scope.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait with cluster-scope acquire (see mbar_wait).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort, int* err,
+                                                  uint64_t limit_ns) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        *abort = 1;
+        report_error(err, kDevErrTimeout);
+        return false;
+      }
+    }
+  }
 }
 
 }  // namespace lt

@@ -132,3 +132,52 @@ def test_bf16_deterministic():
     b = L.linear_attn_fwd(q, k, v)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+SPLIT_CASES = [
+    # (B, Hq, Hkv, N, causal)
+    (1, 2, 2, 1000, True),     # 8 chunks, ragged tail
+    (2, 4, 2, 777, True),      # GQA inside the split kernel
+    (1, 1, 1, 2049, False),    # 17 chunks, non-causal
+    (1, 2, 1, 130, True),      # 2 chunks: clusters larger than the chunk count
+    (1, 1, 1, 16 * 128 * 2 + 3, True),  # 33 chunks: inactive last round on most CTAs
+]
+
+
+@pytest.mark.parametrize("n_split", [1, 2, 3, 5, 8, 16])
+@pytest.mark.parametrize("case", SPLIT_CASES, ids=lambda c: "B%dHq%dHkv%dN%d%s" % (
+    c[0], c[1], c[2], c[3], "c" if c[4] else "nc"))
+def test_split_kernel_cluster_sizes(monkeypatch, n_split, case):
+    """d = dv = 64 runs a sequence split over a cluster of n CTAs that
+    exchange their chunk states through distributed shared memory."""
+    monkeypatch.setenv("LT_SPLIT_N", str(n_split))
+    B, Hq, Hkv, N, causal = case
+    q, k, v = inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16, 0.125, seed=N + n_split)
+    got = run_dense(q, k, v, causal)
+    ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
+    assert row_rel_err(got, ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("case", DENSE_CASES[:8], ids=lambda c: "B%dHq%dHkv%dN%d%s" % (
+    c[0], c[1], c[2], c[3], "c" if c[6] else "nc"))
+def test_sequential_kernel_forced(monkeypatch, case):
+    """The sequential kernel (one CTA per (sequence, KV head)) on the d=64
+    shapes the split kernel normally takes."""
+    monkeypatch.setenv("LT_KERNEL", "seq")
+    B, Hq, Hkv, N, d, dv, causal = case
+    q, k, v = inputs.make_custom(B, Hq, Hkv, N, d, dv, torch.bfloat16, d ** -0.5, seed=N)
+    got = run_dense(q, k, v, causal)
+    ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
+    assert row_rel_err(got, ref) <= TOL_BF16
+
+
+def test_split_and_sequential_agree_closely(monkeypatch):
+    """The two kernels differ only in rounding order (state operand, bf16
+    output rounding of each); two independent bf16 roundings of the same
+    value can differ by 2 ulp (0.78% of an entry), so their outputs must
+    agree to 1e-2 in the row metric, well inside the 2e-2 bar."""
+    q, k, v = inputs.make_custom(2, 8, 8, 4096, 64, 64, torch.bfloat16, 0.125, seed=9)
+    a = run_dense(q, k, v, True)
+    monkeypatch.setenv("LT_KERNEL", "seq")
+    b = run_dense(q, k, v, True)
+    assert row_rel_err(a, b) <= 1e-2
