@@ -1,0 +1,805 @@
+// fwd_bf16_block_sm100.cu -- block-parallel chunked linear attention, bf16
+// I/O with fp32 accumulation, for d = dv = 64 (sm_100a: tcgen05 + TMA + TMEM).
+//
+// Method (lineartile 1.0.0, "How It Works" and "Reference"):
+//     O_i = phi(Q_i) S_i / (phi(Q_i) . z_i + eps),  S_i = sum_{j<=i} phi(K_j)^T V_j,
+//     z_i = sum_{j<=i} phi(K_j),  phi(x) = ELU(x) + 1.
+// Evaluation is the two-level chunked scan of "Why Stream Wins at
+// Ultra-Long Context", section 5.3 (chunk-local work, an inter-chunk carry,
+// and a broadcast correction), applied twice:
+//   * a sequence is cut into blocks of Bc chunks of 128 tokens;
+//   * lt_block_state_kernel: one CTA per block computes the block aggregate
+//     A_b = sum_{c in b} phi(K_c)^T [V_c | 1]  (fp32, to a workspace);
+//   * lt_block_fwd_kernel: one CTA per block walks its chunks in order,
+//     starting from the carry sum_{b' < b} A_b' and then carrying
+//     [S|z] += phi(K_c)^T [V_c|1] from chunk to chunk, and computes
+//         num_c = mask(phi(Q_c) phi(K_c)^T) V_c + phi(Q_c) S_<c
+//         den_c = mask(phi(Q_c) phi(K_c)^T) 1   + phi(Q_c) z_<c
+//     on the tensor cores.
+// No CTA waits on another: the two launches are ordered on the stream.
+// With one block per sequence the first launch is skipped.
+// Non-causal mode: the state kernel computes every block's sum and the
+// forward kernel reads only Q, with [S|z] = sum of all blocks.
+//
+// Forward-kernel warp roles (448 threads):
+//   warps 0-3   transform: phi in place on K and Q tiles (tail rows zeroed);
+//               causal mask of the score tile, bf16 in place in TMEM, and
+//               the score row sums into the accumulator's normaliser column
+//   warps 4-7   epilogue: accumulator -> normalised bf16 rows -> global
+//   warps 8-11  state: running [S|z] in registers -> bf16 B operand
+//   warp 12     TMA producer
+//   warp 13     TMEM allocator and single-thread MMA issuer
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#include "fwd_common.cuh"
+#include "lt_internal.h"
+#include "lt_ptx.cuh"
+
+namespace lt {
+namespace {
+using namespace fwd;
+
+constexpr int D = 64, DV = 64;
+constexpr int E = D * DV + D;  // block aggregate: S (row-major d x dv) then z
+constexpr int QT = kChunk * D * 2, KT = kChunk * D * 2, VT = kChunk * DV * 2;
+constexpr int SOPT = (DV / 64 + 1) * D * kRowBytes;
+constexpr int ONEST = kChunk * kRowBytes;
+constexpr int ACCW = DV + 16;
+
+struct BlockArgs {
+  __nv_bfloat16* out;
+  const int32_t* cu_seqlens;
+  float* ws;        // block aggregates [lane][nb][E], or nullptr
+  int Hq, Hkv, N, G, causal;
+  int nb;           // blocks per sequence (lane)
+  int bc;           // chunks per block
+  float eps;
+  int total_tokens;
+  int* err;
+};
+
+__device__ __forceinline__ bool seq_bounds(const BlockArgs& a, int s, int& t0, int& n) {
+  if (a.cu_seqlens) {
+    const int lo = a.cu_seqlens[s], hi = a.cu_seqlens[s + 1];
+    if (lo < 0 || hi < lo || hi > a.total_tokens) return false;
+    t0 = lo;
+    n = hi - lo;
+  } else {
+    t0 = s * a.N;
+    n = a.N;
+  }
+  return true;
+}
+
+// ========================================================================
+// Block aggregates.  192 threads: warps 0-3 transform (and the final
+// readout), warp 4 producer, warp 5 MMA.
+// ========================================================================
+constexpr int kStThreads = 192;
+constexpr int NS = 4;  // K/V stages
+constexpr int ST_OFF_K = 0, ST_OFF_V = NS * KT, ST_OFF_ONES = ST_OFF_V + NS * VT;
+constexpr int ST_OFF_BAR = ST_OFF_ONES + ONEST;
+constexpr int ST_SMEM = ST_OFF_BAR + (3 * NS + 2) * 8 + 16 + 1024;
+
+__global__ void __launch_bounds__(kStThreads, 1)
+    lt_block_state_kernel(const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const BlockArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ volatile int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int blk = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+  int t0, ntok;
+  if (!seq_bounds(a, s, t0, ntok)) {
+    if (tid == 0) report_error(a.err, kDevErrBadSeqlens);
+    return;
+  }
+  const int nc = (ntok + kChunk - 1) / kChunk;
+  const int c0 = blk * a.bc, c1 = min(c0 + a.bc, nc);
+  const int nchunks = c1 > c0 ? c1 - c0 : 0;
+  float* dst = a.ws + ((size_t)(s * a.Hkv + g) * a.nb + blk) * E;
+  uint8_t* sK = smem + ST_OFF_K;
+  uint8_t* sV = smem + ST_OFF_V;
+  uint8_t* sONES = smem + ST_OFF_ONES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST_OFF_BAR);
+  uint64_t* empty = full + NS;
+  uint64_t* xf = empty + NS;
+  uint64_t* s_full = xf + NS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 2);
+  if (tid == 0) {
+    s_abort = 0;
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&xf[i], 1);
+    }
+    mbar_init(s_full, 1);
+    fence_mbar_init();
+  }
+  init_ones_block(sONES, tid, kStThreads);
+  fence_proxy_async_smem();
+  if (warp == 5) tmem_alloc(tmem_slot, 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* abort_flag = &s_abort;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      int issued = 0;
+      bool ok = true;
+      for (int i = 0; i < nchunks && ok; ++i) {
+        const int st = i % NS, c = c0 + i;
+        ok = mbar_wait(&empty[st], ((i / NS) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&full[st], KT + VT);
+        tma_load_3d(sK + st * KT, &tm_k, &full[st], 0, g, t0 + c * kChunk);
+        tma_load_3d(sV + st * VT, &tm_v, &full[st], 0, g, t0 + c * kChunk);
+        ++issued;
+      }
+      if (!ok) {
+        int dummy = 0;
+        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i)
+          mbar_wait(&full[i % NS], (i / NS) & 1, &dummy, nullptr, kWaitLimitNs);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t ID_SV = idesc_bf16_f32(D, DV, 1, 1);
+      constexpr uint32_t ID_S1 = idesc_bf16_f32(D, 16, 1, 1);
+      const uint64_t dK = smem_desc_sw128(smem_u32(sK), kBox, 1024);
+      const uint64_t dV = smem_desc_sw128(smem_u32(sV), kBox, 1024);
+      const uint64_t d1 = smem_desc_sw128(smem_u32(sONES), kBox, 1024);
+      bool ok = true;
+      for (int i = 0; i < nchunks && ok; ++i) {
+        const int st = i % NS;
+        ok = mbar_wait(&xf[st], (i / NS) & 1, abort_flag, a.err, kWaitLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t kd = desc_advance(dK, st * KT), vd = desc_advance(dV, st * VT);
+#pragma unroll
+        for (int kk = 0; kk < kChunk / 16; ++kk) {
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t ad = desc_advance(kd, kk * 2048);
+          umma_f16_ss(tmem, ad, desc_advance(vd, kk * 2048), ID_SV, acc);
+          umma_f16_ss(tmem + DV, ad, desc_advance(d1, kk * 2048), ID_S1, acc);
+        }
+        umma_commit(&empty[st]);
+      }
+      umma_commit(s_full);
+      int dummy = 0;  // drain the tensor pipe before TMEM is released
+      mbar_wait(s_full, 0, &dummy, nullptr, kWaitLimitNs);
+    }
+  } else {
+    const int x = tid;
+    bool ok = true;
+    for (int i = 0; i < nchunks && ok; ++i) {
+      const int st = i % NS, c = c0 + i;
+      ok = mbar_wait(&full[st], (i / NS) & 1, abort_flag, a.err, kWaitLimitNs);
+      if (!ok) break;
+      const int valid = min(kChunk, ntok - c * kChunk);
+      xf_tile<D / 64>(sK + st * KT, valid, true, x);
+      if (valid < kChunk) xf_tile<DV / 64>(sV + st * VT, valid, false, x);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (x == 0) mbar_arrive(&xf[st]);
+    }
+    // read the aggregate (M = 64 accumulator: row 16*w + l in lane l < 16
+    // of sub-partition w) and store it; an empty block stores zeros
+    if (ok) ok = mbar_wait(s_full, 0, abort_flag, a.err, kWaitLimitNs);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t t = tmem + ((uint32_t)(warp * 32) << 16);
+      float c0v[32], c1v[32], zz[16];
+      tmem_ld32(t, c0v);
+      tmem_ld32(t + 32, c1v);
+      tmem_ld16(t + DV, zz);
+      tmem_wait_ld();
+      if (lane < 16) {
+        const int row = warp * 16 + lane;
+        float4* d4 = reinterpret_cast<float4*>(dst + row * DV);
+        const bool any = nchunks > 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          d4[q] = any ? make_float4(c0v[4 * q], c0v[4 * q + 1], c0v[4 * q + 2], c0v[4 * q + 3])
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          d4[8 + q] = any ? make_float4(c1v[4 * q], c1v[4 * q + 1], c1v[4 * q + 2], c1v[4 * q + 3])
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        dst[D * DV + row] = any ? zz[0] : 0.0f;
+      }
+      tc_fence_before();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ========================================================================
+// Forward pass over one block per CTA.
+// ========================================================================
+constexpr int kThreads = 448;
+constexpr int NQ = 4, NKV = 3;
+constexpr int TM_P = 0, TM_ACC = kChunk, TM_DS = TM_ACC + 2 * ACCW, TM_COLS = 512;
+static_assert(TM_DS + 2 * ACCW <= TM_COLS, "TMEM budget");
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = OFF_Q + NQ * QT;
+constexpr int OFF_V = OFF_K + NKV * KT;
+constexpr int OFF_SOP = OFF_V + NKV * VT;
+constexpr int OFF_ONES = OFF_SOP + SOPT;
+constexpr int OFF_BAR = OFF_ONES + ONEST;
+constexpr int NBARS = 3 * NQ + 3 * NKV + 2 + 2 + 2 * 2 + 2 * 2 + 1;
+constexpr int SMEM = OFF_BAR + NBARS * 8 + 16 + 1024;
+static_assert(SMEM <= 232448, "shared memory budget");
+
+struct Bars {
+  uint64_t *q_full, *q_empty, *q_xf, *kv_full, *kv_empty, *kv_xf;
+  uint64_t *p_full, *pb_full, *sop_full, *sop_empty;
+  uint64_t *ds_full, *ds_empty, *acc_full, *acc_empty, *drain;
+};
+
+__device__ __forceinline__ Bars carve(uint8_t* base) {
+  uint64_t* b = reinterpret_cast<uint64_t*>(base);
+  Bars r;
+  r.q_full = b; b += NQ;
+  r.q_empty = b; b += NQ;
+  r.q_xf = b; b += NQ;
+  r.kv_full = b; b += NKV;
+  r.kv_empty = b; b += NKV;
+  r.kv_xf = b; b += NKV;
+  r.p_full = b++;
+  r.pb_full = b++;
+  r.sop_full = b++;
+  r.sop_empty = b++;
+  r.ds_full = b; b += 2;
+  r.ds_empty = b; b += 2;
+  r.acc_full = b; b += 2;
+  r.acc_empty = b; b += 2;
+  r.drain = b++;
+  return r;
+}
+
+// One row of the [S | z 0 ... 0] operand (MN-major, 128-byte swizzle; row =
+// state row a, columns n = 0..dv+15) from fp32 values.
+__device__ __forceinline__ void write_sop_row(uint8_t* sop, int a, const float* s, float z) {
+#pragma unroll
+  for (int q8 = 0; q8 < DV / 8; ++q8) {
+    const uint4 w = make_uint4(pack_bf16x2(s[q8 * 8 + 0], s[q8 * 8 + 1]),
+                               pack_bf16x2(s[q8 * 8 + 2], s[q8 * 8 + 3]),
+                               pack_bf16x2(s[q8 * 8 + 4], s[q8 * 8 + 5]),
+                               pack_bf16x2(s[q8 * 8 + 6], s[q8 * 8 + 7]));
+    *reinterpret_cast<uint4*>(sop + (q8 >> 3) * (D * kRowBytes) + sw128_off(a, q8 & 7)) = w;
+  }
+  const int grp = DV / 64;
+  *reinterpret_cast<uint4*>(sop + grp * (D * kRowBytes) + sw128_off(a, 0)) =
+      make_uint4(pack_bf16x2(z, 0.0f), 0u, 0u, 0u);
+  *reinterpret_cast<uint4*>(sop + grp * (D * kRowBytes) + sw128_off(a, 1)) =
+      make_uint4(0u, 0u, 0u, 0u);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    lt_block_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const BlockArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ volatile int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int blk = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+  int t0, ntok;
+  if (!seq_bounds(a, s, t0, ntok)) {
+    if (tid == 0) report_error(a.err, kDevErrBadSeqlens);
+    return;
+  }
+  const int nc = (ntok + kChunk - 1) / kChunk;
+  const int c0 = blk * a.bc, c1 = min(c0 + a.bc, nc);
+  if (c1 <= c0) return;  // nothing in this block (uniform over the CTA)
+  const int Ri = c1 - c0;  // chunks of this block, walked in order
+  const int G = a.G;
+  const bool causal = a.causal != 0;
+  const int n_items = Ri * G;
+  // non-causal with a workspace: the state is the sum of all blocks and this
+  // CTA reads only Q
+  const bool nc_from_ws = !causal && a.ws != nullptr;
+
+  uint8_t* sQ = smem + OFF_Q;
+  uint8_t* sK = smem + OFF_K;
+  uint8_t* sV = smem + OFF_V;
+  uint8_t* sSOP = smem + OFF_SOP;
+  uint8_t* sONES = smem + OFF_ONES;
+  Bars bars = carve(smem + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + NBARS * 8);
+
+  if (tid == 0) {
+    s_abort = 0;
+    for (int i = 0; i < NQ; ++i) {
+      mbar_init(&bars.q_full[i], 1);
+      mbar_init(&bars.q_empty[i], 1);
+      mbar_init(&bars.q_xf[i], 1);
+    }
+    for (int i = 0; i < NKV; ++i) {
+      mbar_init(&bars.kv_full[i], 1);
+      mbar_init(&bars.kv_empty[i], 1);
+      mbar_init(&bars.kv_xf[i], 1);
+    }
+    mbar_init(bars.p_full, 1);
+    mbar_init(bars.pb_full, 1);
+    mbar_init(bars.sop_full, 1);
+    mbar_init(bars.sop_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.ds_full[i], 1);
+      mbar_init(&bars.ds_empty[i], 1);
+      mbar_init(&bars.acc_full[i], 1);
+      mbar_init(&bars.acc_empty[i], 1);
+    }
+    mbar_init(bars.drain, 1);
+    fence_mbar_init();
+  }
+  init_ones_block(sONES, tid, kThreads);
+  fence_proxy_async_smem();
+  if (warp == 13) tmem_alloc(tmem_slot, TM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* abort_flag = &s_abort;
+
+  if (warp == 12) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      int q_issued = 0, kv_issued = 0;
+      bool ok = true;
+      auto load_kv = [&](int r) -> bool {
+        const int st = r % NKV, c = c0 + r;
+        if (!mbar_wait(&bars.kv_empty[st], ((r / NKV) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+          return false;
+        mbar_arrive_expect_tx(&bars.kv_full[st], KT + VT);
+        tma_load_3d(sK + st * KT, &tm_k, &bars.kv_full[st], 0, g, t0 + c * kChunk);
+        tma_load_3d(sV + st * VT, &tm_v, &bars.kv_full[st], 0, g, t0 + c * kChunk);
+        ++kv_issued;
+        return true;
+      };
+      auto load_q = [&](int j) -> bool {
+        const int st = j % NQ, r = j / G, h = j % G, c = c0 + r;
+        if (!mbar_wait(&bars.q_empty[st], ((j / NQ) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+          return false;
+        mbar_arrive_expect_tx(&bars.q_full[st], QT);
+        tma_load_3d(sQ + st * QT, &tm_q, &bars.q_full[st], 0, g * G + h, t0 + c * kChunk);
+        ++q_issued;
+        return true;
+      };
+      if (causal) {
+        for (int r = 0; r < Ri && ok; ++r) {
+          ok = load_kv(r);
+          for (int h = 0; h < G && ok; ++h) ok = load_q(r * G + h);
+        }
+      } else {
+        if (!nc_from_ws)
+          for (int r = 0; r < Ri && ok; ++r) ok = load_kv(r);
+        for (int j = 0; j < n_items && ok; ++j) ok = load_q(j);
+      }
+      if (!ok) {  // drain copies in flight (bounded, ignoring the abort flag)
+        int dummy = 0;
+        for (int r = (kv_issued > NKV ? kv_issued - NKV : 0); r < kv_issued; ++r)
+          mbar_wait(&bars.kv_full[r % NKV], (r / NKV) & 1, &dummy, nullptr, kWaitLimitNs);
+        for (int j = (q_issued > NQ ? q_issued - NQ : 0); j < q_issued; ++j)
+          mbar_wait(&bars.q_full[j % NQ], (j / NQ) & 1, &dummy, nullptr, kWaitLimitNs);
+      }
+    }
+  } else if (warp == 13) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_P = idesc_bf16_f32(kChunk, kChunk, 0, 0);
+      constexpr uint32_t ID_SV = idesc_bf16_f32(D, DV, 1, 1);
+      constexpr uint32_t ID_S1 = idesc_bf16_f32(D, 16, 1, 1);
+      constexpr uint32_t ID_PV = idesc_bf16_f32(kChunk, DV, 0, 1);
+      constexpr uint32_t ID_QS = idesc_bf16_f32(kChunk, DV + 16, 0, 1);
+      // descriptor bases, advanced per stage / K step with one 64-bit add
+      const uint64_t dQk = smem_desc_sw128(smem_u32(sQ), 16, 1024);      // K-major
+      const uint64_t dKk = smem_desc_sw128(smem_u32(sK), 16, 1024);      // K-major
+      const uint64_t dKmn = smem_desc_sw128(smem_u32(sK), kBox, 1024);   // MN-major
+      const uint64_t dVmn = smem_desc_sw128(smem_u32(sV), kBox, 1024);   // MN-major
+      const uint64_t d1 = smem_desc_sw128(smem_u32(sONES), kBox, 1024);
+      const uint64_t dSop = smem_desc_sw128(smem_u32(sSOP), D * kRowBytes, 1024);
+      bool ok = true;
+      // dS (or the running S for the non-causal state pass) = phi(K)^T [V | 1]
+      auto issue_ds = [&](int r, uint32_t t_ds, bool accumulate) {
+        const int st = r % NKV;
+        const uint64_t ka = desc_advance(dKmn, st * KT), vb = desc_advance(dVmn, st * VT);
+#pragma unroll
+        for (int kk = 0; kk < kChunk / 16; ++kk) {
+          const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
+          const uint64_t ad = desc_advance(ka, kk * 2048);
+          umma_f16_ss(t_ds, ad, desc_advance(vb, kk * 2048), ID_SV, acc);
+          umma_f16_ss(t_ds + DV, ad, desc_advance(d1, kk * 2048), ID_S1, acc);
+        }
+      };
+      // Acc (+)= phi(Q) [S | z 0 ..]
+      auto issue_qs = [&](uint32_t t_acc, int qs, bool accumulate) {
+        const uint64_t qa = desc_advance(dQk, qs * QT);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_f16_ss(t_acc, desc_advance(qa, (kk >> 2) * kBox + (kk & 3) * 32),
+                      desc_advance(dSop, kk * 2048), ID_QS, (accumulate || kk > 0) ? 1u : 0u);
+      };
+      if (causal) {
+        auto state_mma = [&](int r) -> bool {
+          const int b = r & 1;
+          if (!mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs) ||
+              !mbar_wait(&bars.ds_empty[b], ((r >> 1) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+            return false;
+          tc_fence_after();
+          issue_ds(r, tmem + TM_DS + b * ACCW, false);
+          umma_commit(&bars.ds_full[b]);
+          return true;
+        };
+        ok = state_mma(0);
+        for (int r = 0; r < Ri && ok; ++r) {
+          const uint64_t kd = desc_advance(dKk, (r % NKV) * KT);
+          const uint64_t vd = desc_advance(dVmn, (r % NKV) * VT);
+          for (int h = 0; h < G && ok; ++h) {
+            const int j = r * G + h, qs = j % NQ, as = j & 1;
+            const uint64_t qd = desc_advance(dQk, qs * QT);
+            const uint32_t t_acc = tmem + TM_ACC + as * ACCW;
+            // The previous item's score tile was read by its P V MMAs,
+            // issued before this one: the tensor pipe runs them in order.
+            ok = mbar_wait(&bars.q_xf[qs], (j / NQ) & 1, abort_flag, a.err, kWaitLimitNs);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t o = (kk >> 2) * kBox + (kk & 3) * 32;
+              umma_f16_ss(tmem + TM_P, desc_advance(qd, o), desc_advance(kd, o), ID_P,
+                          kk > 0 ? 1u : 0u);
+            }
+            umma_commit(bars.p_full);
+            // the next chunk's state MMA, after the score MMA so that the
+            // score tile does not wait for the next K tile
+            if (h == 0 && r + 1 < Ri) {
+              ok = state_mma(r + 1);
+              if (!ok) break;
+            }
+            ok = mbar_wait(bars.pb_full, j & 1, abort_flag, a.err, kWaitLimitNs) &&
+                 mbar_wait(&bars.acc_empty[as], ((j >> 1) & 1) ^ 1, abort_flag, a.err,
+                           kWaitLimitNs);
+            if (!ok) break;
+            tc_fence_after();
+            // P V: bf16 scores from TMEM, 16 keys (8 columns) per MMA.  The
+            // normaliser column was initialised with the score row sums.
+#pragma unroll
+            for (int kk = 0; kk < kChunk / 16; ++kk)
+              umma_f16_ts(t_acc, tmem + TM_P + kk * 8, desc_advance(vd, kk * 2048), ID_PV,
+                          kk > 0 ? 1u : 0u);
+            if (h == G - 1) umma_commit(&bars.kv_empty[r % NKV]);
+            if (h == 0) {
+              ok = mbar_wait(bars.sop_full, r & 1, abort_flag, a.err, kWaitLimitNs);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            issue_qs(t_acc, qs, true);
+            umma_commit(&bars.acc_full[as]);
+            umma_commit(&bars.q_empty[qs]);
+          }
+          if (ok) umma_commit(bars.sop_empty);
+        }
+      } else {
+        if (!nc_from_ws) {
+          for (int r = 0; r < Ri && ok; ++r) {
+            ok = mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs);
+            if (!ok) break;
+            tc_fence_after();
+            issue_ds(r, tmem + TM_DS, r > 0);
+            umma_commit(&bars.kv_empty[r % NKV]);
+          }
+          if (ok) umma_commit(&bars.ds_full[0]);
+        }
+        if (ok) ok = mbar_wait(bars.sop_full, 0, abort_flag, a.err, kWaitLimitNs);
+        for (int j = 0; j < n_items && ok; ++j) {
+          const int qs = j % NQ, as = j & 1;
+          ok = mbar_wait(&bars.q_xf[qs], (j / NQ) & 1, abort_flag, a.err, kWaitLimitNs) &&
+               mbar_wait(&bars.acc_empty[as], ((j >> 1) & 1) ^ 1, abort_flag, a.err,
+                         kWaitLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qs(tmem + TM_ACC + as * ACCW, qs, false);
+          umma_commit(&bars.acc_full[as]);
+          umma_commit(&bars.q_empty[qs]);
+        }
+      }
+      umma_commit(bars.drain);
+      int dummy = 0;
+      mbar_wait(bars.drain, 0, &dummy, nullptr, kWaitLimitNs);
+    }
+  } else if (warp < 4) {
+    // ----------------------------------------------- transform warpgroup
+    const int x = tid;
+    bool ok = true;
+    auto xf_kv = [&](int r) -> bool {
+      const int st = r % NKV, c = c0 + r;
+      if (!mbar_wait(&bars.kv_full[st], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs))
+        return false;
+      const int valid = min(kChunk, ntok - c * kChunk);
+      xf_tile<D / 64>(sK + st * KT, valid, true, x);
+      if (valid < kChunk) xf_tile<DV / 64>(sV + st * VT, valid, false, x);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (x == 0) mbar_arrive(&bars.kv_xf[st]);
+      return true;
+    };
+    auto xf_q = [&](int j) -> bool {
+      const int st = j % NQ;
+      if (!mbar_wait(&bars.q_full[st], (j / NQ) & 1, abort_flag, a.err, kWaitLimitNs))
+        return false;
+      xf_tile<D / 64>(sQ + st * QT, kChunk, true, x);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (x == 0) mbar_arrive(&bars.q_xf[st]);
+      return true;
+    };
+    // causal mask and bf16 rounding of the score tile, in place in TMEM:
+    // fp32 columns [32b, 32b+32) become packed bf16 columns [16b, 16b+16),
+    // which only overwrites columns this thread has already read; the row
+    // sum of the rounded scores initialises the accumulator's normaliser
+    auto mask_p = [&](int j) -> bool {
+      const int as = j & 1;
+      if (!mbar_wait(bars.p_full, j & 1, abort_flag, a.err, kWaitLimitNs) ||
+          !mbar_wait(&bars.acc_empty[as], ((j >> 1) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+        return false;
+      tc_fence_after();
+      const uint32_t lane_sel = (uint32_t)(warp * 32) << 16;
+      const uint32_t t_p = tmem + TM_P + lane_sel;
+      const int row = x;
+      float rs = 0.0f;
+#pragma unroll
+      for (int b2 = 0; b2 < kChunk / 64; ++b2) {
+        // two 32-column blocks per TMEM round trip
+        float r0[32], r1[32];
+        const bool h0 = 2 * b2 <= warp, h1 = 2 * b2 + 1 <= warp;  // warp-uniform
+        if (h0) tmem_ld32(t_p + (2 * b2) * 32, r0);
+        if (h1) tmem_ld32(t_p + (2 * b2 + 1) * 32, r1);
+        if (h0) tmem_wait_ld();
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int b = 2 * b2 + half;
+          const float* r = half ? r1 : r0;
+          const bool have = half ? h1 : h0;
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float lo = (!have || b * 32 + 2 * e > row) ? 0.0f : r[2 * e];
+            const float hi = (!have || b * 32 + 2 * e + 1 > row) ? 0.0f : r[2 * e + 1];
+            pk[e] = pack_bf16x2(lo, hi);
+            const float2 rr = unpack_bf16x2(pk[e]);
+            rs += rr.x + rr.y;
+          }
+          tmem_st16(t_p + b * 16, pk);
+        }
+      }
+      tmem_st1(tmem + TM_ACC + as * ACCW + DV + lane_sel, __float_as_uint(rs));
+      tmem_wait_st();
+      tc_fence_before();
+      named_bar_sync(1, 128);
+      if (x == 0) mbar_arrive(bars.pb_full);
+      return true;
+    };
+    if (causal) {
+      ok = xf_kv(0);
+      for (int r = 0; r < Ri && ok; ++r) {
+        for (int h = 0; h < G && ok; ++h) {
+          ok = xf_q(r * G + h);
+          if (ok && h == 0 && r + 1 < Ri) ok = xf_kv(r + 1);  // next K while P runs
+          if (ok) ok = mask_p(r * G + h);
+        }
+      }
+    } else {
+      if (!nc_from_ws)
+        for (int r = 0; r < Ri && ok; ++r) ok = xf_kv(r);
+      for (int j = 0; j < n_items && ok; ++j) ok = xf_q(j);
+    }
+  } else if (warp < 8) {
+    // ----------------------------------------------- epilogue warpgroup
+    const int x = tid - 128, sp = warp & 3;
+    const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+    bool ok = true;
+    for (int j = 0; j < n_items && ok; ++j) {
+      const int r = j / G, h = j % G, as = j & 1, c = c0 + r;
+      ok = mbar_wait(&bars.acc_full[as], (j >> 1) & 1, abort_flag, a.err, kWaitLimitNs);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t t_acc = tmem + TM_ACC + as * ACCW + lane_base;
+      float den[16], n0[32], n1[32];
+      tmem_ld16(t_acc + DV, den);
+      tmem_ld32(t_acc, n0);
+      tmem_ld32(t_acc + 32, n1);
+      tmem_wait_ld();
+      tc_fence_before();
+      named_bar_sync(2, 128);
+      if (x == 0) mbar_arrive(&bars.acc_empty[as]);
+      const float inv = 1.0f / (den[0] + a.eps);
+      const int valid = min(kChunk, ntok - c * kChunk);
+      if (x < valid) {
+        __nv_bfloat16* orow =
+            a.out + ((size_t)(t0 + c * kChunk + x) * a.Hq + (size_t)(g * G + h)) * DV;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          *reinterpret_cast<uint4*>(orow + q4 * 8) =
+              make_uint4(pack_bf16x2(n0[q4 * 8 + 0] * inv, n0[q4 * 8 + 1] * inv),
+                         pack_bf16x2(n0[q4 * 8 + 2] * inv, n0[q4 * 8 + 3] * inv),
+                         pack_bf16x2(n0[q4 * 8 + 4] * inv, n0[q4 * 8 + 5] * inv),
+                         pack_bf16x2(n0[q4 * 8 + 6] * inv, n0[q4 * 8 + 7] * inv));
+          *reinterpret_cast<uint4*>(orow + 32 + q4 * 8) =
+              make_uint4(pack_bf16x2(n1[q4 * 8 + 0] * inv, n1[q4 * 8 + 1] * inv),
+                         pack_bf16x2(n1[q4 * 8 + 2] * inv, n1[q4 * 8 + 3] * inv),
+                         pack_bf16x2(n1[q4 * 8 + 4] * inv, n1[q4 * 8 + 5] * inv),
+                         pack_bf16x2(n1[q4 * 8 + 6] * inv, n1[q4 * 8 + 7] * inv));
+        }
+      }
+    }
+  } else if (warp < 12) {
+    // -------------------------------------------------- state warpgroup
+    // dS is an M=64 accumulator: state row a = 16*sp + l lives in lane l < 16
+    // of TMEM sub-partition sp; that thread owns row a of the running state.
+    const int y = tid - 256, sp = warp & 3;
+    const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+    const bool has_row = lane < 16;
+    const int row = sp * 16 + lane;
+    bool ok = true;
+    float T[DV], Tz = 0.0f;
+#pragma unroll
+    for (int e = 0; e < DV; ++e) T[e] = 0.0f;
+    // carry into this block: the aggregates of the earlier blocks (causal),
+    // or of every block (non-causal), summed in fp32
+    if (a.ws != nullptr && has_row) {
+      const float* base = a.ws + (size_t)(s * a.Hkv + g) * a.nb * E;
+      const int nprev = causal ? blk : a.nb;
+      for (int bb = 0; bb < nprev; ++bb) {
+        const float4* r4 = reinterpret_cast<const float4*>(base + (size_t)bb * E + row * DV);
+#pragma unroll
+        for (int q = 0; q < DV / 4; ++q) {
+          const float4 v = r4[q];
+          T[4 * q] += v.x;
+          T[4 * q + 1] += v.y;
+          T[4 * q + 2] += v.z;
+          T[4 * q + 3] += v.w;
+        }
+        Tz += base[(size_t)bb * E + D * DV + row];
+      }
+    }
+    auto publish_sop = [&](int r) -> bool {
+      if (!mbar_wait(bars.sop_empty, (r & 1) ^ 1, abort_flag, a.err, kWaitLimitNs)) return false;
+      if (has_row) write_sop_row(sSOP, row, T, Tz);
+      fence_proxy_async_smem();
+      named_bar_sync(3, 128);
+      if (y == 0) mbar_arrive(bars.sop_full);
+      return true;
+    };
+    auto add_ds = [&](int b) {
+      const uint32_t t = tmem + TM_DS + b * ACCW + lane_base;
+      float c0v[32], c1v[32], zz[16];
+      tmem_ld32(t, c0v);
+      tmem_ld32(t + 32, c1v);
+      tmem_ld16(t + DV, zz);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        T[e] += c0v[e];
+        T[32 + e] += c1v[e];
+      }
+      Tz += zz[0];
+    };
+    if (causal) {
+      for (int r = 0; r < Ri && ok; ++r) {
+        ok = publish_sop(r);  // [S|z]_<c does not need this chunk's dS
+        if (!ok) break;
+        const int b = r & 1;
+        ok = mbar_wait(&bars.ds_full[b], (r >> 1) & 1, abort_flag, a.err, kWaitLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+        add_ds(b);
+        tc_fence_before();
+        named_bar_sync(3, 128);
+        if (y == 0) mbar_arrive(&bars.ds_empty[b]);
+      }
+    } else {
+      if (!nc_from_ws) {
+        ok = mbar_wait(&bars.ds_full[0], 0, abort_flag, a.err, kWaitLimitNs);
+        if (ok) {
+          tc_fence_after();
+          add_ds(0);
+          tc_fence_before();
+        }
+      }
+      if (ok) ok = publish_sop(0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+}
+
+}  // namespace
+
+bool block_supported(const FwdLaunch& p) { return p.d == 64 && p.dv == 64; }
+
+// Workspace of the block aggregates (none with one block per sequence).
+size_t block_workspace_bytes(const FwdLaunch& p, int nb) {
+  return nb > 1 ? (size_t)p.B * p.Hkv * nb * E * sizeof(float) : 0;
+}
+
+// Blocks per sequence: enough CTAs to cover the SMs about once.
+int block_count(const FwdLaunch& p, int num_sms) {
+  const char* force = getenv("LT_BLOCKS");
+  const int nc = p.cu_seqlens ? 0 : (p.N + kChunk - 1) / kChunk;
+  if (p.cu_seqlens) return 1;  // packed: one block per (sequence, KV head)
+  if (force) {
+    const int f = atoi(force);
+    return f < 1 ? 1 : (f > nc ? nc : f);
+  }
+  const int lanes = p.B * p.Hkv;
+  int nb = num_sms / (lanes > 0 ? lanes : 1);
+  if (nb < 1) nb = 1;
+  if (nb > nc) nb = nc;
+  return nb;
+}
+
+cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
+      !make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64) ||
+      !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64))
+    return cudaErrorInvalidValue;
+  const int nc = p.cu_seqlens ? 0 : (p.N + kChunk - 1) / kChunk;
+  BlockArgs a;
+  a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
+  a.cu_seqlens = p.cu_seqlens;
+  a.ws = nb > 1 ? ws : nullptr;
+  a.Hq = p.Hq;
+  a.Hkv = p.Hkv;
+  a.N = p.N;
+  a.G = p.Hq / p.Hkv;
+  a.causal = p.causal;
+  a.nb = nb;
+  a.bc = nb > 1 ? (nc + nb - 1) / nb : (1 << 30);
+  a.eps = p.eps;
+  a.total_tokens = (int)p.total_tokens;
+  a.err = p.err;
+  cudaError_t e;
+  if (nb > 1) {
+    auto sk = lt_block_state_kernel;
+    e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ST_SMEM);
+    if (e != cudaSuccess) return e;
+    // causal: the last block's aggregate is never needed
+    const int nstate = p.causal ? nb - 1 : nb;
+    sk<<<dim3(nstate, p.Hkv, p.B), kStThreads, ST_SMEM, stream>>>(tk, tv, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  auto fk = lt_block_fwd_kernel;
+  e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) return e;
+  fk<<<dim3(nb, p.Hkv, p.B), kThreads, SMEM, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace lt

@@ -633,10 +633,31 @@ cudaError_t launch_fwd(const FwdLaunch& p, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_fwd_bf16(const FwdLaunch& p, cudaStream_t stream) {
-  // LT_KERNEL=seq selects the sequential kernel for every shape (ablation)
+  // LT_KERNEL selects a kernel for every shape it supports (ablations):
+  //   seq      one CTA per (sequence, KV head), sequential chunks
+  //   cluster  sequence split over a thread-block cluster (d = dv = 64)
   const char* force = getenv("LT_KERNEL");
-  const bool seq = force && force[0] == 's' && force[1] == 'e';
-  if (!seq && split_supported(p)) return launch_fwd_bf16_split(p, stream);
+  const bool seq = force && force[0] == 's';
+  const bool cluster = force && force[0] == 'c';
+  if (cluster && split_supported(p)) return launch_fwd_bf16_split(p, stream);
+  if (!seq && block_supported(p)) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int nb = block_count(p, sms);
+    const size_t bytes = block_workspace_bytes(p, nb);
+    void* ws = nullptr;
+    if (bytes) {
+      cudaError_t e = cudaMallocAsync(&ws, bytes, stream);
+      if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = launch_fwd_bf16_block(p, nb, static_cast<float*>(ws), stream);
+    if (ws) {
+      const cudaError_t f = cudaFreeAsync(ws, stream);
+      if (e == cudaSuccess) e = f;
+    }
+    return e;
+  }
   if (p.d == 64 && p.dv == 64) return launch_fwd<64, 64>(p, stream);
   if (p.d == 128 && p.dv == 128) return launch_fwd<128, 128>(p, stream);
   if (p.d == 64 && p.dv == 128) return launch_fwd<64, 128>(p, stream);

@@ -35,6 +35,12 @@ cudaError_t launch_fwd_bf16(const FwdLaunch& p, cudaStream_t stream);
 // (sequence, KV head) for packed inputs)
 bool split_supported(const FwdLaunch& p);
 cudaError_t launch_fwd_bf16_split(const FwdLaunch& p, cudaStream_t stream);
+// d = dv = 64: block-parallel two-launch scan (block aggregates, then one CTA
+// per block); `ws` holds block_workspace_bytes(p, nb) bytes when nb > 1
+bool block_supported(const FwdLaunch& p);
+int block_count(const FwdLaunch& p, int num_sms);
+size_t block_workspace_bytes(const FwdLaunch& p, int nb);
+cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream);
 cudaError_t launch_fwd_f32(const FwdLaunch& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeLaunch& p, cudaStream_t stream);
 

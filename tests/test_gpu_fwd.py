@@ -148,8 +148,10 @@ SPLIT_CASES = [
 @pytest.mark.parametrize("case", SPLIT_CASES, ids=lambda c: "B%dHq%dHkv%dN%d%s" % (
     c[0], c[1], c[2], c[3], "c" if c[4] else "nc"))
 def test_split_kernel_cluster_sizes(monkeypatch, n_split, case):
-    """d = dv = 64 runs a sequence split over a cluster of n CTAs that
-    exchange their chunk states through distributed shared memory."""
+    """The cluster variant (LT_KERNEL=cluster): a sequence split over a
+    cluster of n CTAs that exchange their chunk states through distributed
+    shared memory."""
+    monkeypatch.setenv("LT_KERNEL", "cluster")
     monkeypatch.setenv("LT_SPLIT_N", str(n_split))
     B, Hq, Hkv, N, causal = case
     q, k, v = inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16, 0.125, seed=N + n_split)
@@ -181,3 +183,40 @@ def test_split_and_sequential_agree_closely(monkeypatch):
     monkeypatch.setenv("LT_KERNEL", "seq")
     b = run_dense(q, k, v, True)
     assert row_rel_err(a, b) <= 1e-2
+
+
+BLOCK_CASES = [
+    # (B, Hq, Hkv, N, causal)
+    (1, 2, 2, 1000, True),      # 8 chunks, ragged tail
+    (2, 4, 2, 777, True),       # GQA
+    (1, 1, 1, 2049, False),     # 17 chunks, non-causal
+    (1, 2, 1, 130, True),       # 2 chunks: more blocks requested than chunks
+    (1, 3, 3, 3 * 128 * 5 + 7, True),  # uneven blocks and a ragged last chunk
+    (2, 2, 2, 1500, False),
+]
+
+
+@pytest.mark.parametrize("nb", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("case", BLOCK_CASES, ids=lambda c: "B%dHq%dHkv%dN%d%s" % (
+    c[0], c[1], c[2], c[3], "c" if c[4] else "nc"))
+def test_block_kernel_block_counts(monkeypatch, nb, case):
+    """d = dv = 64: block aggregates in a first launch, then one CTA per block
+    from the carried prefix.  LT_BLOCKS forces the number of blocks."""
+    monkeypatch.setenv("LT_BLOCKS", str(nb))
+    B, Hq, Hkv, N, causal = case
+    q, k, v = inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16, 0.125, seed=N + 7 * nb)
+    got = run_dense(q, k, v, causal)
+    ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
+    assert row_rel_err(got, ref) <= TOL_BF16
+
+
+def test_block_kernel_deterministic_across_block_counts(monkeypatch):
+    """Every block count computes the same function; results agree to a few
+    bf16 ulps (only the summation order of the carried state differs)."""
+    q, k, v = inputs.make_custom(1, 4, 4, 3000, 64, 64, torch.bfloat16, 0.125, seed=4)
+    outs = []
+    for nb in (1, 4, 12):
+        monkeypatch.setenv("LT_BLOCKS", str(nb))
+        outs.append(run_dense(q, k, v, True))
+    for o in outs[1:]:
+        assert row_rel_err(o, outs[0]) <= 1e-2
