@@ -68,7 +68,10 @@ def peaks():
 
 def source_digest():
     h = hashlib.sha256()
-    for rel in ("causal_linear_attention_chunked_b200/csrc/fwd_bf16_sm100.cu",
+    for rel in ("causal_linear_attention_chunked_b200/csrc/state_bf16_sm100.cu",
+                "causal_linear_attention_chunked_b200/csrc/fwd_bf16_block_sm100.cu",
+                "causal_linear_attention_chunked_b200/csrc/fwd_bf16_sm100.cu",
+                "causal_linear_attention_chunked_b200/csrc/fwd_common.cuh",
                 "causal_linear_attention_chunked_b200/csrc/lt_ptx.cuh"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
@@ -372,6 +375,12 @@ def run_lt(args):
     peak, peak_kind = peaks()
     achieved = nbytes / (ms_step * 1e-3) / 1e9
     traffic = committed_traffic(w.name)
+    packed = w.packed_len is not None
+    nblk, per_step, ws_bytes = L.linear_attn_fwd_plan(w.B, w.Hq, w.Hkv, 1 if packed else w.N,
+                                                      w.d, w.dv, causal=w.causal, packed=packed)
+    kern = ("lt_block_state_kernel + lt_block_fwd_kernel" if w.d == 64 and w.dv == 64 else
+            "lt_block_state_kernel + lt_fwd_bf16_kernel") if per_step == 2 else (
+            "lt_block_fwd_kernel" if w.d == 64 and w.dv == 64 else "lt_fwd_bf16_kernel")
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -387,11 +396,11 @@ def run_lt(args):
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "lt_fwd_bf16_kernel<64,64>",
+                     "kernel": "one forward pass (%s, %d block(s) per sequence)" % (kern, nblk),
                      "algorithmic_bytes_per_launch": nbytes,
                      "avg_launch_us": ms_step * 1e3},
         "clocks": clocks,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * per_step,
     }
     if args.profile:
         pass

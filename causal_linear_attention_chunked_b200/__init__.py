@@ -11,7 +11,8 @@ streams).  ``inputs`` holds the seeded synthetic workloads.
 The binding (and with it the library) is loaded on first use of one of the
 API names below; a missing library raises ImportError.
 """
-_API = ("linear_attn_fwd", "linear_attn_decode_step", "get_last_device_error",
+_API = ("linear_attn_fwd", "linear_attn_fwd_plan", "linear_attn_decode_step",
+        "get_last_device_error",
         "linear_attn_fwd_host", "LtError")
 
 

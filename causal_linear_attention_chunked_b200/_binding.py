@@ -18,8 +18,8 @@ LT_ERR_DEVICE_TIMEOUT, LT_ERR_DEVICE_BAD_SEQLENS = 4, 5
 LT_F32, LT_BF16 = 0, 1
 
 # every entry point declared in include/lt_linear_attn.h
-EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_decode_step", "lt_status_string",
-            "lt_get_last_device_error", "lt_abi_version")
+EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_fwd_plan", "lt_linear_attn_decode_step",
+            "lt_status_string", "lt_get_last_device_error", "lt_abi_version")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("liblt.so is not built (run `python -m "
@@ -30,6 +30,10 @@ _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 lib.lt_linear_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _vp,
                                    _i]
 lib.lt_linear_attn_fwd.restype = _i
+lib.lt_linear_attn_fwd_plan.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                        ctypes.POINTER(_i), ctypes.POINTER(_i),
+                                        ctypes.POINTER(ctypes.c_size_t)]
+lib.lt_linear_attn_fwd_plan.restype = _i
 lib.lt_linear_attn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f,
                                            _vp, _i]
 lib.lt_linear_attn_decode_step.restype = _i
@@ -96,6 +100,18 @@ def linear_attn_fwd(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, out=None, s
                                   int(bool(causal)), float(eps), _ptr(cu_seqlens),
                                   _stream_handle(stream, q.device), _dtype_code(q.dtype)))
     return out
+
+
+def linear_attn_fwd_plan(B, H_q, H_kv, N, d, dv, causal=True, packed=False,
+                         dtype=torch.bfloat16, num_sms=0):
+    """(blocks per sequence, kernel launches, workspace bytes) of one
+    linear_attn_fwd call on this shape; num_sms <= 0 asks the current
+    device."""
+    nb, nl, ws = _i(), _i(), ctypes.c_size_t()
+    _check(lib.lt_linear_attn_fwd_plan(B, H_q, H_kv, N, d, dv, int(bool(causal)),
+                                       int(bool(packed)), _dtype_code(dtype), int(num_sms),
+                                       ctypes.byref(nb), ctypes.byref(nl), ctypes.byref(ws)))
+    return nb.value, nl.value, ws.value
 
 
 def linear_attn_decode_step(q, k, v, S, z, eps=1e-6, out=None, stream=None):

@@ -21,14 +21,14 @@
 // Non-causal mode: the state kernel computes every block's sum and the
 // forward kernel reads only Q, with [S|z] = sum of all blocks.
 //
-// Forward-kernel warp roles (448 threads):
-//   warps 0-3   transform: phi in place on K and Q tiles (tail rows zeroed);
-//               causal mask of the score tile, bf16 in place in TMEM, and
-//               the score row sums into the accumulator's normaliser column
-//   warps 4-7   epilogue: accumulator -> normalised bf16 rows -> global
-//   warps 8-11  state: running [S|z] in registers -> bf16 B operand
-//   warp 12     TMA producer
-//   warp 13     TMEM allocator and single-thread MMA issuer
+// Forward-kernel warp roles (512 threads; TMEM sub-partition = warp % 4):
+//   warps 0-5   transform: phi in place on K and Q tiles (tail rows zeroed)
+//   warps 6-9   mask + epilogue: causal mask of the score tile, bf16 in
+//               place in TMEM, the score row sums into the accumulator's
+//               normaliser; accumulator -> normalised bf16 rows -> global
+//   warps 10-13 state: running [S|z] in registers -> bf16 B operand
+//   warp 14     TMA producer
+//   warp 15     TMEM allocator and single-thread MMA issuer
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -46,6 +46,7 @@ using namespace fwd;
 constexpr int D = 64, DV = 64;
 constexpr int E = D * DV + D;  // block aggregate: S (row-major d x dv) then z
 constexpr int QT = kChunk * D * 2, KT = kChunk * D * 2, VT = kChunk * DV * 2;
+constexpr int KVT = KT + VT;  // one K/V stage: [K][V]
 constexpr int SOPT = (DV / 64 + 1) * D * kRowBytes;
 constexpr int ONEST = kChunk * kRowBytes;
 constexpr int ACCW = DV + 16;
@@ -76,172 +77,20 @@ __device__ __forceinline__ bool seq_bounds(const BlockArgs& a, int s, int& t0, i
 }
 
 // ========================================================================
-// Block aggregates.  192 threads: warps 0-3 transform (and the final
-// readout), warp 4 producer, warp 5 MMA.
-// ========================================================================
-constexpr int kStThreads = 192;
-constexpr int NS = 4;  // K/V stages
-constexpr int ST_OFF_K = 0, ST_OFF_V = NS * KT, ST_OFF_ONES = ST_OFF_V + NS * VT;
-constexpr int ST_OFF_BAR = ST_OFF_ONES + ONEST;
-constexpr int ST_SMEM = ST_OFF_BAR + (3 * NS + 2) * 8 + 16 + 1024;
-
-__global__ void __launch_bounds__(kStThreads, 1)
-    lt_block_state_kernel(const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const BlockArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  __shared__ volatile int s_abort;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int blk = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
-  int t0, ntok;
-  if (!seq_bounds(a, s, t0, ntok)) {
-    if (tid == 0) report_error(a.err, kDevErrBadSeqlens);
-    return;
-  }
-  const int nc = (ntok + kChunk - 1) / kChunk;
-  const int c0 = blk * a.bc, c1 = min(c0 + a.bc, nc);
-  const int nchunks = c1 > c0 ? c1 - c0 : 0;
-  float* dst = a.ws + ((size_t)(s * a.Hkv + g) * a.nb + blk) * E;
-  uint8_t* sK = smem + ST_OFF_K;
-  uint8_t* sV = smem + ST_OFF_V;
-  uint8_t* sONES = smem + ST_OFF_ONES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST_OFF_BAR);
-  uint64_t* empty = full + NS;
-  uint64_t* xf = empty + NS;
-  uint64_t* s_full = xf + NS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 2);
-  if (tid == 0) {
-    s_abort = 0;
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
-      mbar_init(&xf[i], 1);
-    }
-    mbar_init(s_full, 1);
-    fence_mbar_init();
-  }
-  init_ones_block(sONES, tid, kStThreads);
-  fence_proxy_async_smem();
-  if (warp == 5) tmem_alloc(tmem_slot, 128);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  volatile int* abort_flag = &s_abort;
-
-  if (warp == 4) {
-    if (lane == 0) {
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      int issued = 0;
-      bool ok = true;
-      for (int i = 0; i < nchunks && ok; ++i) {
-        const int st = i % NS, c = c0 + i;
-        ok = mbar_wait(&empty[st], ((i / NS) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&full[st], KT + VT);
-        tma_load_3d(sK + st * KT, &tm_k, &full[st], 0, g, t0 + c * kChunk);
-        tma_load_3d(sV + st * VT, &tm_v, &full[st], 0, g, t0 + c * kChunk);
-        ++issued;
-      }
-      if (!ok) {
-        int dummy = 0;
-        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i)
-          mbar_wait(&full[i % NS], (i / NS) & 1, &dummy, nullptr, kWaitLimitNs);
-      }
-    }
-  } else if (warp == 5) {
-    if (lane == 0) {
-      constexpr uint32_t ID_SV = idesc_bf16_f32(D, DV, 1, 1);
-      constexpr uint32_t ID_S1 = idesc_bf16_f32(D, 16, 1, 1);
-      const uint64_t dK = smem_desc_sw128(smem_u32(sK), kBox, 1024);
-      const uint64_t dV = smem_desc_sw128(smem_u32(sV), kBox, 1024);
-      const uint64_t d1 = smem_desc_sw128(smem_u32(sONES), kBox, 1024);
-      bool ok = true;
-      for (int i = 0; i < nchunks && ok; ++i) {
-        const int st = i % NS;
-        ok = mbar_wait(&xf[st], (i / NS) & 1, abort_flag, a.err, kWaitLimitNs);
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t kd = desc_advance(dK, st * KT), vd = desc_advance(dV, st * VT);
-#pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk) {
-          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t ad = desc_advance(kd, kk * 2048);
-          umma_f16_ss(tmem, ad, desc_advance(vd, kk * 2048), ID_SV, acc);
-          umma_f16_ss(tmem + DV, ad, desc_advance(d1, kk * 2048), ID_S1, acc);
-        }
-        umma_commit(&empty[st]);
-      }
-      umma_commit(s_full);
-      int dummy = 0;  // drain the tensor pipe before TMEM is released
-      mbar_wait(s_full, 0, &dummy, nullptr, kWaitLimitNs);
-    }
-  } else {
-    const int x = tid;
-    bool ok = true;
-    for (int i = 0; i < nchunks && ok; ++i) {
-      const int st = i % NS, c = c0 + i;
-      ok = mbar_wait(&full[st], (i / NS) & 1, abort_flag, a.err, kWaitLimitNs);
-      if (!ok) break;
-      const int valid = min(kChunk, ntok - c * kChunk);
-      xf_tile<D / 64>(sK + st * KT, valid, true, x);
-      if (valid < kChunk) xf_tile<DV / 64>(sV + st * VT, valid, false, x);
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (x == 0) mbar_arrive(&xf[st]);
-    }
-    // read the aggregate (M = 64 accumulator: row 16*w + l in lane l < 16
-    // of sub-partition w) and store it; an empty block stores zeros
-    if (ok) ok = mbar_wait(s_full, 0, abort_flag, a.err, kWaitLimitNs);
-    if (ok) {
-      tc_fence_after();
-      const uint32_t t = tmem + ((uint32_t)(warp * 32) << 16);
-      float c0v[32], c1v[32], zz[16];
-      tmem_ld32(t, c0v);
-      tmem_ld32(t + 32, c1v);
-      tmem_ld16(t + DV, zz);
-      tmem_wait_ld();
-      if (lane < 16) {
-        const int row = warp * 16 + lane;
-        float4* d4 = reinterpret_cast<float4*>(dst + row * DV);
-        const bool any = nchunks > 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          d4[q] = any ? make_float4(c0v[4 * q], c0v[4 * q + 1], c0v[4 * q + 2], c0v[4 * q + 3])
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          d4[8 + q] = any ? make_float4(c1v[4 * q], c1v[4 * q + 1], c1v[4 * q + 2], c1v[4 * q + 3])
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-        dst[D * DV + row] = any ? zz[0] : 0.0f;
-      }
-      tc_fence_before();
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 5) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 128);
-  }
-}
-
-// ========================================================================
 // Forward pass over one block per CTA.
 // ========================================================================
-constexpr int kThreads = 448;
-constexpr int NQ = 4, NKV = 3;
-constexpr int TM_P = 0, TM_ACC = kChunk, TM_DS = TM_ACC + 2 * ACCW, TM_COLS = 512;
-static_assert(TM_DS + 2 * ACCW <= TM_COLS, "TMEM budget");
+constexpr int kThreads = 512;
+constexpr int kXf = 192;  // transform threads (warps 0-5)
+constexpr int NQ = 4, NKV = 4;
+// two score tiles (item j uses j & 1), two accumulators, one dS tile
+constexpr int TM_P = 0, TM_ACC = 2 * kChunk, TM_DS = TM_ACC + 2 * ACCW, TM_COLS = 512;
+static_assert(TM_DS + ACCW <= TM_COLS, "TMEM budget");
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + NQ * QT;
-constexpr int OFF_V = OFF_K + NKV * KT;
-constexpr int OFF_SOP = OFF_V + NKV * VT;
-constexpr int OFF_ONES = OFF_SOP + SOPT;
-constexpr int OFF_BAR = OFF_ONES + ONEST;
-constexpr int NBARS = 3 * NQ + 3 * NKV + 2 + 2 + 2 * 2 + 2 * 2 + 1;
+constexpr int OFF_KV = OFF_Q + NQ * QT;  // stage st: [K][V] at st*KVT
+constexpr int OFF_ONES = OFF_KV + NKV * KVT;
+constexpr int OFF_SOP = OFF_ONES + ONEST;
+constexpr int OFF_BAR = OFF_SOP + SOPT;
+constexpr int NBARS = 3 * NQ + 3 * NKV + 2 * 2 + 2 + 2 + 2 * 2 + 1;
 constexpr int SMEM = OFF_BAR + NBARS * 8 + 16 + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
 
@@ -260,12 +109,12 @@ __device__ __forceinline__ Bars carve(uint8_t* base) {
   r.kv_full = b; b += NKV;
   r.kv_empty = b; b += NKV;
   r.kv_xf = b; b += NKV;
-  r.p_full = b++;
-  r.pb_full = b++;
+  r.p_full = b; b += 2;
+  r.pb_full = b; b += 2;
   r.sop_full = b++;
   r.sop_empty = b++;
-  r.ds_full = b; b += 2;
-  r.ds_empty = b; b += 2;
+  r.ds_full = b++;
+  r.ds_empty = b++;
   r.acc_full = b; b += 2;
   r.acc_empty = b; b += 2;
   r.drain = b++;
@@ -317,10 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool nc_from_ws = !causal && a.ws != nullptr;
 
   uint8_t* sQ = smem + OFF_Q;
-  uint8_t* sK = smem + OFF_K;
-  uint8_t* sV = smem + OFF_V;
+  uint8_t* sK = smem + OFF_KV;
+  uint8_t* sV = smem + OFF_KV + KT;
   uint8_t* sSOP = smem + OFF_SOP;
-  uint8_t* sONES = smem + OFF_ONES;
   Bars bars = carve(smem + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + NBARS * 8);
 
@@ -336,29 +184,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.kv_empty[i], 1);
       mbar_init(&bars.kv_xf[i], 1);
     }
-    mbar_init(bars.p_full, 1);
-    mbar_init(bars.pb_full, 1);
     mbar_init(bars.sop_full, 1);
     mbar_init(bars.sop_empty, 1);
+    mbar_init(bars.ds_full, 1);
+    mbar_init(bars.ds_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.ds_full[i], 1);
-      mbar_init(&bars.ds_empty[i], 1);
+      mbar_init(&bars.p_full[i], 1);
+      mbar_init(&bars.pb_full[i], 1);
       mbar_init(&bars.acc_full[i], 1);
       mbar_init(&bars.acc_empty[i], 1);
     }
     mbar_init(bars.drain, 1);
     fence_mbar_init();
   }
-  init_ones_block(sONES, tid, kThreads);
+  init_ones_block(smem + OFF_ONES, tid, kThreads);
   fence_proxy_async_smem();
-  if (warp == 13) tmem_alloc(tmem_slot, TM_COLS);
+  if (warp == 15) tmem_alloc(tmem_slot, TM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int* abort_flag = &s_abort;
 
-  if (warp == 12) {
+  if (warp == 14) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -371,8 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&bars.kv_empty[st], ((r / NKV) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
           return false;
         mbar_arrive_expect_tx(&bars.kv_full[st], KT + VT);
-        tma_load_3d(sK + st * KT, &tm_k, &bars.kv_full[st], 0, g, t0 + c * kChunk);
-        tma_load_3d(sV + st * VT, &tm_v, &bars.kv_full[st], 0, g, t0 + c * kChunk);
+        tma_load_3d(sK + st * KVT, &tm_k, &bars.kv_full[st], 0, g, t0 + c * kChunk);
+        tma_load_3d(sV + st * KVT, &tm_v, &bars.kv_full[st], 0, g, t0 + c * kChunk);
         ++kv_issued;
         return true;
       };
@@ -403,33 +251,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&bars.q_full[j % NQ], (j / NQ) & 1, &dummy, nullptr, kWaitLimitNs);
       }
     }
-  } else if (warp == 13) {
+  } else if (warp == 15) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t ID_P = idesc_bf16_f32(kChunk, kChunk, 0, 0);
-      constexpr uint32_t ID_SV = idesc_bf16_f32(D, DV, 1, 1);
-      constexpr uint32_t ID_S1 = idesc_bf16_f32(D, 16, 1, 1);
+      constexpr uint32_t ID_SV = idesc_bf16_f32(D, DV + 16, 1, 1);
       constexpr uint32_t ID_PV = idesc_bf16_f32(kChunk, DV, 0, 1);
       constexpr uint32_t ID_QS = idesc_bf16_f32(kChunk, DV + 16, 0, 1);
       // descriptor bases, advanced per stage / K step with one 64-bit add
       const uint64_t dQk = smem_desc_sw128(smem_u32(sQ), 16, 1024);      // K-major
       const uint64_t dKk = smem_desc_sw128(smem_u32(sK), 16, 1024);      // K-major
       const uint64_t dKmn = smem_desc_sw128(smem_u32(sK), kBox, 1024);   // MN-major
-      const uint64_t dVmn = smem_desc_sw128(smem_u32(sV), kBox, 1024);   // MN-major
-      const uint64_t d1 = smem_desc_sw128(smem_u32(sONES), kBox, 1024);
+      const uint64_t dVmn = smem_desc_sw128(smem_u32(sV), kBox, 1024);   // MN-major V
+      const uint32_t ones = smem_u32(smem + OFF_ONES);
       const uint64_t dSop = smem_desc_sw128(smem_u32(sSOP), D * kRowBytes, 1024);
       bool ok = true;
       // dS (or the running S for the non-causal state pass) = phi(K)^T [V | 1]
       auto issue_ds = [&](int r, uint32_t t_ds, bool accumulate) {
         const int st = r % NKV;
-        const uint64_t ka = desc_advance(dKmn, st * KT), vb = desc_advance(dVmn, st * VT);
+        // [V | 1]: the second 64-column group is the shared ones block
+        const uint32_t va = smem_u32(sV) + st * KVT;
+        const uint64_t ka = desc_advance(dKmn, st * KVT), vb = smem_desc_sw128(va, ones - va, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk) {
-          const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
-          const uint64_t ad = desc_advance(ka, kk * 2048);
-          umma_f16_ss(t_ds, ad, desc_advance(vb, kk * 2048), ID_SV, acc);
-          umma_f16_ss(t_ds + DV, ad, desc_advance(d1, kk * 2048), ID_S1, acc);
-        }
+        for (int kk = 0; kk < kChunk / 16; ++kk)
+          umma_f16_ss(t_ds, desc_advance(ka, kk * 2048), desc_advance(vb, kk * 2048), ID_SV,
+                      (accumulate || kk > 0) ? 1u : 0u);
       };
       // Acc (+)= phi(Q) [S | z 0 ..]
       auto issue_qs = [&](uint32_t t_acc, int qs, bool accumulate) {
@@ -440,64 +286,69 @@ __global__ void __launch_bounds__(kThreads, 1)
                       desc_advance(dSop, kk * 2048), ID_QS, (accumulate || kk > 0) ? 1u : 0u);
       };
       if (causal) {
+        // dS of chunk r (single TMEM buffer: the state warpgroup drains it)
         auto state_mma = [&](int r) -> bool {
-          const int b = r & 1;
           if (!mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs) ||
-              !mbar_wait(&bars.ds_empty[b], ((r >> 1) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+              !mbar_wait(bars.ds_empty, (r & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
             return false;
           tc_fence_after();
-          issue_ds(r, tmem + TM_DS + b * ACCW, false);
-          umma_commit(&bars.ds_full[b]);
+          issue_ds(r, tmem + TM_DS, false);
+          umma_commit(bars.ds_full);
           return true;
         };
-        ok = state_mma(0);
-        for (int r = 0; r < Ri && ok; ++r) {
-          const uint64_t kd = desc_advance(dKk, (r % NKV) * KT);
-          const uint64_t vd = desc_advance(dVmn, (r % NKV) * VT);
-          for (int h = 0; h < G && ok; ++h) {
-            const int j = r * G + h, qs = j % NQ, as = j & 1;
-            const uint64_t qd = desc_advance(dQk, qs * QT);
-            const uint32_t t_acc = tmem + TM_ACC + as * ACCW;
-            // The previous item's score tile was read by its P V MMAs,
-            // issued before this one: the tensor pipe runs them in order.
-            ok = mbar_wait(&bars.q_xf[qs], (j / NQ) & 1, abort_flag, a.err, kWaitLimitNs);
-            if (!ok) break;
-            tc_fence_after();
+        // score tile of item j into TMEM buffer j & 1.  The buffer last held
+        // item j-2, whose P V MMAs were issued before this: the tensor pipe
+        // runs them in order.
+        auto score_mma = [&](int j) -> bool {
+          const int r = j / G, qs = j % NQ;
+          if (!mbar_wait(&bars.q_xf[qs], (j / NQ) & 1, abort_flag, a.err, kWaitLimitNs) ||
+              !mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs))
+            return false;
+          tc_fence_after();
+          const uint64_t qd = desc_advance(dQk, qs * QT);
+          const uint64_t kd = desc_advance(dKk, (r % NKV) * KVT);
+          const uint32_t t_p = tmem + TM_P + (j & 1) * kChunk;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t o = (kk >> 2) * kBox + (kk & 3) * 32;
-              umma_f16_ss(tmem + TM_P, desc_advance(qd, o), desc_advance(kd, o), ID_P,
-                          kk > 0 ? 1u : 0u);
-            }
-            umma_commit(bars.p_full);
-            // the next chunk's state MMA, after the score MMA so that the
-            // score tile does not wait for the next K tile
-            if (h == 0 && r + 1 < Ri) {
-              ok = state_mma(r + 1);
-              if (!ok) break;
-            }
-            ok = mbar_wait(bars.pb_full, j & 1, abort_flag, a.err, kWaitLimitNs) &&
-                 mbar_wait(&bars.acc_empty[as], ((j >> 1) & 1) ^ 1, abort_flag, a.err,
-                           kWaitLimitNs);
-            if (!ok) break;
-            tc_fence_after();
-            // P V: bf16 scores from TMEM, 16 keys (8 columns) per MMA.  The
-            // normaliser column was initialised with the score row sums.
-#pragma unroll
-            for (int kk = 0; kk < kChunk / 16; ++kk)
-              umma_f16_ts(t_acc, tmem + TM_P + kk * 8, desc_advance(vd, kk * 2048), ID_PV,
-                          kk > 0 ? 1u : 0u);
-            if (h == G - 1) umma_commit(&bars.kv_empty[r % NKV]);
-            if (h == 0) {
-              ok = mbar_wait(bars.sop_full, r & 1, abort_flag, a.err, kWaitLimitNs);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            issue_qs(t_acc, qs, true);
-            umma_commit(&bars.acc_full[as]);
-            umma_commit(&bars.q_empty[qs]);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t o = (kk >> 2) * kBox + (kk & 3) * 32;
+            umma_f16_ss(t_p, desc_advance(qd, o), desc_advance(kd, o), ID_P, kk > 0 ? 1u : 0u);
           }
-          if (ok) umma_commit(bars.sop_empty);
+          umma_commit(&bars.p_full[j & 1]);
+          return true;
+        };
+        ok = score_mma(0) && state_mma(0);
+        for (int j = 0; j < n_items && ok; ++j) {
+          const int r = j / G, h = j % G, qs = j % NQ, as = j & 1;
+          // the next item's score tile first: its mask then overlaps this
+          // item's P V and phi(Q)[S|z] MMAs
+          if (j + 1 < n_items) {
+            ok = score_mma(j + 1);
+            if (ok && (j + 1) % G == 0) ok = state_mma((j + 1) / G);
+            if (!ok) break;
+          }
+          const uint64_t vd = desc_advance(dVmn, (r % NKV) * KVT);
+          const uint32_t t_acc = tmem + TM_ACC + as * ACCW;
+          ok = mbar_wait(&bars.pb_full[as], (j >> 1) & 1, abort_flag, a.err, kWaitLimitNs) &&
+               mbar_wait(&bars.acc_empty[as], ((j >> 1) & 1) ^ 1, abort_flag, a.err,
+                         kWaitLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+          // P V: bf16 scores from TMEM, 16 keys (8 columns) per MMA.  The
+          // normaliser column was initialised with the score row sums.
+#pragma unroll
+          for (int kk = 0; kk < kChunk / 16; ++kk)
+            umma_f16_ts(t_acc, tmem + TM_P + as * kChunk + kk * 8, desc_advance(vd, kk * 2048),
+                        ID_PV, kk > 0 ? 1u : 0u);
+          if (h == G - 1) umma_commit(&bars.kv_empty[r % NKV]);
+          if (h == 0) {
+            ok = mbar_wait(bars.sop_full, r & 1, abort_flag, a.err, kWaitLimitNs);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          issue_qs(t_acc, qs, true);
+          umma_commit(&bars.acc_full[as]);
+          umma_commit(&bars.q_empty[qs]);
+          if (h == G - 1) umma_commit(bars.sop_empty);
         }
       } else {
         if (!nc_from_ws) {
@@ -508,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_ds(r, tmem + TM_DS, r > 0);
             umma_commit(&bars.kv_empty[r % NKV]);
           }
-          if (ok) umma_commit(&bars.ds_full[0]);
+          if (ok) umma_commit(bars.ds_full);
         }
         if (ok) ok = mbar_wait(bars.sop_full, 0, abort_flag, a.err, kWaitLimitNs);
         for (int j = 0; j < n_items && ok; ++j) {
@@ -527,19 +378,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       int dummy = 0;
       mbar_wait(bars.drain, 0, &dummy, nullptr, kWaitLimitNs);
     }
-  } else if (warp < 4) {
-    // ----------------------------------------------- transform warpgroup
-    const int x = tid;
+  } else if (warp < 6) {
+    // ---------------------------------------------- transform warps
+    const int x = tid;  // 0..191
     bool ok = true;
     auto xf_kv = [&](int r) -> bool {
       const int st = r % NKV, c = c0 + r;
       if (!mbar_wait(&bars.kv_full[st], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs))
         return false;
       const int valid = min(kChunk, ntok - c * kChunk);
-      xf_tile<D / 64>(sK + st * KT, valid, true, x);
-      if (valid < kChunk) xf_tile<DV / 64>(sV + st * VT, valid, false, x);
+      xf_tile<D / 64, kXf>(sK + st * KVT, valid, true, x);
+      if (valid < kChunk) xf_tile<DV / 64, kXf>(sV + st * KVT, valid, false, x);
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
+      named_bar_sync(1, kXf);
       if (x == 0) mbar_arrive(&bars.kv_xf[st]);
       return true;
     };
@@ -547,31 +398,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = j % NQ;
       if (!mbar_wait(&bars.q_full[st], (j / NQ) & 1, abort_flag, a.err, kWaitLimitNs))
         return false;
-      xf_tile<D / 64>(sQ + st * QT, kChunk, true, x);
+      xf_tile<D / 64, kXf>(sQ + st * QT, kChunk, true, x);
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
+      named_bar_sync(1, kXf);
       if (x == 0) mbar_arrive(&bars.q_xf[st]);
       return true;
     };
+    if (causal) {
+      ok = xf_kv(0);
+      for (int j = 0; j < n_items && ok; ++j) {
+        if (j % G == 0 && j > 0) ok = xf_kv(j / G);
+        if (ok) ok = xf_q(j);
+      }
+    } else {
+      if (!nc_from_ws)
+        for (int r = 0; r < Ri && ok; ++r) ok = xf_kv(r);
+      for (int j = 0; j < n_items && ok; ++j) ok = xf_q(j);
+    }
+  } else if (warp < 10) {
+    // ---------------------------------------------------- mask warpgroup
+    const int x = tid - 192, sp = warp & 3;
+    const int row = sp * 32 + lane;  // TMEM lane == chunk row
+    const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+    bool ok = true;
     // causal mask and bf16 rounding of the score tile, in place in TMEM:
     // fp32 columns [32b, 32b+32) become packed bf16 columns [16b, 16b+16),
     // which only overwrites columns this thread has already read; the row
-    // sum of the rounded scores initialises the accumulator's normaliser
+    // sum of the masked scores initialises the accumulator's normaliser
     auto mask_p = [&](int j) -> bool {
       const int as = j & 1;
-      if (!mbar_wait(bars.p_full, j & 1, abort_flag, a.err, kWaitLimitNs) ||
+      if (!mbar_wait(&bars.p_full[as], (j >> 1) & 1, abort_flag, a.err, kWaitLimitNs) ||
           !mbar_wait(&bars.acc_empty[as], ((j >> 1) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
         return false;
       tc_fence_after();
-      const uint32_t lane_sel = (uint32_t)(warp * 32) << 16;
-      const uint32_t t_p = tmem + TM_P + lane_sel;
-      const int row = x;
+      const uint32_t lane_sel = (uint32_t)(sp * 32) << 16;
+      const uint32_t t_p = tmem + TM_P + as * kChunk + lane_sel;
       float rs = 0.0f;
 #pragma unroll
       for (int b2 = 0; b2 < kChunk / 64; ++b2) {
         // two 32-column blocks per TMEM round trip
         float r0[32], r1[32];
-        const bool h0 = 2 * b2 <= warp, h1 = 2 * b2 + 1 <= warp;  // warp-uniform
+        const bool h0 = 2 * b2 <= sp, h1 = 2 * b2 + 1 <= sp;  // warp-uniform
         if (h0) tmem_ld32(t_p + (2 * b2) * 32, r0);
         if (h1) tmem_ld32(t_p + (2 * b2 + 1) * 32, r1);
         if (h0) tmem_wait_ld();
@@ -581,13 +448,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float* r = half ? r1 : r0;
           const bool have = half ? h1 : h0;
           uint32_t pk[16];
+          if (!have) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float lo = (!have || b * 32 + 2 * e > row) ? 0.0f : r[2 * e];
-            const float hi = (!have || b * 32 + 2 * e + 1 > row) ? 0.0f : r[2 * e + 1];
-            pk[e] = pack_bf16x2(lo, hi);
-            const float2 rr = unpack_bf16x2(pk[e]);
-            rs += rr.x + rr.y;
+            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+          } else if (b < sp) {  // block entirely left of the diagonal
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              pk[e] = pack_bf16x2(r[2 * e], r[2 * e + 1]);
+              rs += r[2 * e] + r[2 * e + 1];
+            }
+          } else {  // the diagonal block
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float lo = (b * 32 + 2 * e > row) ? 0.0f : r[2 * e];
+              const float hi = (b * 32 + 2 * e + 1 > row) ? 0.0f : r[2 * e + 1];
+              pk[e] = pack_bf16x2(lo, hi);
+              rs += lo + hi;
+            }
           }
           tmem_st16(t_p + b * 16, pk);
         }
@@ -595,33 +472,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st1(tmem + TM_ACC + as * ACCW + DV + lane_sel, __float_as_uint(rs));
       tmem_wait_st();
       tc_fence_before();
-      named_bar_sync(1, 128);
-      if (x == 0) mbar_arrive(bars.pb_full);
+      named_bar_sync(2, 128);
+      if (x == 0) mbar_arrive(&bars.pb_full[as]);
       return true;
     };
-    if (causal) {
-      ok = xf_kv(0);
-      for (int r = 0; r < Ri && ok; ++r) {
-        for (int h = 0; h < G && ok; ++h) {
-          ok = xf_q(r * G + h);
-          if (ok && h == 0 && r + 1 < Ri) ok = xf_kv(r + 1);  // next K while P runs
-          if (ok) ok = mask_p(r * G + h);
-        }
-      }
-    } else {
-      if (!nc_from_ws)
-        for (int r = 0; r < Ri && ok; ++r) ok = xf_kv(r);
-      for (int j = 0; j < n_items && ok; ++j) ok = xf_q(j);
-    }
-  } else if (warp < 8) {
-    // ----------------------------------------------- epilogue warpgroup
-    const int x = tid - 128, sp = warp & 3;
-    const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
-    bool ok = true;
-    for (int j = 0; j < n_items && ok; ++j) {
+    auto epilogue = [&](int j) -> bool {
       const int r = j / G, h = j % G, as = j & 1, c = c0 + r;
-      ok = mbar_wait(&bars.acc_full[as], (j >> 1) & 1, abort_flag, a.err, kWaitLimitNs);
-      if (!ok) break;
+      if (!mbar_wait(&bars.acc_full[as], (j >> 1) & 1, abort_flag, a.err, kWaitLimitNs))
+        return false;
       tc_fence_after();
       const uint32_t t_acc = tmem + TM_ACC + as * ACCW + lane_base;
       float den[16], n0[32], n1[32];
@@ -634,9 +492,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (x == 0) mbar_arrive(&bars.acc_empty[as]);
       const float inv = 1.0f / (den[0] + a.eps);
       const int valid = min(kChunk, ntok - c * kChunk);
-      if (x < valid) {
+      if (row < valid) {
         __nv_bfloat16* orow =
-            a.out + ((size_t)(t0 + c * kChunk + x) * a.Hq + (size_t)(g * G + h)) * DV;
+            a.out + ((size_t)(t0 + c * kChunk + row) * a.Hq + (size_t)(g * G + h)) * DV;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           *reinterpret_cast<uint4*>(orow + q4 * 8) =
@@ -651,17 +509,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                          pack_bf16x2(n1[q4 * 8 + 6] * inv, n1[q4 * 8 + 7] * inv));
         }
       }
+      return true;
+    };
+    // the mask of item j+1 goes before the epilogue of item j: the mask is on
+    // the path to the next MMAs, the epilogue only drains
+    if (causal) {
+      if (n_items > 0) ok = mask_p(0);
+      for (int j = 0; j < n_items && ok; ++j) {
+        if (j + 1 < n_items) ok = mask_p(j + 1);
+        if (ok) ok = epilogue(j);
+      }
+    } else {
+      for (int j = 0; j < n_items && ok; ++j) ok = epilogue(j);
     }
-  } else if (warp < 12) {
+  } else if (warp < 14) {
     // -------------------------------------------------- state warpgroup
     // dS is an M=64 accumulator: state row a = 16*sp + l lives in lane l < 16
     // of TMEM sub-partition sp; that thread owns row a of the running state.
-    const int y = tid - 256, sp = warp & 3;
+    const int y = tid - 320, sp = warp & 3;
     const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     const bool has_row = lane < 16;
     const int row = sp * 16 + lane;
     bool ok = true;
-    float T[DV], Tz = 0.0f;
+    float T[DV], Tz = 0.0f;  // this thread's row of the running [S|z]
 #pragma unroll
     for (int e = 0; e < DV; ++e) T[e] = 0.0f;
     // carry into this block: the aggregates of the earlier blocks (causal),
@@ -690,39 +560,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (y == 0) mbar_arrive(bars.sop_full);
       return true;
     };
-    auto add_ds = [&](int b) {
-      const uint32_t t = tmem + TM_DS + b * ACCW + lane_base;
-      float c0v[32], c1v[32], zz[16];
-      tmem_ld32(t, c0v);
-      tmem_ld32(t + 32, c1v);
+    auto add_ds = [&]() {
+      const uint32_t t = tmem + TM_DS + lane_base;
+#pragma unroll
+      for (int half = 0; half < DV / 32; ++half) {
+        float cv[32];
+        tmem_ld32(t + half * 32, cv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) T[half * 32 + e] += cv[e];
+      }
+      float zz[16];
       tmem_ld16(t + DV, zz);
       tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        T[e] += c0v[e];
-        T[32 + e] += c1v[e];
-      }
       Tz += zz[0];
     };
     if (causal) {
+      // [S|z]_<c+1 is published as soon as chunk c's phi(Q)[S|z] MMAs have
+      // released the operand
+      ok = publish_sop(0);
       for (int r = 0; r < Ri && ok; ++r) {
-        ok = publish_sop(r);  // [S|z]_<c does not need this chunk's dS
-        if (!ok) break;
-        const int b = r & 1;
-        ok = mbar_wait(&bars.ds_full[b], (r >> 1) & 1, abort_flag, a.err, kWaitLimitNs);
+        ok = mbar_wait(bars.ds_full, r & 1, abort_flag, a.err, kWaitLimitNs);
         if (!ok) break;
         tc_fence_after();
-        add_ds(b);
+        add_ds();
         tc_fence_before();
         named_bar_sync(3, 128);
-        if (y == 0) mbar_arrive(&bars.ds_empty[b]);
+        if (y == 0) mbar_arrive(bars.ds_empty);
+        if (r + 1 < Ri) ok = publish_sop(r + 1);
       }
     } else {
       if (!nc_from_ws) {
-        ok = mbar_wait(&bars.ds_full[0], 0, abort_flag, a.err, kWaitLimitNs);
+        ok = mbar_wait(bars.ds_full, 0, abort_flag, a.err, kWaitLimitNs);
         if (ok) {
           tc_fence_after();
-          add_ds(0);
+          add_ds();
           tc_fence_before();
         }
       }
@@ -732,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 13) {
+  if (warp == 15) {
     tc_fence_after();
     tmem_dealloc(tmem, TM_COLS);
   }
@@ -742,61 +614,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool block_supported(const FwdLaunch& p) { return p.d == 64 && p.dv == 64; }
 
-// Workspace of the block aggregates (none with one block per sequence).
-size_t block_workspace_bytes(const FwdLaunch& p, int nb) {
-  return nb > 1 ? (size_t)p.B * p.Hkv * nb * E * sizeof(float) : 0;
-}
-
-// Blocks per sequence: enough CTAs to cover the SMs about once.
-int block_count(const FwdLaunch& p, int num_sms) {
-  const char* force = getenv("LT_BLOCKS");
-  const int nc = p.cu_seqlens ? 0 : (p.N + kChunk - 1) / kChunk;
-  if (p.cu_seqlens) return 1;  // packed: one block per (sequence, KV head)
-  if (force) {
-    const int f = atoi(force);
-    return f < 1 ? 1 : (f > nc ? nc : f);
-  }
-  const int lanes = p.B * p.Hkv;
-  int nb = num_sms / (lanes > 0 ? lanes : 1);
-  if (nb < 1) nb = 1;
-  if (nb > nc) nb = nc;
-  return nb;
-}
-
-cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream) {
+cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, const float* ws,
+                                  cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
   if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
       !make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64) ||
       !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64))
     return cudaErrorInvalidValue;
-  const int nc = p.cu_seqlens ? 0 : (p.N + kChunk - 1) / kChunk;
   BlockArgs a;
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
   a.cu_seqlens = p.cu_seqlens;
-  a.ws = nb > 1 ? ws : nullptr;
+  a.ws = nb > 1 ? const_cast<float*>(ws) : nullptr;
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
   a.N = p.N;
   a.G = p.Hq / p.Hkv;
   a.causal = p.causal;
   a.nb = nb;
-  a.bc = nb > 1 ? (nc + nb - 1) / nb : (1 << 30);
+  a.bc = block_chunks(p, nb);
   a.eps = p.eps;
   a.total_tokens = (int)p.total_tokens;
   a.err = p.err;
-  cudaError_t e;
-  if (nb > 1) {
-    auto sk = lt_block_state_kernel;
-    e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ST_SMEM);
-    if (e != cudaSuccess) return e;
-    // causal: the last block's aggregate is never needed
-    const int nstate = p.causal ? nb - 1 : nb;
-    sk<<<dim3(nstate, p.Hkv, p.B), kStThreads, ST_SMEM, stream>>>(tk, tv, a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
   auto fk = lt_block_fwd_kernel;
-  e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  cudaError_t e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
   fk<<<dim3(nb, p.Hkv, p.B), kThreads, SMEM, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();

@@ -16,9 +16,12 @@
 // it is read once, rounded to bf16 and staged in shared memory as the B
 // operand of phi(Q_c) [S|z]_<c.
 //
-// One CTA owns one (sequence, KV head) pair and walks its chunks in order;
-// every query head of the KV head's group is served from the same K/V tiles
-// and the same state.  Warp roles (320 threads):
+// One CTA owns one block of consecutive chunks of one (sequence, KV head)
+// pair and walks them in order; every query head of the KV head's group is
+// served from the same K/V tiles and the same state.  With more than one
+// block per sequence the state of a block starts from the carry summed from
+// the block aggregates of the state launch (earlier blocks when causal,
+// every block when not), written into the TMEM state accumulator.  Warp roles (320 threads):
 //   warps 0-3  transform warpgroup: phi applied in place to the TMA-loaded
 //              K and Q tiles, tail rows zeroed; causal mask of the score
 //              tile, conversion to bf16, staging as the A operand of P V.
@@ -27,8 +30,9 @@
 //   warp 8     TMA producer.
 //   warp 9     TMEM allocator and single-thread MMA issuer.
 // Non-causal mode (phi(Q)(phi(K)^T V) normalised the same way): first the
-// state over all chunks (K, V only), then every output row as
-// phi(Q_i) [S|z]_n (Q only).
+// state over all chunks (K, V only; taken from the block aggregates when the
+// sequence is split into blocks), then every output row as phi(Q_i) [S|z]_n
+// (Q only).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -130,8 +134,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int g = blockIdx.x;  // KV head
-  const int s = blockIdx.y;  // sequence (batch row or packed sequence)
+  const int blk = blockIdx.x;  // block of chunks within the sequence
+  const int g = blockIdx.y;    // KV head
+  const int s = blockIdx.z;    // sequence (batch row or packed sequence)
 
   // sequence geometry
   int t0, n;
@@ -147,9 +152,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     t0 = s * a.N;
     n = a.N;
   }
+  {
+    // this CTA's block: chunks [blk * bc, min((blk + 1) * bc, nc_seq))
+    const int nc_seq = (n + kChunk - 1) / kChunk;
+    const int c0 = blk * a.bc;  // a.bc is huge only when there is one block
+    if (c0 >= nc_seq) return;
+    const int nchunks = min(nc_seq - c0, a.bc);
+    t0 += c0 * kChunk;
+    n = min(n - c0 * kChunk, nchunks * kChunk);
+  }
   if (n <= 0) return;
   const int nc = (n + kChunk - 1) / kChunk;
   const int G = a.G;
+  // has_carry: the state starts from the block aggregates rather than zero;
+  // carried_state: non-causal and the whole state comes from them
+  const bool has_carry = a.ws != nullptr && (!a.causal || blk > 0);
+  const bool carried_state = a.ws != nullptr && !a.causal;
   const int n_items = nc * G;
 
   uint8_t* sQ = smem + K::OFF_Q;
@@ -244,7 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) ok = load_q(i);
         }
       } else {
-        for (int c = 0; c < nc && ok; ++c) ok = load_kv(c);
+        if (!carried_state)
+          for (int c = 0; c < nc && ok; ++c) ok = load_kv(c);
         for (int i = 0; i < n_items && ok; ++i) ok = load_q(i);
       }
       if (!ok) {
@@ -339,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                  mbar_wait(bars.s_empty, c & 1, abort_flag, a.err, kWaitLimitNs);
             if (!ok) break;
             tc_fence_after();
-            issue_state(c, c > 0);
+            issue_state(c, c > 0 || has_carry);
             umma_commit(bars.s_full);
           }
           const int qs = i % K::NQ, ps = i % K::NP;
@@ -362,15 +381,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok && n_items > 0) ok = issue_acc(n_items - 1);
       } else {
-        for (int c = 0; c < nc && ok; ++c) {
-          const int st = c % K::NKV;
-          ok = mbar_wait(&bars.kv_xf[st], (c / K::NKV) & 1, abort_flag, a.err, kWaitLimitNs);
-          if (!ok) break;
-          tc_fence_after();
-          issue_state(c, c > 0);
-          umma_commit(&bars.kv_empty[st]);
+        if (!carried_state) {
+          for (int c = 0; c < nc && ok; ++c) {
+            const int st = c % K::NKV;
+            ok = mbar_wait(&bars.kv_xf[st], (c / K::NKV) & 1, abort_flag, a.err, kWaitLimitNs);
+            if (!ok) break;
+            tc_fence_after();
+            issue_state(c, c > 0);
+            umma_commit(&bars.kv_empty[st]);
+          }
+          if (ok) umma_commit(bars.s_full);
         }
-        if (ok) umma_commit(bars.s_full);
         if (ok) ok = mbar_wait(&bars.sop_full[0], 0, abort_flag, a.err, kWaitLimitNs);
         for (int i = 0; i < n_items && ok; ++i) {
           const int qs = i % K::NQ, as = i % K::NA;
@@ -475,7 +496,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok && n_items > 0) ok = mask_p(n_items - 1);
     } else {
-      for (int c = 0; c < nc && ok; ++c) ok = xf_kv(c);
+      if (!carried_state)
+        for (int c = 0; c < nc && ok; ++c) ok = xf_kv(c);
       for (int i = 0; i < n_items && ok; ++i) ok = xf_q(i);
     }
   } else {
@@ -484,15 +506,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sp = warp & 3;          // TMEM sub-partition of this warp
     const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     bool ok = true;
-    // Stage [S|z] (fp32 TMEM, or zero) as the bf16 MN-major B operand.
+    // Stage [S|z] as the bf16 MN-major B operand, from zero, from the fp32
+    // TMEM state, or from the carry (the block aggregates summed in fp32; in
+    // causal mode also written into the TMEM state, which the state MMAs of
+    // this block then accumulate onto).
     // For D == 64 the state tile is an M=64 accumulator: rows 16*sp + l
     // live in lanes l < 16 of sub-partition sp.
     // use: how many times this Sop buffer was staged before (phase parity)
-    auto stage_state = [&](int buf, int use, bool zero, int s_parity) -> bool {
+    enum { kFromZero, kFromTmem, kFromCarry };
+    auto stage_state = [&](int buf, int use, int src, int s_parity) -> bool {
       const bool has_row = (D == 128) || (lane < 16);
       const int row = (D == 128) ? x : (sp * 16 + lane);
       float r[DV + 16];
-      if (!zero) {
+      if (src == kFromTmem) {
         if (!mbar_wait(bars.s_full, s_parity, abort_flag, a.err, kWaitLimitNs)) return false;
         tc_fence_after();
         const uint32_t t_s = tmem + K::TM_S + lane_base;
@@ -513,6 +539,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
 #pragma unroll
         for (int e = 0; e < DV + 16; ++e) r[e] = 0.0f;
+        if (src == kFromCarry) {
+          if (has_row) {
+            constexpr int E = D * DV + D;
+            const float* base = a.ws + (size_t)(s * a.Hkv + g) * a.nb * E;
+            const int nsum = a.causal ? blk : a.nb;
+            for (int bb = 0; bb < nsum; ++bb) {
+              const float4* r4 = reinterpret_cast<const float4*>(base + (size_t)bb * E + row * DV);
+#pragma unroll
+              for (int q4 = 0; q4 < DV / 4; ++q4) {
+                const float4 v4 = r4[q4];
+                r[4 * q4] += v4.x;
+                r[4 * q4 + 1] += v4.y;
+                r[4 * q4 + 2] += v4.z;
+                r[4 * q4 + 3] += v4.w;
+              }
+              r[DV] += base[(size_t)bb * E + D * DV + row];
+            }
+          }
+          if (a.causal) {
+            const uint32_t t_s = tmem + K::TM_S + lane_base;
+#pragma unroll
+            for (int cb = 0; cb < (DV + 16) / 16; ++cb) {
+              uint32_t w16[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(r[cb * 16 + e]);
+              tmem_st16(t_s + cb * 16, w16);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+          }
+        }
       }
       named_bar_sync(2, 128);
       if (x == 0) mbar_arrive(bars.s_empty);
@@ -576,9 +633,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // buffer frees only after the chunk's last accumulator MMA, so staging
       // waits until every earlier epilogue of the chunk has released TMEM.
       auto stage_next = [&](int c) -> bool {
-        return stage_state((c + 1) % K::NSOP, (c + 1) / K::NSOP, false, c & 1);
+        return stage_state((c + 1) % K::NSOP, (c + 1) / K::NSOP, kFromTmem, c & 1);
       };
-      ok = stage_state(0, 0, true, 0);
+      ok = stage_state(0, 0, has_carry ? kFromCarry : kFromZero, 0);
       for (int c = 0; c < nc && ok; ++c) {
         const bool early = K::NSOP >= 2;
         if (early && c + 1 < nc) ok = stage_next(c);
@@ -589,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else {
       // the state is complete once every chunk has been accumulated
-      ok = stage_state(0, 0, false, 0);
+      ok = stage_state(0, 0, carried_state ? kFromCarry : kFromTmem, 0);
       for (int i = 0; i < n_items && ok; ++i) ok = epilogue(i);
     }
   }
@@ -603,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, int DV>
-cudaError_t launch_fwd(const FwdLaunch& p, cudaStream_t stream) {
+cudaError_t launch_fwd(const FwdLaunch& p, int nb, const float* ws, cudaStream_t stream) {
   using K = Cfg<D, DV>;
   CUtensorMap tq, tk, tv;
   if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
@@ -616,6 +673,9 @@ cudaError_t launch_fwd(const FwdLaunch& p, cudaStream_t stream) {
   FwdArgs a;
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
   a.cu_seqlens = p.cu_seqlens;
+  a.ws = nb > 1 ? ws : nullptr;
+  a.nb = nb;
+  a.bc = block_chunks(p, nb);
   a.B = p.B;
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
@@ -625,44 +685,72 @@ cudaError_t launch_fwd(const FwdLaunch& p, cudaStream_t stream) {
   a.eps = p.eps;
   a.total_tokens = (int)p.total_tokens;
   a.err = p.err;
-  dim3 grid(p.Hkv, p.B);
+  dim3 grid(nb, p.Hkv, p.B);
   kern<<<grid, kThreads, K::SMEM, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_fwd_bf16(const FwdLaunch& p, cudaStream_t stream) {
-  // LT_KERNEL selects a kernel for every shape it supports (ablations):
-  //   seq      one CTA per (sequence, KV head), sequential chunks
-  //   cluster  sequence split over a thread-block cluster (d = dv = 64)
-  const char* force = getenv("LT_KERNEL");
-  const bool seq = force && force[0] == 's';
-  const bool cluster = force && force[0] == 'c';
-  if (cluster && split_supported(p)) return launch_fwd_bf16_split(p, stream);
-  if (!seq && block_supported(p)) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int nb = block_count(p, sms);
-    const size_t bytes = block_workspace_bytes(p, nb);
-    void* ws = nullptr;
-    if (bytes) {
-      cudaError_t e = cudaMallocAsync(&ws, bytes, stream);
-      if (e != cudaSuccess) return e;
-    }
-    cudaError_t e = launch_fwd_bf16_block(p, nb, static_cast<float*>(ws), stream);
-    if (ws) {
-      const cudaError_t f = cudaFreeAsync(ws, stream);
-      if (e == cudaSuccess) e = f;
-    }
-    return e;
-  }
-  if (p.d == 64 && p.dv == 64) return launch_fwd<64, 64>(p, stream);
-  if (p.d == 128 && p.dv == 128) return launch_fwd<128, 128>(p, stream);
-  if (p.d == 64 && p.dv == 128) return launch_fwd<64, 128>(p, stream);
-  if (p.d == 128 && p.dv == 64) return launch_fwd<128, 64>(p, stream);
+cudaError_t launch_fwd_bf16_seq(const FwdLaunch& p, int nb, const float* ws,
+                                cudaStream_t stream) {
+  if (p.d == 64 && p.dv == 64) return launch_fwd<64, 64>(p, nb, ws, stream);
+  if (p.d == 128 && p.dv == 128) return launch_fwd<128, 128>(p, nb, ws, stream);
+  if (p.d == 64 && p.dv == 128) return launch_fwd<64, 128>(p, nb, ws, stream);
+  if (p.d == 128 && p.dv == 64) return launch_fwd<128, 64>(p, nb, ws, stream);
   return cudaErrorInvalidValue;
+}
+
+// LT_KERNEL selects a forward kernel for every shape it supports (ablations):
+//   seq      the general kernel (one CTA per block of chunks) for d = dv = 64
+//            too; LT_BLOCKS=1 makes it fully sequential
+//   cluster  sequence split over a thread-block cluster (d = dv = 64)
+static bool forced(char c) {
+  const char* force = getenv("LT_KERNEL");
+  return force && force[0] == c;
+}
+
+cudaError_t launch_fwd_bf16_ws(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream) {
+  cudaError_t e = cudaSuccess;
+  if (nb > 1) {
+    e = launch_block_state(p, nb, ws, stream);
+    if (e != cudaSuccess) return e;
+  }
+  if (!forced('s') && block_supported(p)) return launch_fwd_bf16_block(p, nb, ws, stream);
+  return launch_fwd_bf16_seq(p, nb, ws, stream);
+}
+
+void plan_fwd_bf16(const FwdLaunch& p, int num_sms, int* nb, int* launches, size_t* ws_bytes) {
+  if (forced('c') && split_supported(p)) {
+    *nb = 1;
+    *launches = 1;
+    *ws_bytes = 0;
+    return;
+  }
+  *nb = block_count(p, num_sms);
+  *launches = *nb > 1 && (p.causal ? *nb - 1 : *nb) > 0 ? 2 : 1;
+  *ws_bytes = block_workspace_bytes(p, *nb);
+}
+
+cudaError_t launch_fwd_bf16(const FwdLaunch& p, cudaStream_t stream) {
+  if (forced('c') && split_supported(p)) return launch_fwd_bf16_split(p, stream);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int nb = 1, launches = 1;
+  size_t bytes = 0;
+  plan_fwd_bf16(p, sms, &nb, &launches, &bytes);
+  void* ws = nullptr;
+  if (bytes) {
+    cudaError_t e = cudaMallocAsync(&ws, bytes, stream);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = launch_fwd_bf16_ws(p, nb, static_cast<float*>(ws), stream);
+  if (ws) {
+    const cudaError_t f = cudaFreeAsync(ws, stream);
+    if (e == cudaSuccess) e = f;
+  }
+  return e;
 }
 
 }  // namespace lt

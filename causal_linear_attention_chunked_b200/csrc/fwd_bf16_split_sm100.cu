@@ -873,6 +873,9 @@ cudaError_t launch_fwd_bf16_split(const FwdLaunch& p, cudaStream_t stream) {
   const int nc = p.cu_seqlens ? 1 : (p.N + kChunk - 1) / kChunk;
   const int ncl = p.cu_seqlens ? 1 : choose_cluster(p.B * p.Hkv, nc, dev);
   FwdArgs a;
+  a.ws = nullptr;
+  a.nb = 1;
+  a.bc = 1 << 30;
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
   a.cu_seqlens = p.cu_seqlens;
   a.B = p.B;

@@ -20,12 +20,12 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 
 // phi in place over a [kChunk x (NBOX*64)] bf16 tile (rows of 128-byte
 // boxes, swizzled; phi is elementwise so the swizzle does not matter).
-// Rows >= valid are zeroed.  128 threads.
-template <int NBOX>
+// Rows >= valid are zeroed.  NT threads (tid in [0, NT)).
+template <int NBOX, int NT = 128>
 __device__ __forceinline__ void xf_tile(uint8_t* tile, int valid, bool apply_phi, int tid) {
   constexpr int kChunks = kChunk * NBOX * 8;  // 16-byte pieces
 #pragma unroll 4
-  for (int ch = tid; ch < kChunks; ch += 128) {
+  for (int ch = tid; ch < kChunks; ch += NT) {
     const int rem = ch % (kChunk * 8);
     const int row = rem >> 3;
     uint4* p = reinterpret_cast<uint4*>(tile + (ch / (kChunk * 8)) * kBox + rem * 16);
@@ -53,7 +53,10 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int jj) {
 struct FwdArgs {
   __nv_bfloat16* out;
   const int32_t* cu_seqlens;
+  const float* ws;  // block aggregates [sequence][KV head][nb][d*dv + d], or nullptr
   int B, Hq, Hkv, N, G, causal;
+  int nb;  // blocks per sequence
+  int bc;  // chunks per block
   float eps;
   int total_tokens;
   int* err;

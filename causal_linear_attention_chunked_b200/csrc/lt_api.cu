@@ -77,7 +77,7 @@ lt_status_t lt_linear_attn_fwd(const void* q, const void* k, const void* v, void
   if (!q || !k || !v || !out) return LT_ERR_INVALID_ARG;
   if (B <= 0 || H_q <= 0 || H_kv <= 0 || N <= 0) return LT_ERR_INVALID_ARG;
   if (H_q % H_kv != 0) return LT_ERR_INVALID_ARG;
-  if (B > 65535) return LT_ERR_INVALID_ARG;  // grid y extent
+  if (B > 65535 || H_kv > 65535) return LT_ERR_INVALID_ARG;  // grid y/z extents
   if (causal != 0 && causal != 1) return LT_ERR_INVALID_ARG;
   if (!(eps >= 0.0f) || !isfinite(eps)) return LT_ERR_INVALID_ARG;
   if (!width_ok(d) || !width_ok(dv)) return LT_ERR_UNSUPPORTED;
@@ -116,6 +116,46 @@ lt_status_t lt_linear_attn_fwd(const void* q, const void* k, const void* v, void
   const cudaError_t e = dtype == LT_BF16 ? lt::launch_fwd_bf16(p, (cudaStream_t)stream)
                                          : lt::launch_fwd_f32(p, (cudaStream_t)stream);
   return e == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status_t lt_linear_attn_fwd_plan(int B, int H_q, int H_kv, int N, int d, int dv, int causal,
+                                    int packed, lt_dtype_t dtype, int num_sms, int* blocks,
+                                    int* launches, size_t* workspace_bytes) {
+  if (dtype != LT_F32 && dtype != LT_BF16) return LT_ERR_UNSUPPORTED;
+  if (!blocks || !launches || !workspace_bytes) return LT_ERR_INVALID_ARG;
+  if (B <= 0 || H_q <= 0 || H_kv <= 0 || N <= 0 || H_q % H_kv != 0) return LT_ERR_INVALID_ARG;
+  if (B > 65535 || H_kv > 65535) return LT_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return LT_ERR_INVALID_ARG;
+  if (packed != 0 && packed != 1) return LT_ERR_INVALID_ARG;
+  if (!width_ok(d) || !width_ok(dv)) return LT_ERR_UNSUPPORTED;
+  const long long tokens = packed ? (long long)N : (long long)B * (long long)N;
+  if (tokens >= (1ll << 31)) return LT_ERR_INVALID_ARG;
+  if (dtype == LT_F32) {
+    *blocks = 1;
+    *launches = 1;
+    *workspace_bytes = 0;
+    return LT_OK;
+  }
+  if (num_sms <= 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return LT_ERR_CUDA;
+    }
+  }
+  lt::FwdLaunch p = {};
+  p.cu_seqlens = packed ? reinterpret_cast<const int32_t*>(16) : nullptr;  // only tested for null
+  p.B = B;
+  p.Hq = H_q;
+  p.Hkv = H_kv;
+  p.N = N;
+  p.d = d;
+  p.dv = dv;
+  p.causal = causal;
+  p.total_tokens = tokens;
+  lt::plan_fwd_bf16(p, num_sms, blocks, launches, workspace_bytes);
+  return LT_OK;
 }
 
 lt_status_t lt_linear_attn_decode_step(const void* q, const void* k, const void* v, float* S,

@@ -30,17 +30,34 @@ struct DecodeLaunch {
   int bf16;  // 1: bf16 q/k/v/out, 0: fp32
 };
 
+// bf16 forward: picks the block count, allocates the block workspace
+// (stream-ordered) and runs the state launch then the forward launch
 cudaError_t launch_fwd_bf16(const FwdLaunch& p, cudaStream_t stream);
+// what launch_fwd_bf16 does for p on a device with num_sms SMs: blocks per
+// sequence, kernel launches, workspace bytes
+void plan_fwd_bf16(const FwdLaunch& p, int num_sms, int* nb, int* launches, size_t* ws_bytes);
+// the same with a caller-provided workspace of at least
+// block_workspace_bytes(p, nb) bytes (nullptr when that is 0)
+cudaError_t launch_fwd_bf16_ws(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream);
 // d = dv = 64: sequence split over a thread-block cluster (or one CTA per
 // (sequence, KV head) for packed inputs)
 bool split_supported(const FwdLaunch& p);
 cudaError_t launch_fwd_bf16_split(const FwdLaunch& p, cudaStream_t stream);
-// d = dv = 64: block-parallel two-launch scan (block aggregates, then one CTA
-// per block); `ws` holds block_workspace_bytes(p, nb) bytes when nb > 1
-bool block_supported(const FwdLaunch& p);
+// Block-parallel scan.  A dense sequence is cut into nb blocks of
+// block_chunks(p, nb) chunks; the state launch writes each block's aggregate
+// phi(K)^T [V | 1] (fp32, d x dv then d) to the workspace and the forward
+// launch starts block b from the sum of the aggregates before it (causal) or
+// of all of them (non-causal).  nb = 1: no workspace, no state launch.
 int block_count(const FwdLaunch& p, int num_sms);
+int block_chunks(const FwdLaunch& p, int nb);
 size_t block_workspace_bytes(const FwdLaunch& p, int nb);
-cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream);
+cudaError_t launch_block_state(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream);
+// forward launches: d = dv = 64 specialised kernel; every width pair
+bool block_supported(const FwdLaunch& p);
+cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, const float* ws,
+                                  cudaStream_t stream);
+cudaError_t launch_fwd_bf16_seq(const FwdLaunch& p, int nb, const float* ws,
+                                cudaStream_t stream);
 cudaError_t launch_fwd_f32(const FwdLaunch& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeLaunch& p, cudaStream_t stream);
 

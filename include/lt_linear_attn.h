@@ -19,7 +19,13 @@
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers (cudaMalloc / cudaMallocAsync
  *     / managed memory) owned by the caller; the library keeps no reference
- *     to them after the call returns and allocates nothing.
+ *     to them after the call returns.
+ *   - Scratch memory: lt_linear_attn_fwd with LT_BF16 on a dense batch cuts
+ *     each sequence into blocks and, when there is more than one, allocates
+ *     a stream-ordered workspace on `stream` (cudaMallocAsync, released by
+ *     cudaFreeAsync on the same stream before the call returns) for the
+ *     per-block partial states; lt_linear_attn_fwd_plan() gives its size.
+ *     No other entry point allocates.
  *   - Layouts are token-major and dense (row-major, no padding):
  *       dense:   q [B][N][H_q][d],  k [B][N][H_kv][d],  v [B][N][H_kv][dv],
  *                out [B][N][H_q][dv]
@@ -39,6 +45,7 @@
 #ifndef LT_LINEAR_ATTN_H
 #define LT_LINEAR_ATTN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -74,8 +81,8 @@ typedef enum {
  * q, k, v   inputs of element type `dtype`, layouts above; 16-byte aligned.
  * out       output, same element type, layout [.][N][H_q][dv]; 16-byte
  *           aligned; must not overlap q, k or v.
- * B         dense: batch rows; packed: number of sequences.  B >= 1.
- * H_q, H_kv query and KV heads, H_kv >= 1, H_q a multiple of H_kv.
+ * B         dense: batch rows; packed: number of sequences.  1 <= B <= 65535.
+ * H_q, H_kv query and KV heads, 1 <= H_kv <= 65535, H_q a multiple of H_kv.
  * N         dense: tokens per row; packed: total tokens.  N >= 1 and the
  *           total token count (B*N dense, N packed) below 2^31.
  * d, dv     key and value widths, each 64 or 128.
@@ -89,12 +96,38 @@ typedef enum {
  * stream    CUDA stream to enqueue on.
  * dtype     LT_BF16 (tensor-core path) or LT_F32 (fp32 FMA path).
  *
+ * Evaluation (bf16): chunks of 128 tokens; the intra-chunk part as masked
+ * dense products and the inter-chunk part through the carried state
+ * ("Why Stream Wins at Ultra-Long Context", section 5.3: chunk-local work
+ * plus a carry).  A dense sequence is cut into blocks of consecutive chunks
+ * so that every SM has work: one launch writes each block's partial state
+ * to the workspace, a second runs the blocks from the carry.
+ *
  * Returns LT_OK when the work was enqueued.
  */
 LT_API lt_status_t lt_linear_attn_fwd(const void *q, const void *k, const void *v, void *out,
                                int B, int H_q, int H_kv, int N, int d, int dv, int causal,
                                float eps, const int32_t *cu_seqlens, lt_stream_t stream,
                                lt_dtype_t dtype);
+
+/*
+ * How lt_linear_attn_fwd evaluates a shape: blocks each sequence is cut
+ * into, kernel launches per call, and bytes of stream-ordered workspace the
+ * call allocates (0: none).  Host-only arithmetic, nothing is launched.
+ *
+ * B .. causal, dtype   as for lt_linear_attn_fwd.
+ * packed               1 when cu_seqlens will be passed (packed sequences
+ *                      run one block each), 0 for dense inputs.
+ * num_sms              SM count of the target device; <= 0 queries the
+ *                      current device (needs a working CUDA runtime).
+ * blocks, launches, workspace_bytes   outputs (non-NULL host pointers).
+ * Returns LT_OK, LT_ERR_INVALID_ARG / LT_ERR_UNSUPPORTED for arguments that
+ * lt_linear_attn_fwd would reject, LT_ERR_CUDA if the device query failed.
+ */
+LT_API lt_status_t lt_linear_attn_fwd_plan(int B, int H_q, int H_kv, int N, int d, int dv,
+                                           int causal, int packed, lt_dtype_t dtype,
+                                           int num_sms, int *blocks, int *launches,
+                                           size_t *workspace_bytes);
 
 /*
  * One recurrent decode step: the fixed-size state (S, z) plays the role of

@@ -57,6 +57,7 @@ FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every case fails before th
     (dict(dtype=7), 2),
     (dict(B=70000), 1),
     (dict(B=1 << 16, N=1 << 16), 1),
+    (dict(Hkv=70000, Hq=70000), 1),
 ])
 def test_fwd_rejects_invalid_arguments(case, expect):
     from causal_linear_attention_chunked_b200 import _binding as b
@@ -101,3 +102,45 @@ def test_oracle_and_library_share_no_code():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "lt_oracle" not in txt, f
+
+
+@pytest.mark.parametrize("shape,expect", [
+    # (B, H_q, H_kv, N, d, dv, causal, packed, dtype), num_sms = 148
+    ((2, 8, 8, 4096, 64, 64, 1, 0, 1), (9, 2, 2 * 8 * 9 * (64 * 64 + 64) * 4)),
+    ((1, 8, 8, 65536, 64, 64, 0, 0, 1), (18, 2, 8 * 18 * (64 * 64 + 64) * 4)),
+    ((2, 32, 8, 16384, 128, 128, 1, 0, 1), (9, 2, 2 * 8 * 9 * (128 * 128 + 128) * 4)),
+    ((1, 1, 1, 300, 64, 128, 1, 0, 1), (3, 2, 3 * (64 * 128 + 64) * 4)),   # capped by 3 chunks
+    ((1, 1, 1, 100, 64, 64, 1, 0, 1), (1, 1, 0)),                            # one chunk
+    ((64, 8, 8, 50000, 64, 64, 1, 1, 1), (1, 1, 0)),                         # packed
+    ((2, 8, 8, 4096, 64, 64, 1, 0, 0), (1, 1, 0)),                           # fp32 path
+    ((1, 2, 1, 8192, 64, 64, 1, 0, 1), (64, 2, 64 * (64 * 64 + 64) * 4)),  # 148 SMs, 64 chunks
+])
+def test_fwd_plan_host_arithmetic(monkeypatch, shape, expect):
+    """Blocks per sequence: the SM count over the (sequence, KV head) lanes,
+    at most the chunk count; one launch when there is one block; the
+    workspace holds one fp32 d x dv + d partial state per block."""
+    monkeypatch.delenv("LT_BLOCKS", raising=False)
+    monkeypatch.delenv("LT_KERNEL", raising=False)
+    from causal_linear_attention_chunked_b200 import _binding as b
+    B, Hq, Hkv, N, d, dv, causal, packed, dt = shape
+    nb, nl, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    st = b.lib.lt_linear_attn_fwd_plan(B, Hq, Hkv, N, d, dv, causal, packed, dt, 148,
+                                       ctypes.byref(nb), ctypes.byref(nl), ctypes.byref(ws))
+    assert st == 0
+    assert (nb.value, nl.value, ws.value) == expect
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(d=32), 2), (dict(dtype=3), 2), (dict(B=0), 1), (dict(Hkv=3, Hq=8), 1),
+    (dict(causal=5), 1), (dict(packed=2), 1), (dict(out=None), 1), (dict(Hkv=70000, Hq=70000), 1),
+])
+def test_fwd_plan_rejects_invalid_arguments(case, expect):
+    from causal_linear_attention_chunked_b200 import _binding as b
+    a = dict(B=1, Hq=8, Hkv=8, N=16, d=64, dv=64, causal=1, packed=0, dtype=1, out=True)
+    a.update(case)
+    nb, nl, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    st = b.lib.lt_linear_attn_fwd_plan(a["B"], a["Hq"], a["Hkv"], a["N"], a["d"], a["dv"],
+                                       a["causal"], a["packed"], a["dtype"], 148,
+                                       ctypes.byref(nb), ctypes.byref(nl),
+                                       ctypes.byref(ws) if a["out"] else None)
+    assert st == expect

@@ -163,9 +163,11 @@ def test_split_kernel_cluster_sizes(monkeypatch, n_split, case):
 @pytest.mark.parametrize("case", DENSE_CASES[:8], ids=lambda c: "B%dHq%dHkv%dN%d%s" % (
     c[0], c[1], c[2], c[3], "c" if c[6] else "nc"))
 def test_sequential_kernel_forced(monkeypatch, case):
-    """The sequential kernel (one CTA per (sequence, KV head)) on the d=64
-    shapes the split kernel normally takes."""
+    """The general kernel run fully sequentially (one CTA per (sequence,
+    KV head)) on the d = dv = 64 shapes the specialised kernel normally
+    takes."""
     monkeypatch.setenv("LT_KERNEL", "seq")
+    monkeypatch.setenv("LT_BLOCKS", "1")
     B, Hq, Hkv, N, d, dv, causal = case
     q, k, v = inputs.make_custom(B, Hq, Hkv, N, d, dv, torch.bfloat16, d ** -0.5, seed=N)
     got = run_dense(q, k, v, causal)
@@ -220,3 +222,32 @@ def test_block_kernel_deterministic_across_block_counts(monkeypatch):
         outs.append(run_dense(q, k, v, True))
     for o in outs[1:]:
         assert row_rel_err(o, outs[0]) <= 1e-2
+
+
+GENERAL_BLOCK_CASES = [
+    # (B, Hq, Hkv, N, d, dv, causal)
+    (1, 4, 2, 1000, 128, 128, True),   # GQA, ragged tail
+    (2, 2, 2, 777, 128, 128, False),
+    (1, 2, 2, 1300, 64, 128, True),
+    (1, 4, 2, 900, 128, 64, True),
+    (1, 2, 1, 1100, 64, 128, False),
+    (1, 4, 4, 1200, 64, 64, True),     # the general kernel on d = dv = 64
+]
+
+
+@pytest.mark.parametrize("nb", [1, 2, 3, 5])
+@pytest.mark.parametrize("case", GENERAL_BLOCK_CASES, ids=lambda c: "B%dHq%dHkv%dN%dd%ddv%d%s" % (
+    c[0], c[1], c[2], c[3], c[4], c[5], "c" if c[6] else "nc"))
+def test_general_kernel_block_counts(monkeypatch, nb, case):
+    """The general kernel (every width pair) with the sequence cut into nb
+    blocks: the state launch's block aggregates are summed into the carry
+    each block starts from (written into its TMEM state accumulator when
+    causal, used as the whole state when not)."""
+    monkeypatch.setenv("LT_KERNEL", "seq")
+    monkeypatch.setenv("LT_BLOCKS", str(nb))
+    B, Hq, Hkv, N, d, dv, causal = case
+    q, k, v = inputs.make_custom(B, Hq, Hkv, N, d, dv, torch.bfloat16, d ** -0.5,
+                                 seed=N + 11 * nb)
+    got = run_dense(q, k, v, causal)
+    ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
+    assert row_rel_err(got, ref) <= TOL_BF16
