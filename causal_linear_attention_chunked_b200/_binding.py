@@ -14,12 +14,13 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblt.so")
 
 LT_OK, LT_ERR_INVALID_ARG, LT_ERR_UNSUPPORTED, LT_ERR_CUDA = 0, 1, 2, 3
-LT_ERR_DEVICE_TIMEOUT, LT_ERR_DEVICE_BAD_SEQLENS = 4, 5
+LT_ERR_DEVICE_TIMEOUT, LT_ERR_DEVICE_BAD_SEQLENS, LT_ERR_SCRATCH_TOO_SMALL = 4, 5, 6
 LT_F32, LT_BF16 = 0, 1
 
 # every entry point declared in include/lt_linear_attn.h
-EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_fwd_plan", "lt_linear_attn_decode_step",
-            "lt_status_string", "lt_get_last_device_error", "lt_abi_version")
+EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_fwd_noalloc", "lt_linear_attn_fwd_plan",
+            "lt_linear_attn_decode_step", "lt_status_string", "lt_get_last_device_error",
+            "lt_abi_version")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("liblt.so is not built (run `python -m "
@@ -30,6 +31,9 @@ _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 lib.lt_linear_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _vp,
                                    _i]
 lib.lt_linear_attn_fwd.restype = _i
+lib.lt_linear_attn_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
+                                           _vp, _vp]
+lib.lt_linear_attn_fwd_noalloc.restype = _i
 lib.lt_linear_attn_fwd_plan.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                         ctypes.POINTER(_i), ctypes.POINTER(_i),
                                         ctypes.POINTER(ctypes.c_size_t)]

@@ -53,6 +53,10 @@ bool width_ok(int w) { return w == 64 || w == 128; }
 
 }  // namespace
 
+namespace lt {
+int* device_error_word_current() { return device_error_word(); }
+}  // namespace lt
+
 extern "C" {
 
 int lt_abi_version(void) { return 1; }
@@ -65,6 +69,8 @@ const char* lt_status_string(lt_status_t s) {
     case LT_ERR_CUDA: return "LT_ERR_CUDA: CUDA runtime or launch failure";
     case LT_ERR_DEVICE_TIMEOUT: return "LT_ERR_DEVICE_TIMEOUT: a kernel gave up a stalled wait";
     case LT_ERR_DEVICE_BAD_SEQLENS: return "LT_ERR_DEVICE_BAD_SEQLENS: inconsistent cu_seqlens";
+    case LT_ERR_SCRATCH_TOO_SMALL:
+      return "LT_ERR_SCRATCH_TOO_SMALL: the shape needs more than the fixed scratch array holds";
   }
   return "unknown lt_status_t";
 }

@@ -58,6 +58,8 @@ cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, const float* ws,
                                   cudaStream_t stream);
 cudaError_t launch_fwd_bf16_seq(const FwdLaunch& p, int nb, const float* ws,
                                 cudaStream_t stream);
+// the per-device error word of the current device (looked up once per device)
+int* device_error_word_current();
 cudaError_t launch_fwd_f32(const FwdLaunch& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeLaunch& p, cudaStream_t stream);
 

@@ -67,7 +67,9 @@ typedef enum {
   LT_ERR_UNSUPPORTED = 2,     /* d or dv not in {64, 128}, unknown dtype */
   LT_ERR_CUDA = 3,            /* a CUDA runtime call or launch failed */
   LT_ERR_DEVICE_TIMEOUT = 4,  /* a kernel gave up on a stalled wait */
-  LT_ERR_DEVICE_BAD_SEQLENS = 5 /* a kernel found cu_seqlens inconsistent */
+  LT_ERR_DEVICE_BAD_SEQLENS = 5, /* a kernel found cu_seqlens inconsistent */
+  LT_ERR_SCRATCH_TOO_SMALL = 6   /* lt_linear_attn_fwd_noalloc: the shape needs
+                                    more than LT_NOALLOC_SCRATCH_BYTES */
 } lt_status_t;
 
 typedef enum {
@@ -109,6 +111,42 @@ LT_API lt_status_t lt_linear_attn_fwd(const void *q, const void *k, const void *
                                int B, int H_q, int H_kv, int N, int d, int dv, int causal,
                                float eps, const int32_t *cu_seqlens, lt_stream_t stream,
                                lt_dtype_t dtype);
+
+/*
+ * lt_linear_attn_fwd_noalloc: the bf16 forward pass of lt_linear_attn_fwd
+ * (same arguments, dtype fixed to LT_BF16, same kernels and results) for
+ * callers that cannot let a library allocate device memory.  The paper has
+ * no counterpart; it exists for integration only.
+ *
+ * Who needs it: lt_linear_attn_fwd takes a stream-ordered workspace
+ * (cudaMallocAsync) for the per-block partial states.  A program that hands
+ * all device memory to its own caching allocator at start-up, a set-up
+ * without stream-ordered allocation (memory pools unsupported), or code that
+ * must keep a fixed memory footprint with no allocator work in its launch
+ * path cannot accept that.  This call allocates nothing: the workspace is a
+ * fixed array of LT_NOALLOC_SCRATCH_BYTES inside the library, which every
+ * device that loads the library holds until the process exits.  16 MiB
+ * covers every shape at the default block count on a GPU with up to 254 SMs
+ * (at most one partial state of d*dv + d floats per SM).
+ *
+ * Set-up: the first call on a device (with that device current) looks up
+ * the array's device address with cudaGetSymbolAddress; make that first
+ * call before any stream capture.
+ *
+ * Sharing: all calls on a device use the same array.  Calls whose work can
+ * overlap on the GPU (unordered streams, concurrent host threads) race on it
+ * and may return wrong results: order them.  Nothing in the array needs to
+ * start at zero; each call writes every partial state it later reads.
+ *
+ * Returns LT_ERR_UNSUPPORTED, LT_ERR_INVALID_ARG, LT_ERR_CUDA as
+ * lt_linear_attn_fwd does; LT_ERR_SCRATCH_TOO_SMALL (nothing enqueued) when
+ * the shape's workspace (lt_linear_attn_fwd_plan) exceeds the array.
+ */
+#define LT_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+LT_API lt_status_t lt_linear_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                                              void *out, int B, int H_q, int H_kv, int N,
+                                              int d, int dv, int causal, float eps,
+                                              const int32_t *cu_seqlens, lt_stream_t stream);
 
 /*
  * How lt_linear_attn_fwd evaluates a shape: blocks each sequence is cut
