@@ -24,11 +24,11 @@
 // Forward-kernel warp roles (512 threads; TMEM sub-partition = warp % 4):
 //   warps 0-5   transform: phi in place on K and Q tiles (tail rows zeroed)
 //   warps 6-9   mask + epilogue: causal mask of the score tile, bf16 in
-//               place in TMEM, the score row sums into the accumulator's
-//               normaliser; accumulator -> normalised bf16 rows -> global
+//               place in TMEM; accumulator -> normalised bf16 rows -> global
 //   warps 10-13 state: running [S|z] in registers -> bf16 B operand
 //   warp 14     TMA producer
 //   warp 15     TMEM allocator and single-thread MMA issuer
+// The normaliser is the extra column of P [V | 1] and phi(Q) [S | z].
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t ID_P = idesc_bf16_f32(kChunk, kChunk, 0, 0);
       constexpr uint32_t ID_SV = idesc_bf16_f32(D, DV + 16, 1, 1);
-      constexpr uint32_t ID_PV = idesc_bf16_f32(kChunk, DV, 0, 1);
+      constexpr uint32_t ID_PV = idesc_bf16_f32(kChunk, DV + 16, 0, 1);
       constexpr uint32_t ID_QS = idesc_bf16_f32(kChunk, DV + 16, 0, 1);
       // descriptor bases, advanced per stage / K step with one 64-bit add
       const uint64_t dQk = smem_desc_sw128(smem_u32(sQ), 16, 1024);      // K-major
@@ -326,15 +326,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok && (j + 1) % G == 0) ok = state_mma((j + 1) / G);
             if (!ok) break;
           }
-          const uint64_t vd = desc_advance(dVmn, (r % NKV) * KVT);
+          const uint32_t va = smem_u32(sV) + (r % NKV) * KVT;
+          const uint64_t vd = smem_desc_sw128(va, ones - va, 1024);  // [V | 1]
           const uint32_t t_acc = tmem + TM_ACC + as * ACCW;
           ok = mbar_wait(&bars.pb_full[as], (j >> 1) & 1, abort_flag, a.err, kWaitLimitNs) &&
                mbar_wait(&bars.acc_empty[as], ((j >> 1) & 1) ^ 1, abort_flag, a.err,
                          kWaitLimitNs);
           if (!ok) break;
           tc_fence_after();
-          // P V: bf16 scores from TMEM, 16 keys (8 columns) per MMA.  The
-          // normaliser column was initialised with the score row sums.
+          // P [V | 1]: bf16 scores from TMEM, 16 keys (8 columns) per MMA;
+          // the ones column gives the row sums of the masked scores
 #pragma unroll
           for (int kk = 0; kk < kChunk / 16; ++kk)
             umma_f16_ts(t_acc, tmem + TM_P + as * kChunk + kk * 8, desc_advance(vd, kk * 2048),
@@ -387,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&bars.kv_full[st], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs))
         return false;
       const int valid = min(kChunk, ntok - c * kChunk);
-      xf_tile<D / 64, kXf>(sK + st * KVT, valid, true, x);
+      prep_tile<D / 64, kXf>(sK + st * KVT, valid, true, x);
       if (valid < kChunk) xf_tile<DV / 64, kXf>(sV + st * KVT, valid, false, x);
       fence_proxy_async_smem();
       named_bar_sync(1, kXf);
@@ -398,7 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = j % NQ;
       if (!mbar_wait(&bars.q_full[st], (j / NQ) & 1, abort_flag, a.err, kWaitLimitNs))
         return false;
-      xf_tile<D / 64, kXf>(sQ + st * QT, kChunk, true, x);
+      // rows past the end of the sequence only feed output rows that are
+      // never stored
+      phi_tile_full<D / 64, kXf>(sQ + st * QT, x);
       fence_proxy_async_smem();
       named_bar_sync(1, kXf);
       if (x == 0) mbar_arrive(&bars.q_xf[st]);
@@ -423,17 +426,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     // causal mask and bf16 rounding of the score tile, in place in TMEM:
     // fp32 columns [32b, 32b+32) become packed bf16 columns [16b, 16b+16),
-    // which only overwrites columns this thread has already read; the row
-    // sum of the masked scores initialises the accumulator's normaliser
+    // which only overwrites columns this thread has already read
     auto mask_p = [&](int j) -> bool {
       const int as = j & 1;
-      if (!mbar_wait(&bars.p_full[as], (j >> 1) & 1, abort_flag, a.err, kWaitLimitNs) ||
-          !mbar_wait(&bars.acc_empty[as], ((j >> 1) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+      if (!mbar_wait(&bars.p_full[as], (j >> 1) & 1, abort_flag, a.err, kWaitLimitNs))
         return false;
       tc_fence_after();
       const uint32_t lane_sel = (uint32_t)(sp * 32) << 16;
       const uint32_t t_p = tmem + TM_P + as * kChunk + lane_sel;
-      float rs = 0.0f;
 #pragma unroll
       for (int b2 = 0; b2 < kChunk / 64; ++b2) {
         // two 32-column blocks per TMEM round trip
@@ -453,23 +453,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 16; ++e) pk[e] = 0u;
           } else if (b < sp) {  // block entirely left of the diagonal
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              pk[e] = pack_bf16x2(r[2 * e], r[2 * e + 1]);
-              rs += r[2 * e] + r[2 * e + 1];
-            }
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(r[2 * e], r[2 * e + 1]);
           } else {  // the diagonal block
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const float lo = (b * 32 + 2 * e > row) ? 0.0f : r[2 * e];
               const float hi = (b * 32 + 2 * e + 1 > row) ? 0.0f : r[2 * e + 1];
               pk[e] = pack_bf16x2(lo, hi);
-              rs += lo + hi;
             }
           }
           tmem_st16(t_p + b * 16, pk);
         }
       }
-      tmem_st1(tmem + TM_ACC + as * ACCW + DV + lane_sel, __float_as_uint(rs));
       tmem_wait_st();
       tc_fence_before();
       named_bar_sync(2, 128);
@@ -563,12 +558,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto add_ds = [&]() {
       const uint32_t t = tmem + TM_DS + lane_base;
 #pragma unroll
-      for (int half = 0; half < DV / 32; ++half) {
-        float cv[32];
-        tmem_ld32(t + half * 32, cv);
+      for (int q = 0; q < DV / 16; ++q) {
+        float cv[16];
+        tmem_ld16(t + q * 16, cv);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) T[half * 32 + e] += cv[e];
+        for (int e = 0; e < 16; ++e) T[q * 16 + e] += cv[e];
       }
       float zz[16];
       tmem_ld16(t + DV, zz);

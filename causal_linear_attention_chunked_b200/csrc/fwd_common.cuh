@@ -44,6 +44,43 @@ __device__ __forceinline__ void xf_tile(uint8_t* tile, int valid, bool apply_phi
   }
 }
 
+// phi in place over a full [kChunk x (NBOX*64)] bf16 tile (every row
+// valid).  The NBOX boxes are contiguous, so thread t takes the 16-byte
+// pieces t, t + NT, ...; all loads are issued before the arithmetic.
+template <int NBOX, int NT>
+__device__ __forceinline__ void phi_tile_full(uint8_t* tile, int tid) {
+  constexpr int kPieces = kChunk * NBOX * 8;
+  constexpr int kIt = (kPieces + NT - 1) / NT;
+  constexpr bool kRagged = kPieces % NT != 0;  // the last round covers part of the threads
+  uint4* p = reinterpret_cast<uint4*>(tile) + tid;
+  const bool last = !kRagged || tid + (kIt - 1) * NT < kPieces;
+  uint4 v[kIt];
+#pragma unroll
+  for (int i = 0; i < kIt; ++i)
+    if (i < kIt - 1 || last) v[i] = p[i * NT];
+#pragma unroll
+  for (int i = 0; i < kIt; ++i) {
+    v[i].x = phi_bf16x2(v[i].x);
+    v[i].y = phi_bf16x2(v[i].y);
+    v[i].z = phi_bf16x2(v[i].z);
+    v[i].w = phi_bf16x2(v[i].w);
+  }
+#pragma unroll
+  for (int i = 0; i < kIt; ++i)
+    if (i < kIt - 1 || last) p[i * NT] = v[i];
+}
+
+// phi (apply_phi) and zeroing of the rows >= valid: the fast path for full
+// tiles, the general loop for the ragged last chunk.
+template <int NBOX, int NT>
+__device__ __forceinline__ void prep_tile(uint8_t* tile, int valid, bool apply_phi, int tid) {
+  if (valid >= kChunk) {
+    if (apply_phi) phi_tile_full<NBOX, NT>(tile, tid);
+  } else {
+    xf_tile<NBOX, NT>(tile, valid, apply_phi, tid);
+  }
+}
+
 // Byte offset of the 16-byte piece holding columns [8*jj, 8*jj+8) of row
 // `row` inside a 128-byte-swizzled 64-column box (1024-byte aligned).
 __device__ __forceinline__ uint32_t sw128_off(int row, int jj) {

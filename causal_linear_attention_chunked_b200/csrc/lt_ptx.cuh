@@ -269,29 +269,23 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   return __bfloat1622float2(h);
 }
 
-// Feature map on a pair of packed bf16 values:
-//     phi(x) = ELU(x) + 1 = max(x, 0) + exp(min(x, 0))
-// (x > 0: x + e^0 = x + 1; x <= 0: 0 + e^x).  The exponent argument
-// min(x,0)*log2(e) is formed in fp32 and rounded once to bf16 for the
-// packed hardware base-2 exponential (two results per instruction); the sum
-// is rounded to bf16, the precision of the tensor-core operand anyway.
-__device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
-  uint32_t y;
-  asm("{\n\t.reg .b32 zero, neg, pos, t, e;\n\t"
-      ".reg .f32 lo, hi;\n\t"
-      "mov.b32 zero, 0;\n\t"
-      "min.bf16x2 neg, %1, zero;\n\t"
-      "max.bf16x2 pos, %1, zero;\n\t"
-      "shl.b32 lo, neg, 16;\n\t"              // low half -> fp32
-      "and.b32 hi, neg, 0xFFFF0000;\n\t"      // high half -> fp32
-      "mul.f32 lo, lo, 0f3FB8AA3B;\n\t"       // * log2(e)
-      "mul.f32 hi, hi, 0f3FB8AA3B;\n\t"
-      "cvt.rn.bf16x2.f32 t, hi, lo;\n\t"
-      "ex2.approx.ftz.bf16x2 e, t;\n\t"
-      "add.rn.bf16x2 %0, pos, e;\n\t}"
-      : "=r"(y)
-      : "r"(x));
+// Hardware base-2 exponential (MUFU), fp32 in and out.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Feature map on a pair of packed bf16 values, phi(x) = ELU(x) + 1:
+// x + 1 for x > 0, e^x = 2^(x log2 e) otherwise, each evaluated in fp32 and
+// rounded once to bf16 (the precision of the tensor-core operand).  The
+// exponential is taken for every x and discarded for x > 0 (where it may
+// overflow to +inf); NaN propagates through the exponential.
+__device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
+  const float lo = __uint_as_float(x << 16), hi = __uint_as_float(x & 0xFFFF0000u);
+  const float elo = ex2_approx(lo * 1.4426950408889634f);
+  const float ehi = ex2_approx(hi * 1.4426950408889634f);
+  return pack_bf16x2(lo > 0.0f ? lo + 1.0f : elo, hi > 0.0f ? hi + 1.0f : ehi);
 }
 
 // Feature map of the method: phi(x) = ELU(x) + 1 = x + 1 (x > 0), e^x (x <= 0).

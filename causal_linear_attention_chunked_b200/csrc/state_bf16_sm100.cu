@@ -11,10 +11,10 @@
 // Ultra-Long Context", section 5.3.  The forward launch then starts block b
 // from sum_{b' < b} A_b' (causal) or sum_b A_b (non-causal).
 //
-// One CTA per (block, KV head, sequence); 192 threads: warps 0-3 apply phi
-// to the TMA-loaded K tiles (tail rows zeroed) and store the result, warp 4
-// is the TMA producer, warp 5 allocates TMEM and issues the MMAs that
-// accumulate A_b in TMEM.
+// One CTA per (block, KV head, sequence); 320 threads: warps 0-7 apply phi
+// to the TMA-loaded K tiles (tail rows zeroed; two warps per SM
+// sub-partition) and warps 0-3 store the result, warp 8 is the TMA producer,
+// warp 9 allocates TMEM and issues the MMAs that accumulate A_b in TMEM.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -29,7 +29,8 @@ namespace lt {
 namespace {
 using namespace fwd;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kXf = 256;  // transform threads
 
 template <int D, int DV>
 struct SCfg {
@@ -102,14 +103,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   init_ones_block(smem + K::OFF_ONES, tid, kThreads);
   fence_proxy_async_smem();
-  if (warp == 5) tmem_alloc(tmem_slot, K::TM_COLS);
+  if (warp == 9) tmem_alloc(tmem_slot, K::TM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int* abort_flag = &s_abort;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&full[i % K::NS], (i / K::NS) & 1, &dummy, nullptr, kWaitLimitNs);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       // dv = 64: [V | 1] is one N = 80 MN-major operand whose second group is
       // the shared ones block (per-stage leading byte offset); dv = 128: the
@@ -176,16 +177,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = mbar_wait(&full[st], (i / K::NS) & 1, abort_flag, a.err, kWaitLimitNs);
       if (!ok) break;
       const int valid = min(kChunk, ntok - c * kChunk);
-      xf_tile<D / 64>(sK + st * K::KVT, valid, true, x);
-      if (valid < kChunk) xf_tile<DV / 64>(sV + st * K::KVT, valid, false, x);
+      prep_tile<D / 64, kXf>(sK + st * K::KVT, valid, true, x);
+      if (valid < kChunk) xf_tile<DV / 64, kXf>(sV + st * K::KVT, valid, false, x);
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
+      named_bar_sync(1, kXf);
       if (x == 0) mbar_arrive(&xf[st]);
     }
     // store A_b.  M = 64 accumulator: state row 16*w + l in lane l < 16 of
     // sub-partition w; M = 128: row 32*w + l in lane l.
-    if (ok) ok = mbar_wait(s_full, 0, abort_flag, a.err, kWaitLimitNs);
-    if (ok) {
+    if (ok && warp < 4) ok = mbar_wait(s_full, 0, abort_flag, a.err, kWaitLimitNs);
+    if (ok && warp < 4) {
       tc_fence_after();
       const uint32_t t = tmem + ((uint32_t)(warp * 32) << 16);
       const bool has_row = (D == 128) || lane < 16;
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, K::TM_COLS);
   }
@@ -258,7 +259,8 @@ int block_count(const FwdLaunch& p, int num_sms) {
   int nb = num_sms / (lanes > 0 ? lanes : 1);
   if (nb < 1) nb = 1;
   if (nb > nc) nb = nc;
-  return nb;
+  const int bc = (nc + nb - 1) / nb;
+  return (nc + bc - 1) / bc;  // no block left empty by the rounding
 }
 
 int block_chunks(const FwdLaunch& p, int nb) {

@@ -106,7 +106,7 @@ def test_oracle_and_library_share_no_code():
 
 @pytest.mark.parametrize("shape,expect", [
     # (B, H_q, H_kv, N, d, dv, causal, packed, dtype), num_sms = 148
-    ((2, 8, 8, 4096, 64, 64, 1, 0, 1), (9, 2, 2 * 8 * 9 * (64 * 64 + 64) * 4)),
+    ((2, 8, 8, 4096, 64, 64, 1, 0, 1), (8, 2, 2 * 8 * 8 * (64 * 64 + 64) * 4)),  # 9 -> 8 blocks of 4
     ((1, 8, 8, 65536, 64, 64, 0, 0, 1), (18, 2, 8 * 18 * (64 * 64 + 64) * 4)),
     ((2, 32, 8, 16384, 128, 128, 1, 0, 1), (9, 2, 2 * 8 * 9 * (128 * 128 + 128) * 4)),
     ((1, 1, 1, 300, 64, 128, 1, 0, 1), (3, 2, 3 * (64 * 128 + 64) * 4)),   # capped by 3 chunks
