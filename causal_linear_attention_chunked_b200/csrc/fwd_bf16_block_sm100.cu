@@ -21,13 +21,15 @@
 // Non-causal mode: the state kernel computes every block's sum and the
 // forward kernel reads only Q, with [S|z] = sum of all blocks.
 //
-// Forward-kernel warp roles (512 threads; TMEM sub-partition = warp % 4):
-//   warps 0-5   transform: phi in place on K and Q tiles (tail rows zeroed)
-//   warps 6-9   mask + epilogue: causal mask of the score tile, bf16 in
+// Forward-kernel warp roles (576 threads; TMEM sub-partition = warp % 4):
+//   warps 0-7   transform: phi in place on K and Q tiles (tail rows zeroed)
+//   warps 8-11  mask + epilogue: causal mask of the score tile, bf16 in
 //               place in TMEM; accumulator -> normalised bf16 rows -> global
-//   warps 10-13 state: running [S|z] in registers -> bf16 B operand
-//   warp 14     TMA producer
-//   warp 15     TMEM allocator and single-thread MMA issuer
+//   warps 12-15 state: carry into the TMEM state accumulator, which the
+//               tensor cores advance by phi(K)^T [V | 1] per chunk; TMEM
+//               state -> bf16 B operand before every chunk
+//   warp 16     TMA producer
+//   warp 17     TMEM allocator and single-thread MMA issuer
 // The normaliser is the extra column of P [V | 1] and phi(Q) [S | z].
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -79,12 +81,12 @@ __device__ __forceinline__ bool seq_bounds(const BlockArgs& a, int s, int& t0, i
 // ========================================================================
 // Forward pass over one block per CTA.
 // ========================================================================
-constexpr int kThreads = 512;
-constexpr int kXf = 192;  // transform threads (warps 0-5)
+constexpr int kThreads = 576;
+constexpr int kXf = 256;  // transform threads (warps 0-7, two per SM sub-partition)
 constexpr int NQ = 4, NKV = 4;
-// two score tiles (item j uses j & 1), two accumulators, one dS tile
-constexpr int TM_P = 0, TM_ACC = 2 * kChunk, TM_DS = TM_ACC + 2 * ACCW, TM_COLS = 512;
-static_assert(TM_DS + ACCW <= TM_COLS, "TMEM budget");
+// two score tiles (item j uses j & 1), two accumulators, the running state
+constexpr int TM_P = 0, TM_ACC = 2 * kChunk, TM_S = TM_ACC + 2 * ACCW, TM_COLS = 512;
+static_assert(TM_S + ACCW <= TM_COLS, "TMEM budget");
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + NQ * QT;  // stage st: [K][V] at st*KVT
 constexpr int OFF_ONES = OFF_KV + NKV * KVT;
@@ -97,7 +99,7 @@ static_assert(SMEM <= 232448, "shared memory budget");
 struct Bars {
   uint64_t *q_full, *q_empty, *q_xf, *kv_full, *kv_empty, *kv_xf;
   uint64_t *p_full, *pb_full, *sop_full, *sop_empty;
-  uint64_t *ds_full, *ds_empty, *acc_full, *acc_empty, *drain;
+  uint64_t *s_full, *s_empty, *acc_full, *acc_empty, *drain;
 };
 
 __device__ __forceinline__ Bars carve(uint8_t* base) {
@@ -113,30 +115,12 @@ __device__ __forceinline__ Bars carve(uint8_t* base) {
   r.pb_full = b; b += 2;
   r.sop_full = b++;
   r.sop_empty = b++;
-  r.ds_full = b++;
-  r.ds_empty = b++;
+  r.s_full = b++;
+  r.s_empty = b++;
   r.acc_full = b; b += 2;
   r.acc_empty = b; b += 2;
   r.drain = b++;
   return r;
-}
-
-// One row of the [S | z 0 ... 0] operand (MN-major, 128-byte swizzle; row =
-// state row a, columns n = 0..dv+15) from fp32 values.
-__device__ __forceinline__ void write_sop_row(uint8_t* sop, int a, const float* s, float z) {
-#pragma unroll
-  for (int q8 = 0; q8 < DV / 8; ++q8) {
-    const uint4 w = make_uint4(pack_bf16x2(s[q8 * 8 + 0], s[q8 * 8 + 1]),
-                               pack_bf16x2(s[q8 * 8 + 2], s[q8 * 8 + 3]),
-                               pack_bf16x2(s[q8 * 8 + 4], s[q8 * 8 + 5]),
-                               pack_bf16x2(s[q8 * 8 + 6], s[q8 * 8 + 7]));
-    *reinterpret_cast<uint4*>(sop + (q8 >> 3) * (D * kRowBytes) + sw128_off(a, q8 & 7)) = w;
-  }
-  const int grp = DV / 64;
-  *reinterpret_cast<uint4*>(sop + grp * (D * kRowBytes) + sw128_off(a, 0)) =
-      make_uint4(pack_bf16x2(z, 0.0f), 0u, 0u, 0u);
-  *reinterpret_cast<uint4*>(sop + grp * (D * kRowBytes) + sw128_off(a, 1)) =
-      make_uint4(0u, 0u, 0u, 0u);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -186,8 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bars.sop_full, 1);
     mbar_init(bars.sop_empty, 1);
-    mbar_init(bars.ds_full, 1);
-    mbar_init(bars.ds_empty, 1);
+    mbar_init(bars.s_full, 1);
+    mbar_init(bars.s_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.p_full[i], 1);
       mbar_init(&bars.pb_full[i], 1);
@@ -199,14 +183,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   init_ones_block(smem + OFF_ONES, tid, kThreads);
   fence_proxy_async_smem();
-  if (warp == 15) tmem_alloc(tmem_slot, TM_COLS);
+  if (warp == 17) tmem_alloc(tmem_slot, TM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int* abort_flag = &s_abort;
 
-  if (warp == 14) {
+  if (warp == 16) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -251,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&bars.q_full[j % NQ], (j / NQ) & 1, &dummy, nullptr, kWaitLimitNs);
       }
     }
-  } else if (warp == 15) {
+  } else if (warp == 17) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t ID_P = idesc_bf16_f32(kChunk, kChunk, 0, 0);
@@ -286,14 +270,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                       desc_advance(dSop, kk * 2048), ID_QS, (accumulate || kk > 0) ? 1u : 0u);
       };
       if (causal) {
-        // dS of chunk r (single TMEM buffer: the state warpgroup drains it)
+        // S_acc += dS of chunk r, once the state warpgroup has read S_<r
+        // (phase r of s_empty; phase 0 is the carry it wrote).  Only chunks
+        // before the block's last one feed a later state.
         auto state_mma = [&](int r) -> bool {
+          if (r + 1 >= Ri) return true;
           if (!mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs) ||
-              !mbar_wait(bars.ds_empty, (r & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+              !mbar_wait(bars.s_empty, r & 1, abort_flag, a.err, kWaitLimitNs))
             return false;
           tc_fence_after();
-          issue_ds(r, tmem + TM_DS, false);
-          umma_commit(bars.ds_full);
+          issue_ds(r, tmem + TM_S, true);
+          umma_commit(bars.s_full);
           return true;
         };
         // score tile of item j into TMEM buffer j & 1.  The buffer last held
@@ -357,10 +344,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs);
             if (!ok) break;
             tc_fence_after();
-            issue_ds(r, tmem + TM_DS, r > 0);
+            issue_ds(r, tmem + TM_S, r > 0);
             umma_commit(&bars.kv_empty[r % NKV]);
           }
-          if (ok) umma_commit(bars.ds_full);
+          if (ok) umma_commit(bars.s_full);
         }
         if (ok) ok = mbar_wait(bars.sop_full, 0, abort_flag, a.err, kWaitLimitNs);
         for (int j = 0; j < n_items && ok; ++j) {
@@ -379,9 +366,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int dummy = 0;
       mbar_wait(bars.drain, 0, &dummy, nullptr, kWaitLimitNs);
     }
-  } else if (warp < 6) {
+  } else if (warp < 8) {
     // ---------------------------------------------- transform warps
-    const int x = tid;  // 0..191
+    const int x = tid;  // 0..255
     bool ok = true;
     auto xf_kv = [&](int r) -> bool {
       const int st = r % NKV, c = c0 + r;
@@ -418,9 +405,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int r = 0; r < Ri && ok; ++r) ok = xf_kv(r);
       for (int j = 0; j < n_items && ok; ++j) ok = xf_q(j);
     }
-  } else if (warp < 10) {
+  } else if (warp < 12) {
     // ---------------------------------------------------- mask warpgroup
-    const int x = tid - 192, sp = warp & 3;
+    const int x = tid - 256, sp = warp & 3;
     const int row = sp * 32 + lane;  // TMEM lane == chunk row
     const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     bool ok = true;
@@ -435,23 +422,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lane_sel = (uint32_t)(sp * 32) << 16;
       const uint32_t t_p = tmem + TM_P + as * kChunk + lane_sel;
 #pragma unroll
-      for (int b2 = 0; b2 < kChunk / 64; ++b2) {
-        // two 32-column blocks per TMEM round trip
-        float r0[32], r1[32];
-        const bool h0 = 2 * b2 <= sp, h1 = 2 * b2 + 1 <= sp;  // warp-uniform
-        if (h0) tmem_ld32(t_p + (2 * b2) * 32, r0);
-        if (h1) tmem_ld32(t_p + (2 * b2 + 1) * 32, r1);
-        if (h0) tmem_wait_ld();
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int b = 2 * b2 + half;
-          const float* r = half ? r1 : r0;
-          const bool have = half ? h1 : h0;
-          uint32_t pk[16];
-          if (!have) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = 0u;
-          } else if (b < sp) {  // block entirely left of the diagonal
+      for (int b = 0; b < kChunk / 32; ++b) {
+        uint32_t pk[16];
+        if (b <= sp) {  // warp-uniform: blocks right of the diagonal are all zero
+          float r[32];
+          tmem_ld32(t_p + b * 32, r);
+          tmem_wait_ld();
+          if (b < sp) {  // block entirely left of the diagonal
 #pragma unroll
             for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(r[2 * e], r[2 * e + 1]);
           } else {  // the diagonal block
@@ -462,8 +439,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[e] = pack_bf16x2(lo, hi);
             }
           }
-          tmem_st16(t_p + b * 16, pk);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
         }
+        tmem_st16(t_p + b * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -477,32 +457,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         return false;
       tc_fence_after();
       const uint32_t t_acc = tmem + TM_ACC + as * ACCW + lane_base;
-      float den[16], n0[32], n1[32];
-      tmem_ld16(t_acc + DV, den);
-      tmem_ld32(t_acc, n0);
-      tmem_ld32(t_acc + 32, n1);
-      tmem_wait_ld();
+      // numerator columns -> normalised packed bf16, 32 at a time; the
+      // accumulator is released before the stores
+      uint32_t pk[DV / 2];
+      float inv;
+      {
+        float n[32];
+        const float den = tmem_ld1(t_acc + DV);
+        tmem_ld32(t_acc, n);
+        tmem_wait_ld();
+        inv = 1.0f / (den + a.eps);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(n[2 * e] * inv, n[2 * e + 1] * inv);
+      }
+#pragma unroll
+      for (int cb = 1; cb < DV / 32; ++cb) {
+        float n[32];
+        tmem_ld32(t_acc + cb * 32, n);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[cb * 16 + e] = pack_bf16x2(n[2 * e] * inv, n[2 * e + 1] * inv);
+      }
       tc_fence_before();
       named_bar_sync(2, 128);
       if (x == 0) mbar_arrive(&bars.acc_empty[as]);
-      const float inv = 1.0f / (den[0] + a.eps);
       const int valid = min(kChunk, ntok - c * kChunk);
       if (row < valid) {
-        __nv_bfloat16* orow =
-            a.out + ((size_t)(t0 + c * kChunk + row) * a.Hq + (size_t)(g * G + h)) * DV;
+        uint4* orow = reinterpret_cast<uint4*>(
+            a.out + ((size_t)(t0 + c * kChunk + row) * a.Hq + (size_t)(g * G + h)) * DV);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          *reinterpret_cast<uint4*>(orow + q4 * 8) =
-              make_uint4(pack_bf16x2(n0[q4 * 8 + 0] * inv, n0[q4 * 8 + 1] * inv),
-                         pack_bf16x2(n0[q4 * 8 + 2] * inv, n0[q4 * 8 + 3] * inv),
-                         pack_bf16x2(n0[q4 * 8 + 4] * inv, n0[q4 * 8 + 5] * inv),
-                         pack_bf16x2(n0[q4 * 8 + 6] * inv, n0[q4 * 8 + 7] * inv));
-          *reinterpret_cast<uint4*>(orow + 32 + q4 * 8) =
-              make_uint4(pack_bf16x2(n1[q4 * 8 + 0] * inv, n1[q4 * 8 + 1] * inv),
-                         pack_bf16x2(n1[q4 * 8 + 2] * inv, n1[q4 * 8 + 3] * inv),
-                         pack_bf16x2(n1[q4 * 8 + 4] * inv, n1[q4 * 8 + 5] * inv),
-                         pack_bf16x2(n1[q4 * 8 + 6] * inv, n1[q4 * 8 + 7] * inv));
-        }
+        for (int q = 0; q < DV / 8; ++q)
+          orow[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       }
       return true;
     };
@@ -517,89 +503,117 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       for (int j = 0; j < n_items && ok; ++j) ok = epilogue(j);
     }
-  } else if (warp < 14) {
+  } else if (warp < 16) {
     // -------------------------------------------------- state warpgroup
-    // dS is an M=64 accumulator: state row a = 16*sp + l lives in lane l < 16
-    // of TMEM sub-partition sp; that thread owns row a of the running state.
-    const int y = tid - 320, sp = warp & 3;
-    const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+    // The running [S | z] is an fp32 M=64 accumulator in TMEM (S_acc): state
+    // row a = 16*sp + l lives in lane l < 16 of sub-partition sp.  This
+    // group writes the carry into it, and before every chunk copies it,
+    // rounded to bf16, into the MN-major [S | z 0 ..] operand.
+    const int y = tid - 384, sp = warp & 3;
+    const uint32_t t_s = tmem + TM_S + ((uint32_t)(sp * 32) << 16);
     const bool has_row = lane < 16;
     const int row = sp * 16 + lane;
     bool ok = true;
-    float T[DV], Tz = 0.0f;  // this thread's row of the running [S|z]
+    uint32_t w[ACCW / 2];  // this thread's row of [S | z 0 ..], packed bf16
+    // carry: the aggregates of the earlier blocks (causal) or of every block
+    // (non-causal), summed in fp32; zero without a workspace.  Causal: also
+    // the initial value of S_acc.
+    auto load_carry = [&](bool to_tmem) {
+      const float* base = a.ws != nullptr ? a.ws + (size_t)(s * a.Hkv + g) * a.nb * E : nullptr;
+      const int nprev = a.ws == nullptr ? 0 : (causal ? blk : a.nb);
 #pragma unroll
-    for (int e = 0; e < DV; ++e) T[e] = 0.0f;
-    // carry into this block: the aggregates of the earlier blocks (causal),
-    // or of every block (non-causal), summed in fp32
-    if (a.ws != nullptr && has_row) {
-      const float* base = a.ws + (size_t)(s * a.Hkv + g) * a.nb * E;
-      const int nprev = causal ? blk : a.nb;
-      for (int bb = 0; bb < nprev; ++bb) {
-        const float4* r4 = reinterpret_cast<const float4*>(base + (size_t)bb * E + row * DV);
+      for (int q = 0; q < ACCW / 16; ++q) {
+        float c[16];
 #pragma unroll
-        for (int q = 0; q < DV / 4; ++q) {
-          const float4 v = r4[q];
-          T[4 * q] += v.x;
-          T[4 * q + 1] += v.y;
-          T[4 * q + 2] += v.z;
-          T[4 * q + 3] += v.w;
+        for (int e = 0; e < 16; ++e) c[e] = 0.0f;
+        if (has_row) {
+          for (int bb = 0; bb < nprev; ++bb) {
+            const float* ab = base + (size_t)bb * E;
+            if (q < DV / 16) {
+              const float4* r4 = reinterpret_cast<const float4*>(ab + row * DV + q * 16);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float4 v = r4[u];
+                c[4 * u] += v.x;
+                c[4 * u + 1] += v.y;
+                c[4 * u + 2] += v.z;
+                c[4 * u + 3] += v.w;
+              }
+            } else {
+              c[0] += ab[D * DV + row];
+            }
+          }
         }
-        Tz += base[(size_t)bb * E + D * DV + row];
+        if (to_tmem) {
+          uint32_t u16[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) u16[e] = __float_as_uint(c[e]);
+          tmem_st16(t_s + q * 16, u16);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[q * 8 + e] = pack_bf16x2(c[2 * e], c[2 * e + 1]);
       }
-    }
+      if (to_tmem) tmem_wait_st();
+    };
+    auto read_state = [&]() {
+#pragma unroll
+      for (int q = 0; q < ACCW / 16; ++q) {
+        float c[16];
+        tmem_ld16(t_s + q * 16, c);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[q * 8 + e] = pack_bf16x2(c[2 * e], c[2 * e + 1]);
+      }
+    };
+    // w -> the operand (pieces of 8 columns; columns dv.. are [z 0 ..])
     auto publish_sop = [&](int r) -> bool {
       if (!mbar_wait(bars.sop_empty, (r & 1) ^ 1, abort_flag, a.err, kWaitLimitNs)) return false;
-      if (has_row) write_sop_row(sSOP, row, T, Tz);
+      if (has_row) {
+#pragma unroll
+        for (int q8 = 0; q8 < ACCW / 8; ++q8)
+          *reinterpret_cast<uint4*>(sSOP + (q8 >> 3) * (D * kRowBytes) + sw128_off(row, q8 & 7)) =
+              make_uint4(w[4 * q8], w[4 * q8 + 1], w[4 * q8 + 2], w[4 * q8 + 3]);
+      }
       fence_proxy_async_smem();
       named_bar_sync(3, 128);
       if (y == 0) mbar_arrive(bars.sop_full);
       return true;
     };
-    auto add_ds = [&]() {
-      const uint32_t t = tmem + TM_DS + lane_base;
-#pragma unroll
-      for (int q = 0; q < DV / 16; ++q) {
-        float cv[16];
-        tmem_ld16(t + q * 16, cv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) T[q * 16 + e] += cv[e];
-      }
-      float zz[16];
-      tmem_ld16(t + DV, zz);
-      tmem_wait_ld();
-      Tz += zz[0];
+    // phase r of s_empty: S_<r has been read (r = 0: the carry written)
+    auto release_state = [&]() {
+      tc_fence_before();
+      named_bar_sync(3, 128);
+      if (y == 0) mbar_arrive(bars.s_empty);
     };
     if (causal) {
-      // [S|z]_<c+1 is published as soon as chunk c's phi(Q)[S|z] MMAs have
-      // released the operand
+      load_carry(true);
+      release_state();
       ok = publish_sop(0);
-      for (int r = 0; r < Ri && ok; ++r) {
-        ok = mbar_wait(bars.ds_full, r & 1, abort_flag, a.err, kWaitLimitNs);
+      for (int r = 1; r < Ri && ok; ++r) {
+        ok = mbar_wait(bars.s_full, (r - 1) & 1, abort_flag, a.err, kWaitLimitNs);
         if (!ok) break;
         tc_fence_after();
-        add_ds();
-        tc_fence_before();
-        named_bar_sync(3, 128);
-        if (y == 0) mbar_arrive(bars.ds_empty);
-        if (r + 1 < Ri) ok = publish_sop(r + 1);
+        read_state();
+        release_state();
+        ok = publish_sop(r);
       }
+    } else if (nc_from_ws) {
+      load_carry(false);
+      ok = publish_sop(0);
     } else {
-      if (!nc_from_ws) {
-        ok = mbar_wait(bars.ds_full, 0, abort_flag, a.err, kWaitLimitNs);
-        if (ok) {
-          tc_fence_after();
-          add_ds();
-          tc_fence_before();
-        }
+      ok = mbar_wait(bars.s_full, 0, abort_flag, a.err, kWaitLimitNs);
+      if (ok) {
+        tc_fence_after();
+        read_state();
+        tc_fence_before();
+        ok = publish_sop(0);
       }
-      if (ok) ok = publish_sop(0);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 15) {
+  if (warp == 17) {
     tc_fence_after();
     tmem_dealloc(tmem, TM_COLS);
   }
