@@ -168,7 +168,9 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------- distributed
-def dist_setup(want):
+def dist_setup(want, backend=None):
+    """One process per GPU under torchrun: (world, rank, local rank).  NCCL on
+    GPUs; gloo when there is no GPU (the host-side tests of this path)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -176,9 +178,13 @@ def dist_setup(want):
         import datetime
         import torch.distributed as dist
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     elif want > 1:
         raise SystemExit("--gpus %d needs a torchrun launch (one process per GPU)" % want)
     return world, rank, local
@@ -194,9 +200,20 @@ def max_over_ranks(x, world):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(base, rank):
+    """Each rank draws its own batch: the workload's seed offset by rank."""
+    return base + 1000 * rank
+
+
+def whole_job_rate(units_per_rank, world, ms_max):
+    """Units of all ranks over the slowest rank's time (weak scaling)."""
+    return units_per_rank * world / (ms_max / 1e3)
 
 
 # --------------------------------------------------------------- GPU arm
@@ -262,14 +279,14 @@ def fwd_step_fns(L, w, sets, stream):
     return fns
 
 
-def measure_workload(L, w, K, W, stream, device, world, l2_bytes):
+def measure_workload(L, w, K, W, stream, device, world, l2_bytes, rank=0):
     """Throughput of one workload: (tokens/s, ms per step, bytes per step)."""
     q0, _, _, cu0 = inputs.make(w)
     total_tokens = int(cu0[-1]) if cu0 is not None else w.B * w.N
     nbytes = algorithmic_bytes(w, total_tokens)
     R = max(1, math.ceil(3 * l2_bytes / nbytes))
     lengths = None if cu0 is None else (cu0[1:] - cu0[:-1]).tolist()  # same lengths in every set
-    sets = make_sets(w, R, w.seed, device, lengths)
+    sets = make_sets(w, R, rank_seed(w.seed, rank), device, lengths)
     fns = fwd_step_fns(L, w, sets, stream)
     with torch.cuda.stream(stream):
         for i in range(W):
@@ -375,10 +392,10 @@ def run_lt(args):
     sampler = ClockSampler(device)
     sampler.start()
     units, ms_step, nbytes, R, window = measure_workload(L, w, args.steps, args.warmup, stream,
-                                                         device, world, l2)
+                                                         device, world, l2, rank)
     clocks = sampler.summary(*window)
     sampler.stop()
-    value = units * world / (ms_step / 1e3)
+    value = whole_job_rate(units, world, ms_step)
     peak, peak_kind = peaks()
     achieved = nbytes / (ms_step * 1e-3) / 1e9
     traffic = committed_traffic(w.name)
