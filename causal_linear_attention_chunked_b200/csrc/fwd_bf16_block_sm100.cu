@@ -303,16 +303,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&bars.p_full[j & 1]);
           return true;
         };
-        ok = score_mma(0) && state_mma(0);
-        for (int j = 0; j < n_items && ok; ++j) {
-          const int r = j / G, h = j % G, qs = j % NQ, as = j & 1;
-          // the next item's score tile first: its mask then overlaps this
-          // item's P V and phi(Q)[S|z] MMAs
-          if (j + 1 < n_items) {
-            ok = score_mma(j + 1);
-            if (ok && (j + 1) % G == 0) ok = state_mma((j + 1) / G);
+        // item t's score tile (and the state product of its chunk) ahead of
+        // item t-1's P V and phi(Q)[S|z]: the mask of item t then overlaps
+        // those products.  Each step is issued from one place in the loop.
+        for (int t = 0; t <= n_items && ok; ++t) {
+          if (t < n_items) {
+            ok = score_mma(t);
+            if (ok && t % G == 0) ok = state_mma(t / G);
             if (!ok) break;
           }
+          if (t == 0) continue;
+          const int j = t - 1;
+          const int r = j / G, h = j % G, qs = j % NQ, as = j & 1;
           const uint32_t va = smem_u32(sV) + (r % NKV) * KVT;
           const uint64_t vd = smem_desc_sw128(va, ones - va, 1024);  // [V | 1]
           const uint32_t t_acc = tmem + TM_ACC + as * ACCW;
@@ -370,40 +372,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------- transform warps
     const int x = tid;  // 0..255
     bool ok = true;
-    auto xf_kv = [&](int r) -> bool {
-      const int st = r % NKV, c = c0 + r;
-      if (!mbar_wait(&bars.kv_full[st], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs))
-        return false;
-      const int valid = min(kChunk, ntok - c * kChunk);
-      prep_tile<D / 64, kXf>(sK + st * KVT, valid, true, x);
-      if (valid < kChunk) xf_tile<DV / 64, kXf>(sV + st * KVT, valid, false, x);
-      fence_proxy_async_smem();
-      named_bar_sync(1, kXf);
-      if (x == 0) mbar_arrive(&bars.kv_xf[st]);
-      return true;
-    };
-    auto xf_q = [&](int j) -> bool {
-      const int st = j % NQ;
-      if (!mbar_wait(&bars.q_full[st], (j / NQ) & 1, abort_flag, a.err, kWaitLimitNs))
-        return false;
-      // rows past the end of the sequence only feed output rows that are
-      // never stored
-      phi_tile_full<D / 64, kXf>(sQ + st * QT, x);
-      fence_proxy_async_smem();
-      named_bar_sync(1, kXf);
-      if (x == 0) mbar_arrive(&bars.q_xf[st]);
-      return true;
-    };
-    if (causal) {
-      ok = xf_kv(0);
-      for (int j = 0; j < n_items && ok; ++j) {
-        if (j % G == 0 && j > 0) ok = xf_kv(j / G);
-        if (ok) ok = xf_q(j);
+    // One loop over the tiles in arrival order (causal: K_r then the Q of
+    // each head of chunk r; non-causal: every K, then every Q), so that the
+    // transform code exists once in the kernel image.
+    const int nkv = nc_from_ws ? 0 : Ri;
+    const int T = causal ? Ri * (G + 1) : nkv + n_items;
+    for (int t = 0; t < T && ok; ++t) {
+      bool is_kv;
+      int r, j;
+      if (causal) {
+        r = t / (G + 1);
+        const int k = t - r * (G + 1);
+        is_kv = k == 0;
+        j = r * G + k - 1;
+      } else {
+        is_kv = t < nkv;
+        r = t;
+        j = t - nkv;
       }
-    } else {
-      if (!nc_from_ws)
-        for (int r = 0; r < Ri && ok; ++r) ok = xf_kv(r);
-      for (int j = 0; j < n_items && ok; ++j) ok = xf_q(j);
+      const int st = is_kv ? r % NKV : j % NQ;
+      const uint32_t par = is_kv ? (r / NKV) & 1 : (j / NQ) & 1;
+      ok = mbar_wait(is_kv ? &bars.kv_full[st] : &bars.q_full[st], par, abort_flag, a.err,
+                     kWaitLimitNs);
+      if (!ok) break;
+      uint8_t* tile = is_kv ? sK + st * KVT : sQ + st * QT;
+      // Q rows past the end of the sequence only feed output rows that are
+      // never stored, so a Q tile is always transformed whole
+      const int valid = is_kv ? min(kChunk, ntok - (c0 + r) * kChunk) : kChunk;
+      if (valid >= kChunk) {
+        phi_tile_full<D / 64, kXf>(tile, x);
+      } else {
+        // ragged end: phi on K with the rows past it zeroed, and those V rows zeroed
+#pragma unroll 1
+        for (int u = 0; u < 2; ++u) xf_tile<D / 64, kXf>(tile + u * KT, valid, u == 0, x);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, kXf);
+      if (x == 0) mbar_arrive(is_kv ? &bars.kv_xf[st] : &bars.q_xf[st]);
     }
   } else if (warp < 12) {
     // ---------------------------------------------------- mask warpgroup
@@ -494,14 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // the mask of item j+1 goes before the epilogue of item j: the mask is on
     // the path to the next MMAs, the epilogue only drains
-    if (causal) {
-      if (n_items > 0) ok = mask_p(0);
-      for (int j = 0; j < n_items && ok; ++j) {
-        if (j + 1 < n_items) ok = mask_p(j + 1);
-        if (ok) ok = epilogue(j);
-      }
-    } else {
-      for (int j = 0; j < n_items && ok; ++j) ok = epilogue(j);
+    for (int t = 0; t <= n_items && ok; ++t) {
+      if (causal && t < n_items) ok = mask_p(t);
+      if (ok && t > 0) ok = epilogue(t - 1);
     }
   } else if (warp < 16) {
     // -------------------------------------------------- state warpgroup
@@ -516,12 +516,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     uint32_t w[ACCW / 2];  // this thread's row of [S | z 0 ..], packed bf16
     // carry: the aggregates of the earlier blocks (causal) or of every block
-    // (non-causal), summed in fp32; zero without a workspace.  Causal: also
-    // the initial value of S_acc.
-    auto load_carry = [&](bool to_tmem) {
+    // (non-causal), summed in fp32, into S_acc (zero without a workspace;
+    // S_acc is otherwise unused in non-causal mode with a workspace)
+    auto load_carry = [&]() {
       const float* base = a.ws != nullptr ? a.ws + (size_t)(s * a.Hkv + g) * a.nb * E : nullptr;
       const int nprev = a.ws == nullptr ? 0 : (causal ? blk : a.nb);
-#pragma unroll
+#pragma unroll 1
       for (int q = 0; q < ACCW / 16; ++q) {
         float c[16];
 #pragma unroll
@@ -544,17 +544,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (to_tmem) {
-          uint32_t u16[16];
+        uint32_t u16[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) u16[e] = __float_as_uint(c[e]);
-          tmem_st16(t_s + q * 16, u16);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w[q * 8 + e] = pack_bf16x2(c[2 * e], c[2 * e + 1]);
+        for (int e = 0; e < 16; ++e) u16[e] = __float_as_uint(c[e]);
+        tmem_st16(t_s + q * 16, u16);
       }
-      if (to_tmem) tmem_wait_st();
+      tmem_wait_st();
     };
+    // S_acc -> w, rounded to bf16
     auto read_state = [&]() {
 #pragma unroll
       for (int q = 0; q < ACCW / 16; ++q) {
@@ -565,9 +562,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 8; ++e) w[q * 8 + e] = pack_bf16x2(c[2 * e], c[2 * e + 1]);
       }
     };
-    // w -> the operand (pieces of 8 columns; columns dv.. are [z 0 ..])
-    auto publish_sop = [&](int r) -> bool {
-      if (!mbar_wait(bars.sop_empty, (r & 1) ^ 1, abort_flag, a.err, kWaitLimitNs)) return false;
+    // Causal: step r publishes [S|z]_<r for chunk r; step 0 starts S_acc from
+    // the carry, step r > 0 reads it once the state product of chunk r-1 has
+    // landed, then releases it (phase r of s_empty) for the product of chunk
+    // r.  Non-causal: one step, with the carry or the state of this block.
+    const int nsteps = causal ? Ri : 1;
+    for (int r = 0; r < nsteps && ok; ++r) {
+      if (r == 0 && (causal || nc_from_ws)) {
+        load_carry();
+      } else {
+        ok = mbar_wait(bars.s_full, (causal ? r - 1 : 0) & 1, abort_flag, a.err, kWaitLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      read_state();
+      tc_fence_before();
+      if (causal) {
+        named_bar_sync(3, 128);
+        if (y == 0) mbar_arrive(bars.s_empty);
+      }
+      // w -> the operand (pieces of 8 columns; columns dv.. are [z 0 ..])
+      ok = mbar_wait(bars.sop_empty, (r & 1) ^ 1, abort_flag, a.err, kWaitLimitNs);
+      if (!ok) break;
       if (has_row) {
 #pragma unroll
         for (int q8 = 0; q8 < ACCW / 8; ++q8)
@@ -577,37 +593,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       named_bar_sync(3, 128);
       if (y == 0) mbar_arrive(bars.sop_full);
-      return true;
-    };
-    // phase r of s_empty: S_<r has been read (r = 0: the carry written)
-    auto release_state = [&]() {
-      tc_fence_before();
-      named_bar_sync(3, 128);
-      if (y == 0) mbar_arrive(bars.s_empty);
-    };
-    if (causal) {
-      load_carry(true);
-      release_state();
-      ok = publish_sop(0);
-      for (int r = 1; r < Ri && ok; ++r) {
-        ok = mbar_wait(bars.s_full, (r - 1) & 1, abort_flag, a.err, kWaitLimitNs);
-        if (!ok) break;
-        tc_fence_after();
-        read_state();
-        release_state();
-        ok = publish_sop(r);
-      }
-    } else if (nc_from_ws) {
-      load_carry(false);
-      ok = publish_sop(0);
-    } else {
-      ok = mbar_wait(bars.s_full, 0, abort_flag, a.err, kWaitLimitNs);
-      if (ok) {
-        tc_fence_after();
-        read_state();
-        tc_fence_before();
-        ok = publish_sop(0);
-      }
     }
   }
 
