@@ -705,12 +705,27 @@ cudaError_t launch_fwd_bf16_seq(const FwdLaunch& p, int nb, const float* ws,
 //   seq      the general kernel (one CTA per block of chunks) for d = dv = 64
 //            too; LT_BLOCKS=1 makes it fully sequential
 //   cluster  sequence split over a thread-block cluster (d = dv = 64)
+//   pair     the two-launch block scan (state launch, then forward launch)
+//            also where the one-launch cluster exchange applies
 static bool forced(char c) {
   const char* force = getenv("LT_KERNEL");
   return force && force[0] == c;
 }
 
+static bool use_block_fused(const FwdLaunch& p, int nb, int num_sms) {
+  return !forced('s') && !forced('p') && block_fused_supported(p, nb, num_sms);
+}
+
+static int current_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return sms;
+}
+
 cudaError_t launch_fwd_bf16_ws(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream) {
+  if (use_block_fused(p, nb, current_sms())) return launch_fwd_bf16_block_fused(p, nb, ws, stream);
   cudaError_t e = cudaSuccess;
   if (nb > 1) {
     e = launch_block_state(p, nb, ws, stream);
@@ -728,6 +743,11 @@ void plan_fwd_bf16(const FwdLaunch& p, int num_sms, int* nb, int* launches, size
     return;
   }
   *nb = block_count(p, num_sms);
+  if (use_block_fused(p, *nb, num_sms)) {
+    *launches = 1;
+    *ws_bytes = block_workspace_bytes(p, *nb);
+    return;
+  }
   *launches = *nb > 1 && (p.causal ? *nb - 1 : *nb) > 0 ? 2 : 1;
   *ws_bytes = block_workspace_bytes(p, *nb);
 }

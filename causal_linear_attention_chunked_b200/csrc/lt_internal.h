@@ -58,6 +58,13 @@ cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, const float* ws,
                                   cudaStream_t stream);
 cudaError_t launch_fwd_bf16_seq(const FwdLaunch& p, int nb, const float* ws,
                                 cudaStream_t stream);
+// d = dv = 64, dense, blocks of at most 4 chunks, one CTA per SM: one
+// cooperative launch in which every block publishes its aggregate to the
+// workspace, the CTAs meet at a grid barrier, and each block gathers its
+// carry from the others (the workspace of the two-launch path)
+bool block_fused_supported(const FwdLaunch& p, int nb, int num_sms);
+cudaError_t launch_fwd_bf16_block_fused(const FwdLaunch& p, int nb, float* ws,
+                                        cudaStream_t stream);
 // the per-device error word of the current device (looked up once per device)
 int* device_error_word_current();
 cudaError_t launch_fwd_f32(const FwdLaunch& p, cudaStream_t stream);

@@ -10,6 +10,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <cooperative_groups.h>
+
 namespace lt {
 
 // ----------------------------------------------------------------- errors
@@ -403,6 +405,46 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
         return false;
       }
     }
+  }
+}
+
+// ------------------------------------------------------------ grid barrier
+// Grid-wide barrier of a cooperative launch, on the barrier word the driver
+// provides to such a launch (the word and the flip-bit protocol of the
+// cooperative-groups grid synchronisation: every CTA adds 1 and block
+// (0,0,0) adds 2^31 - (ctas - 1), so the top bit flips once every CTA has
+// arrived and the low bits return to their former value).  One thread per
+// CTA, exactly once per CTA and launch, on every path.  wait = false:
+// arrive only.  The wait is bounded like mbar_wait.
+__device__ __forceinline__ bool grid_barrier(bool wait, volatile int* abort, int* err,
+                                             uint64_t limit_ns) {
+  cooperative_groups::details::grid_workspace* gw =
+      cooperative_groups::details::get_grid_workspace();
+  if (gw == nullptr) {  // not a cooperative launch
+    *abort = 1;
+    report_error(err, kDevErrTimeout);
+    return false;
+  }
+  unsigned int* bar = &gw->barrier;
+  const unsigned int ctas = gridDim.x * gridDim.y * gridDim.z;
+  const bool master = (blockIdx.x | blockIdx.y | blockIdx.z) == 0;
+  const unsigned int inc = master ? 0x80000000u - (ctas - 1u) : 1u;
+  unsigned int old;
+  asm volatile("atom.add.release.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(bar), "r"(inc)
+               : "memory");
+  if (!wait) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    unsigned int cur;
+    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(bar) : "memory");
+    if ((cur ^ old) & 0x80000000u) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      report_error(err, kDevErrTimeout);
+      return false;
+    }
+    __nanosleep(32);
   }
 }
 

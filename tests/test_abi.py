@@ -106,14 +106,17 @@ def test_oracle_and_library_share_no_code():
 
 @pytest.mark.parametrize("shape,expect", [
     # (B, H_q, H_kv, N, d, dv, causal, packed, dtype), num_sms = 148
-    ((2, 8, 8, 4096, 64, 64, 1, 0, 1), (8, 2, 2 * 8 * 8 * (64 * 64 + 64) * 4)),  # 9 -> 8 blocks of 4
+    # 9 -> 8 blocks of 4 chunks, 128 CTAs: one cooperative launch; the
+    # workspace holds the aggregates
+    ((2, 8, 8, 4096, 64, 64, 1, 0, 1), (8, 1, 2 * 8 * 8 * (64 * 64 + 64) * 4)),
+    ((2, 8, 8, 8192, 64, 64, 1, 0, 1), (8, 2, 2 * 8 * 8 * (64 * 64 + 64) * 4)),  # blocks of 8
     ((1, 8, 8, 65536, 64, 64, 0, 0, 1), (18, 2, 8 * 18 * (64 * 64 + 64) * 4)),
     ((2, 32, 8, 16384, 128, 128, 1, 0, 1), (9, 2, 2 * 8 * 9 * (128 * 128 + 128) * 4)),
     ((1, 1, 1, 300, 64, 128, 1, 0, 1), (3, 2, 3 * (64 * 128 + 64) * 4)),   # capped by 3 chunks
     ((1, 1, 1, 100, 64, 64, 1, 0, 1), (1, 1, 0)),                            # one chunk
     ((64, 8, 8, 50000, 64, 64, 1, 1, 1), (1, 1, 0)),                         # packed
     ((2, 8, 8, 4096, 64, 64, 1, 0, 0), (1, 1, 0)),                           # fp32 path
-    ((1, 2, 1, 8192, 64, 64, 1, 0, 1), (64, 2, 64 * (64 * 64 + 64) * 4)),  # 148 SMs, 64 chunks
+    ((1, 2, 1, 8192, 64, 64, 1, 0, 1), (64, 1, 64 * (64 * 64 + 64) * 4)),  # 64 chunks, one launch
 ])
 def test_fwd_plan_host_arithmetic(monkeypatch, shape, expect):
     """Blocks per sequence: the SM count over the (sequence, KV head) lanes,
@@ -128,6 +131,19 @@ def test_fwd_plan_host_arithmetic(monkeypatch, shape, expect):
                                        ctypes.byref(nb), ctypes.byref(nl), ctypes.byref(ws))
     assert st == 0
     assert (nb.value, nl.value, ws.value) == expect
+
+
+def test_fwd_plan_pair_forced(monkeypatch):
+    """LT_KERNEL=pair keeps the two-launch block scan where the one-launch
+    cluster exchange would apply."""
+    monkeypatch.delenv("LT_BLOCKS", raising=False)
+    monkeypatch.setenv("LT_KERNEL", "pair")
+    from causal_linear_attention_chunked_b200 import _binding as b
+    nb, nl, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    st = b.lib.lt_linear_attn_fwd_plan(2, 8, 8, 4096, 64, 64, 1, 0, 1, 148,
+                                       ctypes.byref(nb), ctypes.byref(nl), ctypes.byref(ws))
+    assert st == 0
+    assert (nb.value, nl.value, ws.value) == (8, 2, 2 * 8 * 8 * (64 * 64 + 64) * 4)
 
 
 @pytest.mark.parametrize("case,expect", [

@@ -198,18 +198,101 @@ BLOCK_CASES = [
 ]
 
 
+@pytest.mark.parametrize("mode", ["auto", "pair"])
 @pytest.mark.parametrize("nb", [1, 2, 3, 5, 8])
 @pytest.mark.parametrize("case", BLOCK_CASES, ids=lambda c: "B%dHq%dHkv%dN%d%s" % (
     c[0], c[1], c[2], c[3], "c" if c[4] else "nc"))
-def test_block_kernel_block_counts(monkeypatch, nb, case):
-    """d = dv = 64: block aggregates in a first launch, then one CTA per block
-    from the carried prefix.  LT_BLOCKS forces the number of blocks."""
+def test_block_kernel_block_counts(monkeypatch, nb, case, mode):
+    """d = dv = 64, the sequence cut into nb blocks (LT_BLOCKS).  "pair": the
+    block aggregates in a first launch, then one CTA per block from the
+    carried prefix.  "auto": blocks of at most four chunks, at most eight of
+    them, run as one launch whose blocks form a cluster and exchange their
+    aggregates in shared memory; other shapes as "pair"."""
     monkeypatch.setenv("LT_BLOCKS", str(nb))
+    if mode == "pair":
+        monkeypatch.setenv("LT_KERNEL", "pair")
+    else:
+        monkeypatch.delenv("LT_KERNEL", raising=False)
     B, Hq, Hkv, N, causal = case
     q, k, v = inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16, 0.125, seed=N + 7 * nb)
     got = run_dense(q, k, v, causal)
     ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
     assert row_rel_err(got, ref) <= TOL_BF16
+
+
+FUSED_CASES = [
+    # (B, Hq, Hkv, N, causal, forced block count or 0): one cooperative launch
+    # in which the blocks publish and gather the aggregates themselves
+    (2, 8, 8, 4096, True, 0),        # the headline shape: 8 blocks of 4 chunks
+    (4, 8, 8, 2000, True, 0),        # 4 blocks of 4 chunks, ragged last chunk
+    (1, 4, 4, 7 * 128 + 117, True, 0),  # 8 blocks of 1 chunk
+    (2, 4, 1, 1000, True, 0),        # 4 query heads per KV head
+    (1, 8, 2, 3000, True, 6),        # GQA, 6 blocks of 4 chunks
+    (1, 2, 2, 1024, False, 0),
+    (3, 2, 2, 900, False, 0),
+    (1, 4, 2, 1500, False, 3),       # 3 blocks of 4 chunks
+]
+
+
+@pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: "B%dHq%dHkv%dN%d%s%s" % (
+    c[0], c[1], c[2], c[3], "c" if c[4] else "nc", "-nb%d" % c[5] if c[5] else ""))
+def test_fused_launch_matches_two_launches_bitwise(monkeypatch, case):
+    """The one-launch path and the two-launch path compute the same block
+    aggregates with the same products and sum the carry in the same block
+    order, so their outputs agree bit for bit; both match the oracle."""
+    import causal_linear_attention_chunked_b200 as L
+    B, Hq, Hkv, N, causal, nb_forced = case
+    monkeypatch.delenv("LT_KERNEL", raising=False)
+    if nb_forced:
+        monkeypatch.setenv("LT_BLOCKS", str(nb_forced))
+    else:
+        monkeypatch.delenv("LT_BLOCKS", raising=False)
+    nb, launches, ws = L.linear_attn_fwd_plan(B, Hq, Hkv, N, 64, 64, causal=causal)
+    assert nb >= 2 and launches == 1 and ws > 0
+    q, k, v = inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16, 0.125, seed=N + B)
+    one = run_dense(q, k, v, causal)
+    monkeypatch.setenv("LT_KERNEL", "pair")
+    assert L.linear_attn_fwd_plan(B, Hq, Hkv, N, 64, 64, causal=causal)[1] == 2
+    two = run_dense(q, k, v, causal)
+    assert np.array_equal(one, two)
+    ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
+    assert row_rel_err(one, ref) <= TOL_BF16
+
+
+def test_fused_launch_in_cuda_graph_replays_with_new_inputs(monkeypatch):
+    """A captured one-launch call replayed with new input contents: each
+    replay publishes its own aggregates and meets at its own grid barrier,
+    so no replay takes another replay's aggregates for its own."""
+    import causal_linear_attention_chunked_b200 as L
+    monkeypatch.delenv("LT_BLOCKS", raising=False)
+    monkeypatch.delenv("LT_KERNEL", raising=False)
+    B, Hq, Hkv, N = 2, 8, 8, 4096
+    assert L.linear_attn_fwd_plan(B, Hq, Hkv, N, 64, 64, causal=True)[1] == 1
+    q, k, v = (t.cuda() for t in inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16,
+                                                     0.125, seed=900))
+    out = torch.empty((B, N, Hq, 64), dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        L.linear_attn_fwd(q, k, v, causal=True, out=out, stream=s)  # warm-up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        L.linear_attn_fwd(q, k, v, causal=True, out=out, stream=s)
+    for seed in (901, 902, 903):
+        q2, k2, v2 = inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16, 0.125, seed=seed)
+        q.copy_(q2)
+        k.copy_(k2)
+        v.copy_(v2)
+        out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert L.get_last_device_error() == 0
+        sel = np.array([(b, n, h) for b in range(B) for n in (0, 1, 511, 512, 2047, 2048, 3000, 4095)
+                        for h in range(Hq)])
+        ref = oracle.fwd_rows(q2, k2, v2, sel, causal=True, eps=1e-6)
+        o = out.float().cpu().numpy()
+        got = o[sel[:, 0], sel[:, 1], sel[:, 2]]
+        assert row_rel_err(got, ref) <= TOL_BF16
 
 
 def test_block_kernel_deterministic_across_block_counts(monkeypatch):

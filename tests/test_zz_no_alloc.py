@@ -44,7 +44,8 @@ def test_noalloc_matches_allocating_entry_point_on_consecutive_calls(monkeypatch
     cases = [
         # (B, Hq, Hkv, N, d, dv, causal): each cuts its sequences into
         # several blocks, so each call writes and reads the fixed array
-        ((2, 8, 8, 4096, 64, 64), True),
+        ((2, 8, 8, 4096, 64, 64), True),   # one cooperative launch
+        ((2, 8, 8, 8192, 64, 64), True),   # two launches
         ((1, 8, 2, 3000, 128, 128), False),
         ((1, 4, 2, 2000, 128, 64), True),
     ]
