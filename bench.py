@@ -402,9 +402,13 @@ def run_lt(args):
     packed = w.packed_len is not None
     nblk, per_step, ws_bytes = L.linear_attn_fwd_plan(w.B, w.Hq, w.Hkv, 1 if packed else w.N,
                                                       w.d, w.dv, causal=w.causal, packed=packed)
-    kern = ("lt_block_state_kernel + lt_block_fwd_kernel" if w.d == 64 and w.dv == 64 else
-            "lt_block_state_kernel + lt_fwd_bf16_kernel") if per_step == 2 else (
-            "lt_block_fwd_kernel" if w.d == 64 and w.dv == 64 else "lt_fwd_bf16_kernel")
+    d64 = w.d == 64 and w.dv == 64
+    if per_step == 2:
+        kern = "lt_block_state_kernel + " + ("lt_block_fwd_kernel" if d64 else "lt_fwd_bf16_kernel")
+    elif d64 and nblk > 1:
+        kern = "lt_fused_fwd_kernel (one cooperative launch)"
+    else:
+        kern = "lt_block_fwd_kernel" if d64 else "lt_fwd_bf16_kernel"
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,

@@ -63,10 +63,6 @@ struct BlockArgs {
   float eps;
   int total_tokens;
   int* err;
-  // fused: one cooperative launch in which every block first publishes its
-  // own aggregate to ws, all CTAs meet at a grid barrier, and each block
-  // then gathers its carry itself
-  int fused;
 };
 
 __device__ __forceinline__ bool seq_bounds(const BlockArgs& a, int s, int& t0, int& n) {
@@ -87,7 +83,7 @@ __device__ __forceinline__ bool seq_bounds(const BlockArgs& a, int s, int& t0, i
 // ========================================================================
 constexpr int kThreads = 576;
 constexpr int kXf = 256;  // transform threads (warps 0-7, two per SM sub-partition)
-constexpr int NQ = 3, NKV = 4, NSOP = 2;
+constexpr int NQ = 4, NKV = 4;
 // two score tiles (item j uses j & 1), two accumulators, the running state
 constexpr int TM_P = 0, TM_ACC = 2 * kChunk, TM_S = TM_ACC + 2 * ACCW, TM_COLS = 512;
 static_assert(TM_S + ACCW <= TM_COLS, "TMEM budget");
@@ -95,9 +91,9 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + NQ * QT;  // stage st: [K][V] at st*KVT
 constexpr int OFF_ONES = OFF_KV + NKV * KVT;
 constexpr int OFF_SOP = OFF_ONES + ONEST;
-constexpr int OFF_BAR = OFF_SOP + NSOP * SOPT;
-constexpr int NBARS = 3 * NQ + 3 * NKV + 2 * 2 + 2 * NSOP + 2 + 2 * 2 + 1 + 1;
-static_assert(NSOP * SOPT >= E * 4, "the carry is staged in the state operand buffers");
+constexpr int OFF_Z = OFF_SOP + SOPT;
+constexpr int OFF_BAR = OFF_Z + D * 4;
+constexpr int NBARS = 3 * NQ + 3 * NKV + 2 * 2 + 2 + 2 + 2 * 2 + 1;
 constexpr int SMEM = OFF_BAR + NBARS * 8 + 16 + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
 
@@ -105,7 +101,6 @@ struct Bars {
   uint64_t *q_full, *q_empty, *q_xf, *kv_full, *kv_empty, *kv_xf;
   uint64_t *p_full, *pb_full, *sop_full, *sop_empty;
   uint64_t *s_full, *s_empty, *acc_full, *acc_empty, *drain;
-  uint64_t* agg_full;  // fused mode: the block aggregate is in S_acc
 };
 
 __device__ __forceinline__ Bars carve(uint8_t* base) {
@@ -119,43 +114,46 @@ __device__ __forceinline__ Bars carve(uint8_t* base) {
   r.kv_xf = b; b += NKV;
   r.p_full = b; b += 2;
   r.pb_full = b; b += 2;
-  r.sop_full = b; b += NSOP;
-  r.sop_empty = b; b += NSOP;
+  r.sop_full = b++;
+  r.sop_empty = b++;
   r.s_full = b++;
   r.s_empty = b++;
   r.acc_full = b; b += 2;
   r.acc_empty = b; b += 2;
   r.drain = b++;
-  r.agg_full = b++;
   return r;
 }
 
 // Sum, in block order, of the aggregates of blocks [0, nsum) of one lane
-// (base: that lane's first aggregate) into stage (fp32, E floats): thread u of
-// NT sums the float4s u, u + NT, ...; the loads of four blocks are in flight
-// together.
+// (base: that lane's first aggregate) into fp32 stages (S: d*dv floats, z: d
+// floats).  Thread u of NT sums the S float4s u, u + NT, ... and, for
+// u < d/4, z float4 u; the loads of four blocks are in flight together.
 template <int NT>
-__device__ __forceinline__ void sum_aggregates(const float4* base, int nsum, float* stage, int u) {
-  constexpr int E4 = E / 4, PER = (E4 + NT - 1) / NT;
-  float4 acc[PER];
+__device__ __forceinline__ void sum_aggregates(const float4* base, int nsum, float* stage_s,
+                                               float* stage_z, int u) {
+  constexpr int E4 = E / 4, S4 = D * DV / 4, PER = (S4 + NT - 1) / NT;
+  const bool has_z = u < D / 4;
+  float4 acc[PER + 1];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int e = 0; e <= PER; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
   for (int b0 = 0; b0 < nsum; b0 += 4) {
-    float4 v[4][PER];
+    float4 v[4][PER + 1];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       if (b0 + k < nsum) {
+        const float4* blkp = base + (size_t)(b0 + k) * E4;
 #pragma unroll
         for (int e = 0; e < PER; ++e)
-          if (u + e * NT < E4) v[k][e] = __ldcg(base + (size_t)(b0 + k) * E4 + u + e * NT);
+          if (u + e * NT < S4) v[k][e] = __ldcg(blkp + u + e * NT);
+        if (has_z) v[k][PER] = __ldcg(blkp + S4 + u);
       }
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       if (b0 + k < nsum) {
 #pragma unroll
-        for (int e = 0; e < PER; ++e) {
+        for (int e = 0; e <= PER; ++e) {
           acc[e].x += v[k][e].x;
           acc[e].y += v[k][e].y;
           acc[e].z += v[k][e].z;
@@ -164,12 +162,17 @@ __device__ __forceinline__ void sum_aggregates(const float4* base, int nsum, flo
       }
     }
   }
-  float4* st4 = reinterpret_cast<float4*>(stage);
 #pragma unroll
   for (int e = 0; e < PER; ++e)
-    if (u + e * NT < E4) st4[u + e * NT] = acc[e];
+    if (u + e * NT < S4) reinterpret_cast<float4*>(stage_s)[u + e * NT] = acc[e];
+  if (has_z) reinterpret_cast<float4*>(stage_z)[u] = acc[PER];
 }
 
+// kCarry: the sequence is cut into several blocks and this launch starts
+// each from the aggregates of the state launch.  Without it (one block per
+// sequence, e.g. packed inputs) the carry code is left out of the image: the
+// instruction working set of the warp roles matters to this kernel's speed.
+template <bool kCarry>
 __global__ void __launch_bounds__(kThreads, 1)
     lt_block_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -187,21 +190,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int nc = (ntok + kChunk - 1) / kChunk;
   const int c0 = blk * a.bc, c1 = min(c0 + a.bc, nc);
-  if (c1 <= c0) return;  // nothing in this block (uniform over the CTA; never in fused mode)
+  if (c1 <= c0) return;  // nothing in this block (uniform over the CTA)
   const int Ri = c1 - c0;  // chunks of this block, walked in order
   const int G = a.G;
   const bool causal = a.causal != 0;
   const int n_items = Ri * G;
   // non-causal with a workspace: the state is the sum of all blocks and this
   // CTA reads only Q
-  const bool fused = a.fused != 0;
-  const bool nc_from_ws = !causal && a.ws != nullptr && !fused;
-  // fused mode: this CTA first reduces its block's K, V to the aggregate
-  // (phase A) and publishes it, then gathers the carry from the aggregates
-  // the other CTAs of the launch publish; the K/V ring holds every chunk of
-  // the block, so each tile is loaded once
-  // non-causal and the whole state comes from the carry
-  const bool nc_carry = !causal && (nc_from_ws || fused);
+  const bool nc_from_ws = !causal && a.ws != nullptr;
 
   uint8_t* sQ = smem + OFF_Q;
   uint8_t* sK = smem + OFF_KV;
@@ -222,10 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.kv_empty[i], 1);
       mbar_init(&bars.kv_xf[i], 1);
     }
-    for (int i = 0; i < NSOP; ++i) {
-      mbar_init(&bars.sop_full[i], 1);
-      mbar_init(&bars.sop_empty[i], 1);
-    }
+    mbar_init(bars.sop_full, 1);
+    mbar_init(bars.sop_empty, 1);
     mbar_init(bars.s_full, 1);
     mbar_init(bars.s_empty, 1);
     for (int i = 0; i < 2; ++i) {
@@ -235,7 +229,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.acc_empty[i], 1);
     }
     mbar_init(bars.drain, 1);
-    mbar_init(bars.agg_full, 1);
     fence_mbar_init();
   }
   init_ones_block(smem + OFF_ONES, tid, kThreads);
@@ -246,35 +239,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int* abort_flag = &s_abort;
-
   // Carry: the aggregates of the earlier blocks (causal) or of every block
-  // (non-causal), summed in fp32 in block order into the state operand
-  // buffers (free until the state warps first stage [S|z]).  Warps 0-15
-  // share the work so that the loads of several blocks are in flight at
-  // once; the state warps read the sum after named barrier 4.
-  // the number of aggregates in the carry, and where this lane's aggregates
-  // start; the sum is staged (fp32) in the state operand buffers, free until
-  // the state warps first stage [S|z]
-  const int nprev = a.ws == nullptr ? 0 : (causal ? blk : a.nb);
-  const float4* agg_base =
-      a.ws == nullptr ? nullptr
-                      : reinterpret_cast<const float4*>(a.ws) + (size_t)(s * a.Hkv + g) * a.nb * (E / 4);
-  float* carry_stage = reinterpret_cast<float*>(smem + OFF_SOP);
-  if (!fused && nprev > 0 && warp < 16) {
-    // two-launch mode: the aggregates are complete; warps 0-15 sum them
-    sum_aggregates<512>(agg_base, nprev, carry_stage, tid);
+  // (non-causal), summed in fp32 in block order by warps 0-15 (the loads of
+  // several blocks in flight at once) into the state operand buffer and the
+  // z slot, which the state warps read after named barrier 4
+  const int nprev = (!kCarry || a.ws == nullptr) ? 0 : (causal ? blk : a.nb);
+  float* carry_s = reinterpret_cast<float*>(smem + OFF_SOP);
+  float* carry_z = reinterpret_cast<float*>(smem + OFF_Z);
+  if (kCarry && nprev > 0 && warp < 16) {
+    sum_aggregates<512>(reinterpret_cast<const float4*>(a.ws) + (size_t)(s * a.Hkv + g) * a.nb * (E / 4),
+                        nprev, carry_s, carry_z, tid);
     named_bar_sync(4, 512);
   }
-  // fused mode: the transform warps and the state warps (384 threads) sum the
-  // aggregates between two barriers 5, once the state warps have seen every
-  // needed flag.  Both groups pass both barriers on every path (an abort
-  // skips only the loads), so no barrier is left waiting.
-  const bool gather = fused && nprev > 0;
-  auto gather_part = [&](int u) {
-    named_bar_sync(5, 384);
-    if (!*abort_flag) sum_aggregates<384>(agg_base, nprev, carry_stage, u);
-    named_bar_sync(5, 384);
-  };
 
   if (warp == 16) {
     // ------------------------------------------------------------ producer
@@ -303,12 +279,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++q_issued;
         return true;
       };
-      if (causal && !fused) {
+      if (causal) {
         for (int r = 0; r < Ri && ok; ++r) {
           ok = load_kv(r);
           for (int h = 0; h < G && ok; ++h) ok = load_q(r * G + h);
         }
-      } else {  // every K/V tile first (non-causal, or phase A of fused mode)
+      } else {
         if (!nc_from_ws)
           for (int r = 0; r < Ri && ok; ++r) ok = load_kv(r);
         for (int j = 0; j < n_items && ok; ++j) ok = load_q(j);
@@ -349,26 +325,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                       (accumulate || kk > 0) ? 1u : 0u);
       };
       // Acc (+)= phi(Q) [S | z 0 ..]
-      auto issue_qs = [&](uint32_t t_acc, int qs, int sb, bool accumulate) {
+      auto issue_qs = [&](uint32_t t_acc, int qs, bool accumulate) {
         const uint64_t qa = desc_advance(dQk, qs * QT);
-        const uint64_t sd = desc_advance(dSop, sb * SOPT);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           umma_f16_ss(t_acc, desc_advance(qa, (kk >> 2) * kBox + (kk & 3) * 32),
-                      desc_advance(sd, kk * 2048), ID_QS, (accumulate || kk > 0) ? 1u : 0u);
+                      desc_advance(dSop, kk * 2048), ID_QS, (accumulate || kk > 0) ? 1u : 0u);
       };
-      if (fused) {
-        // phase A: S_acc = this block's aggregate sum_r phi(K_r)^T [V_r | 1]
-        for (int r = 0; r < Ri && ok; ++r) {
-          ok = mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs);
-          if (!ok) break;
-          tc_fence_after();
-          issue_ds(r, tmem + TM_S, r > 0);
-        }
-        if (ok) umma_commit(bars.agg_full);
-      }
-      if (!ok) {
-      } else if (causal) {
+      if (causal) {
         // S_acc += dS of chunk r, once the state warpgroup has read S_<r
         // (phase r of s_empty; phase 0 is the carry it wrote).  Only chunks
         // before the block's last one feed a later state.
@@ -430,18 +394,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ID_PV, kk > 0 ? 1u : 0u);
           if (h == G - 1) umma_commit(&bars.kv_empty[r % NKV]);
           if (h == 0) {
-            ok = mbar_wait(&bars.sop_full[r % NSOP], (r / NSOP) & 1, abort_flag, a.err,
-                           kWaitLimitNs);
+            ok = mbar_wait(bars.sop_full, r & 1, abort_flag, a.err, kWaitLimitNs);
             if (!ok) break;
             tc_fence_after();
           }
-          issue_qs(t_acc, qs, r % NSOP, true);
+          issue_qs(t_acc, qs, true);
           umma_commit(&bars.acc_full[as]);
           umma_commit(&bars.q_empty[qs]);
-          if (h == G - 1) umma_commit(&bars.sop_empty[r % NSOP]);
+          if (h == G - 1) umma_commit(bars.sop_empty);
         }
       } else {
-        if (!nc_carry) {
+        if (!nc_from_ws) {
           for (int r = 0; r < Ri && ok; ++r) {
             ok = mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs);
             if (!ok) break;
@@ -451,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (ok) umma_commit(bars.s_full);
         }
-        if (ok) ok = mbar_wait(&bars.sop_full[0], 0, abort_flag, a.err, kWaitLimitNs);
+        if (ok) ok = mbar_wait(bars.sop_full, 0, abort_flag, a.err, kWaitLimitNs);
         for (int j = 0; j < n_items && ok; ++j) {
           const int qs = j % NQ, as = j & 1;
           ok = mbar_wait(&bars.q_xf[qs], (j / NQ) & 1, abort_flag, a.err, kWaitLimitNs) &&
@@ -459,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          kWaitLimitNs);
           if (!ok) break;
           tc_fence_after();
-          issue_qs(tmem + TM_ACC + as * ACCW, qs, 0, false);
+          issue_qs(tmem + TM_ACC + as * ACCW, qs, false);
           umma_commit(&bars.acc_full[as]);
           umma_commit(&bars.q_empty[qs]);
         }
@@ -477,15 +440,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // each head of chunk r; non-causal: every K, then every Q), so that the
     // transform code exists once in the kernel image.
     const int nkv = nc_from_ws ? 0 : Ri;
-    const int T = (causal && !fused) ? Ri * (G + 1) : nkv + n_items;
-    // fused mode: the Q tiles past the ring wait for a product that needs the
-    // carry, so the gather comes after the first NQ of them
-    const int join_t = nkv + min(n_items, NQ) - 1;
-    bool joined = !gather;
+    const int T = causal ? Ri * (G + 1) : nkv + n_items;
     for (int t = 0; t < T && ok; ++t) {
       bool is_kv;
       int r, j;
-      if (causal && !fused) {
+      if (causal) {
         r = t / (G + 1);
         const int k = t - r * (G + 1);
         is_kv = k == 0;
@@ -514,12 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       named_bar_sync(1, kXf);
       if (x == 0) mbar_arrive(is_kv ? &bars.kv_xf[st] : &bars.q_xf[st]);
-      if (!joined && t == join_t) {
-        gather_part(x);
-        joined = true;
-      }
     }
-    if (!joined) gather_part(x);  // after an abort: keep the barrier sequence
   } else if (warp < 12) {
     // ---------------------------------------------------- mask warpgroup
     const int x = tid - 256, sp = warp & 3;
@@ -625,53 +579,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = sp * 16 + lane;
     bool ok = true;
     uint32_t w[ACCW / 2];  // this thread's row of [S | z 0 ..], packed bf16
-    const float* cS = carry_stage;
-    const float* cZ = carry_stage + D * DV;
-    const bool have_carry = nprev > 0;
-    // Fused mode, before the first chunk: S_acc holds this block's aggregate
-    // (phase A).  Publish it to the workspace (causal: unless this is the
-    // last block, whose aggregate no block needs); every CTA arrives once at
-    // the grid barrier, on every path; a CTA with a carry waits there, then
-    // sums the aggregates together with the transform warps.
-    auto publish_and_gather = [&](bool do_gather) {
-      const bool pok = mbar_wait(bars.agg_full, 0, abort_flag, a.err, kWaitLimitNs);
-      tc_fence_after();
-      if (pok && (!causal || blk + 1 < a.nb)) {
-        float* dst = a.ws + ((size_t)(s * a.Hkv + g) * a.nb + blk) * E;
-#pragma unroll
-        for (int q = 0; q < ACCW / 16; ++q) {
-          float c[16];
-          tmem_ld16(t_s + q * 16, c);
-          tmem_wait_ld();
-          if (has_row) {
-            if (q < DV / 16) {
-              float4* d4 = reinterpret_cast<float4*>(dst + row * DV + q * 16);
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                d4[u] = make_float4(c[4 * u], c[4 * u + 1], c[4 * u + 2], c[4 * u + 3]);
-            } else {
-              dst[D * DV + row] = c[0];
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      __threadfence();
-      named_bar_sync(3, 128);
-      if (y == 0) grid_barrier(do_gather, abort_flag, a.err, kWaitLimitNs);
-      if (do_gather) gather_part(256 + y);
-    };
-    // step 0: the carry (zero without earlier blocks) -> w and, in causal
-    // mode, the starting value of S_acc
+    // carry: the staged sum (zero without earlier blocks) into S_acc
     auto load_carry = [&]() {
-#pragma unroll
+#pragma unroll 1
       for (int q = 0; q < ACCW / 16; ++q) {
         float c[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) c[e] = 0.0f;
-        if (have_carry && has_row) {
+        if (kCarry && nprev > 0 && has_row) {
           if (q < DV / 16) {
-            const float4* r4 = reinterpret_cast<const float4*>(cS + row * DV + q * 16);
+            const float4* r4 = reinterpret_cast<const float4*>(carry_s + row * DV + q * 16);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const float4 v = r4[u];
@@ -681,19 +598,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               c[4 * u + 3] = v.w;
             }
           } else {
-            c[0] = cZ[row];
+            c[0] = carry_z[row];
           }
         }
-        if (causal) {
-          uint32_t u16[16];
+        uint32_t u16[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) u16[e] = __float_as_uint(c[e]);
-          tmem_st16(t_s + q * 16, u16);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w[q * 8 + e] = pack_bf16x2(c[2 * e], c[2 * e + 1]);
+        for (int e = 0; e < 16; ++e) u16[e] = __float_as_uint(c[e]);
+        tmem_st16(t_s + q * 16, u16);
       }
-      if (causal) tmem_wait_st();
+      tmem_wait_st();
     };
     // S_acc -> w, rounded to bf16
     auto read_state = [&]() {
@@ -710,42 +623,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the carry, step r > 0 reads it once the state product of chunk r-1 has
     // landed, then releases it (phase r of s_empty) for the product of chunk
     // r.  Non-causal: one step, with the carry or the state of this block.
-    // The operand of chunk r goes to buffer r % NSOP, so staging chunk r
-    // waits only for the last product that read chunk r - NSOP's operand.
-    // Step 0 reads the carry from the operand buffers themselves: barrier 3
-    // below orders every thread's read before the first operand write.
-    if (fused) {
-      // causal block 0 has no carry but publishes its aggregate
-      publish_and_gather(gather);
-      ok = !*abort_flag;
-    }
     const int nsteps = causal ? Ri : 1;
     for (int r = 0; r < nsteps && ok; ++r) {
-      if (r == 0 && (causal || nc_carry)) {
+      if (r == 0 && (causal || nc_from_ws)) {
         load_carry();
       } else {
         ok = mbar_wait(bars.s_full, (causal ? r - 1 : 0) & 1, abort_flag, a.err, kWaitLimitNs);
         if (!ok) break;
         tc_fence_after();
-        read_state();
       }
+      read_state();
       tc_fence_before();
+      // also orders every thread's read of the staged carry (in the operand
+      // buffer) before the operand is written
       named_bar_sync(3, 128);
       if (causal && y == 0) mbar_arrive(bars.s_empty);
       // w -> the operand (pieces of 8 columns; columns dv.. are [z 0 ..])
-      const int sb = r % NSOP;
-      ok = mbar_wait(&bars.sop_empty[sb], ((r / NSOP) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs);
+      ok = mbar_wait(bars.sop_empty, (r & 1) ^ 1, abort_flag, a.err, kWaitLimitNs);
       if (!ok) break;
       if (has_row) {
-        uint8_t* sop = sSOP + sb * SOPT;
 #pragma unroll
         for (int q8 = 0; q8 < ACCW / 8; ++q8)
-          *reinterpret_cast<uint4*>(sop + (q8 >> 3) * (D * kRowBytes) + sw128_off(row, q8 & 7)) =
+          *reinterpret_cast<uint4*>(sSOP + (q8 >> 3) * (D * kRowBytes) + sw128_off(row, q8 & 7)) =
               make_uint4(w[4 * q8], w[4 * q8 + 1], w[4 * q8 + 2], w[4 * q8 + 3]);
       }
       fence_proxy_async_smem();
       named_bar_sync(3, 128);
-      if (y == 0) mbar_arrive(&bars.sop_full[sb]);
+      if (y == 0) mbar_arrive(bars.sop_full);
     }
   }
 
@@ -761,19 +665,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool block_supported(const FwdLaunch& p) { return p.d == 64 && p.dv == 64; }
 
-// One launch: dense sequences whose blocks fit the K/V ring (every tile is
-// loaded once) and whose CTAs are all resident at once (one per SM; the
-// launch is cooperative, so it fails rather than run them in waves).  Every
-// block must hold at least one chunk: an empty block would publish nothing.
-bool block_fused_supported(const FwdLaunch& p, int nb, int num_sms) {
-  if (!block_supported(p) || p.cu_seqlens != nullptr || nb < 2) return false;
-  const int nc = (p.N + kChunk - 1) / kChunk, bc = block_chunks(p, nb);
-  return bc <= NKV && (long long)(nb - 1) * bc < nc &&
-         (long long)nb * p.Hkv * p.B <= (long long)num_sms;
-}
-
-static cudaError_t launch_block(const FwdLaunch& p, int nb, float* ws, bool fused,
-                                cudaStream_t stream) {
+cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, const float* ws,
+                                  cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
   if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
       !make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64) ||
@@ -782,7 +675,7 @@ static cudaError_t launch_block(const FwdLaunch& p, int nb, float* ws, bool fuse
   BlockArgs a;
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
   a.cu_seqlens = p.cu_seqlens;
-  a.ws = nb > 1 ? ws : nullptr;
+  a.ws = nb > 1 ? const_cast<float*>(ws) : nullptr;
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
   a.N = p.N;
@@ -793,36 +686,11 @@ static cudaError_t launch_block(const FwdLaunch& p, int nb, float* ws, bool fuse
   a.eps = p.eps;
   a.total_tokens = (int)p.total_tokens;
   a.err = p.err;
-  a.fused = fused ? 1 : 0;
-  auto fk = lt_block_fwd_kernel;
+  auto fk = (nb > 1 && ws != nullptr) ? lt_block_fwd_kernel<true> : lt_block_fwd_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  if (!fused) {
-    fk<<<dim3(nb, p.Hkv, p.B), kThreads, SMEM, stream>>>(tq, tk, tv, a);
-    return cudaGetLastError();
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(nb, p.Hkv, p.B);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = SMEM;
-  cfg.stream = stream;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeCooperative;
-  at[0].val.cooperative = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fk, tq, tk, tv, a);
-}
-
-cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, const float* ws,
-                                  cudaStream_t stream) {
-  return launch_block(p, nb, const_cast<float*>(ws), false, stream);
-}
-
-cudaError_t launch_fwd_bf16_block_fused(const FwdLaunch& p, int nb, float* ws,
-                                        cudaStream_t stream) {
-  if (ws == nullptr) return cudaErrorInvalidValue;
-  return launch_block(p, nb, ws, true, stream);
+  fk<<<dim3(nb, p.Hkv, p.B), kThreads, SMEM, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
 }
 
 }  // namespace lt

@@ -52,7 +52,8 @@ int block_count(const FwdLaunch& p, int num_sms);
 int block_chunks(const FwdLaunch& p, int nb);
 size_t block_workspace_bytes(const FwdLaunch& p, int nb);
 cudaError_t launch_block_state(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream);
-// forward launches: d = dv = 64 specialised kernel; every width pair
+// forward launches: d = dv = 64 specialised kernel (the carry, when nb > 1,
+// from the state launch's aggregates); every width pair
 bool block_supported(const FwdLaunch& p);
 cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, const float* ws,
                                   cudaStream_t stream);
