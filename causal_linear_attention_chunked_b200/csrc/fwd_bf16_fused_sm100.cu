@@ -186,9 +186,13 @@ __device__ __forceinline__ void sum_aggregates(const float4* base, int nsum, flo
       }
     }
   }
+  // S is staged with the float4 index of a row XOR-ed with the row, so that
+  // the state warps, one row per thread, read it without bank conflicts
 #pragma unroll
-  for (int e = 0; e < PER; ++e)
-    if (u + e * NT < S4) reinterpret_cast<float4*>(stage_s)[u + e * NT] = acc[e];
+  for (int e = 0; e < PER; ++e) {
+    const int i = u + e * NT;
+    if (i < S4) reinterpret_cast<float4*>(stage_s)[(i & ~15) | ((i ^ (i >> 4)) & 15)] = acc[e];
+  }
   if (has_z) reinterpret_cast<float4*>(stage_z)[u] = acc[PER];
 }
 
@@ -418,46 +422,38 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
           }
           umma_commit(&bars.p_full[t & 1]);
         };
-        // single issuer: S_acc += dS of chunk r, once the state warpgroup has
-        // read S_<r (phase r of s_empty); chunks before the last only
-        auto state_mma = [&](int r) -> bool {
-          if (r + 1 >= Ri) return true;
-          if (!mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs) ||
-              !mbar_wait(bars.s_empty, r & 1, abort_flag, a.err, kWaitLimitNs))
-            return false;
-          tc_fence_after();
-          issue_ds(r, tmem + TM_S, true);
-          umma_commit(bars.s_full);
-          return true;
-        };
-        for (int t = 0; t <= n_items && ok; ++t) {
-          // item t's score ahead of item t-1's products, so that its mask
-          // overlaps them (split: only when its tiles are ready already)
-          bool scored = false;
-          if (t < n_items && (!kSplit || score_ready(t))) {
-            if (!kSplit) {
-              const int r = t / G;
-              ok = mbar_wait(&bars.q_xf[t % NQ], (t / NQ) & 1, abort_flag, a.err, kWaitLimitNs) &&
-                   mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err,
-                             kWaitLimitNs);
-              if (!ok) break;
-            }
+        // Issue by polling, so that products whose inputs are ready never
+        // wait behind one whose inputs are late (the first items' scores,
+        // masks and P V run while the carry is still being gathered):
+        //   QS(j)  once P V(j) is issued and the chunk's operand is staged
+        //   SC(j)  once its tiles are ready and P V(j-2) (the last user of
+        //          TMEM buffer j & 1) is issued
+        //   PV(j)  once the mask warps have rounded P(j) and the epilogue has
+        //          drained accumulator j & 1
+        int sc = 0, pv = 0, qn = 0;
+        uint32_t idle = 0;
+        uint64_t idle_t0 = 0;
+        while (qn < n_items && ok) {
+          bool did = false;
+          if (qn < pv && (qn % G != 0 || mbar_test(&bars.sop_full[(qn / G) % NSOP],
+                                                     ((qn / G) / NSOP) & 1))) {
             tc_fence_after();
-            score(t);
-            scored = true;
-            if (!kSplit && t % G == 0) {
-              ok = state_mma(t / G);
-              if (!ok) break;
-            }
-          }
-          if (t > 0) {
-            const int j = t - 1;
-            const int r = j / G, h = j % G, as = j & 1;
-            ok = mbar_wait(&bars.pb_full[as], (j >> 1) & 1, abort_flag, a.err, kWaitLimitNs) &&
-                 mbar_wait(&bars.acc_empty[as], ((j >> 1) & 1) ^ 1, abort_flag, a.err,
-                           kWaitLimitNs);
-            if (!ok) break;
+            const int r = qn / G, h = qn % G, as = qn & 1;
+            issue_qs(tmem + TM_ACC + as * ACCW, qn % NQ, r % NSOP, true);
+            umma_commit(&bars.acc_full[as]);
+            umma_commit(&bars.q_empty[qn % NQ]);
+            if (h == G - 1) umma_commit(&bars.sop_empty[r % NSOP]);
+            ++qn;
+            did = true;
+          } else if (sc < n_items && sc <= pv + 1 && score_ready(sc)) {
             tc_fence_after();
+            score(sc);
+            ++sc;
+            did = true;
+          } else if (pv < sc && mbar_test(&bars.pb_full[pv & 1], (pv >> 1) & 1) &&
+                     mbar_test(&bars.acc_empty[pv & 1], ((pv >> 1) & 1) ^ 1)) {
+            tc_fence_after();
+            const int r = pv / G, h = pv % G, as = pv & 1;
             const uint32_t va = smem_u32(sV) + (r % NKV) * KVT;
             const uint64_t vd = smem_desc_sw128(va, ones - va, 1024);  // [V | 1]
             const uint32_t t_acc = tmem + TM_ACC + as * ACCW;
@@ -468,24 +464,21 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
               umma_f16_ts(t_acc, tmem + TM_P + as * kChunk + kk * 8, desc_advance(vd, kk * 2048),
                           ID_PV, kk > 0 ? 1u : 0u);
             if (h == G - 1) umma_commit(&bars.kv_empty[r % NKV]);
-            if (h == 0) {
-              ok = mbar_wait(&bars.sop_full[r % NSOP], (r / NSOP) & 1, abort_flag, a.err,
-                             kWaitLimitNs);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            issue_qs(t_acc, j % NQ, r % NSOP, true);
-            umma_commit(&bars.acc_full[as]);
-            umma_commit(&bars.q_empty[j % NQ]);
-            if (h == G - 1) umma_commit(&bars.sop_empty[r % NSOP]);
+            ++pv;
+            did = true;
           }
-          if (t < n_items && !scored) {
-            const int r = t / G;
-            ok = mbar_wait(&bars.q_xf[t % NQ], (t / NQ) & 1, abort_flag, a.err, kWaitLimitNs) &&
-                 mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs);
-            if (!ok) break;
-            tc_fence_after();
-            score(t);
+          if (did) {
+            idle = 0;
+          } else if ((++idle & 255u) == 0) {
+            if (*abort_flag) {
+              ok = false;
+            } else if (idle == 256) {
+              idle_t0 = global_timer_ns();
+            } else if (global_timer_ns() - idle_t0 > kWaitLimitNs) {
+              *abort_flag = 1;
+              report_error(a.err, kDevErrTimeout);
+              ok = false;
+            }
           }
         }
       } else {
@@ -769,10 +762,10 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
         for (int e = 0; e < 16; ++e) c[e] = 0.0f;
         if (have_carry && has_row) {
           if (q < DV / 16) {
-            const float4* r4 = reinterpret_cast<const float4*>(cS + row * DV + q * 16);
+            const float4* r4 = reinterpret_cast<const float4*>(cS) + row * (DV / 4);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              const float4 v = r4[u];
+              const float4 v = r4[(q * 4 + u) ^ (row & 15)];
               c[4 * u] = v.x;
               c[4 * u + 1] = v.y;
               c[4 * u + 2] = v.z;
