@@ -70,6 +70,7 @@ def source_digest():
     h = hashlib.sha256()
     for rel in ("causal_linear_attention_chunked_b200/csrc/state_bf16_sm100.cu",
                 "causal_linear_attention_chunked_b200/csrc/fwd_bf16_block_sm100.cu",
+                "causal_linear_attention_chunked_b200/csrc/fwd_bf16_fused_sm100.cu",
                 "causal_linear_attention_chunked_b200/csrc/fwd_bf16_sm100.cu",
                 "causal_linear_attention_chunked_b200/csrc/fwd_common.cuh",
                 "causal_linear_attention_chunked_b200/csrc/lt_ptx.cuh"):
