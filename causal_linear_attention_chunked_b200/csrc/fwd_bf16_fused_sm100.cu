@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
                                              ~uintptr_t(1023));
   using L = Layout<NQ, NSOP>;
   __shared__ volatile int s_abort;
+  __shared__ volatile int s_me_next;  // mask/epilogue warps: the step thread 0 chose
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int blk = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
   int t0, ntok;
@@ -698,11 +699,46 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
       }
       return true;
     };
-    // the mask of item j+1 goes before the epilogue of item j: the mask is on
-    // the path to the next MMAs, the epilogue only drains
-    for (int t = 0; t <= n_items && ok; ++t) {
-      if (causal && t < n_items) ok = mask_p(t);
-      if (ok && t > 0) ok = epilogue(t - 1);
+    // Masks and epilogues in whichever order their inputs arrive (a mask
+    // whose score tile is ready never waits behind an epilogue whose
+    // accumulator needs the carry).  Thread 0 polls and picks the step; the
+    // group barrier at the end of every step orders the next pick after
+    // everyone has read this one.  Masks go first when both are ready.
+    int mt = 0, et = 0;
+    while (et < n_items && ok) {
+      if (x == 0) {
+        int c = -1;
+        uint32_t spins = 0;
+        uint64_t w0 = 0;
+        while (c < 0) {
+          if (causal && mt < n_items && mbar_test(&bars.p_full[mt & 1], (mt >> 1) & 1)) {
+            c = 0;
+          } else if (et < (causal ? mt : n_items) &&
+                     mbar_test(&bars.acc_full[et & 1], (et >> 1) & 1)) {
+            c = 1;
+          } else if ((++spins & 255u) == 0) {
+            if (*abort_flag) {
+              c = 2;
+            } else if (spins == 256) {
+              w0 = global_timer_ns();
+            } else if (global_timer_ns() - w0 > kWaitLimitNs) {
+              *abort_flag = 1;
+              report_error(a.err, kDevErrTimeout);
+              c = 2;
+            }
+          }
+        }
+        s_me_next = c;
+      }
+      named_bar_sync(2, 128);
+      const int c = s_me_next;
+      if (c == 2) {
+        ok = false;
+      } else if (c == 0) {
+        ok = mask_p(mt++);
+      } else {
+        ok = epilogue(et++);
+      }
     }
   } else if (warp < 16) {
     // -------------------------------------------------- state warpgroup
@@ -884,9 +920,9 @@ cudaError_t launch_fwd_bf16_block_fused(const FwdLaunch& p, int nb, float* ws,
   a.total_tokens = (int)p.total_tokens;
   a.err = p.err;
   a.fused = 1;
-  // three Q stages, two operand buffers
-  using L = Layout<3, 2>;
-  auto fk = lt_fused_fwd_kernel<3, 2, true>;
+  // four Q stages (every Q tile of a block is loaded at once), one operand buffer
+  using L = Layout<4, 1>;
+  auto fk = lt_fused_fwd_kernel<4, 1, true>;
   cudaError_t e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
