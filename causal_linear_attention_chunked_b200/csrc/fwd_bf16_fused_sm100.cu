@@ -69,10 +69,6 @@ struct FusedArgs {
   float eps;
   int total_tokens;
   int* err;
-  // fused: one cooperative launch in which every block first publishes its
-  // own aggregate to ws, all CTAs meet at a grid barrier, and each block
-  // then gathers its carry itself
-  int fused;
 };
 
 __device__ __forceinline__ bool seq_bounds(const FusedArgs& a, int s, int& t0, int& n) {
@@ -91,9 +87,7 @@ __device__ __forceinline__ bool seq_bounds(const FusedArgs& a, int s, int& t0, i
 // ========================================================================
 // Forward pass over one block per CTA.
 // ========================================================================
-// warps 0-17, plus warp 18 (the state-product issuer) in the one-launch mode;
-// without it the register budget per thread is larger
-constexpr int kThreadsFor(bool fused) { return fused ? 608 : 576; }
+constexpr int kThreads = 608;
 constexpr int kXf = 256;  // transform threads (warps 0-7, two per SM sub-partition)
 constexpr int NKV = 4;
 // two score tiles (item j uses j & 1), two accumulators, the running state
@@ -120,7 +114,7 @@ struct Bars {
   uint64_t *q_full, *q_empty, *q_xf, *kv_full, *kv_empty, *kv_xf;
   uint64_t *p_full, *pb_full, *sop_full, *sop_empty;
   uint64_t *s_full, *s_empty, *acc_full, *acc_empty, *drain;
-  uint64_t* agg_full;  // fused mode: the block aggregate is in S_acc
+  uint64_t* agg_full;  // phase A: the block aggregate is in S_acc
   uint64_t* drain2;    // the state issuer's products are complete
 };
 
@@ -196,15 +190,12 @@ __device__ __forceinline__ void sum_aggregates(const float4* base, int nsum, flo
   if (has_z) reinterpret_cast<float4*>(stage_z)[u] = acc[PER];
 }
 
-// kFused: the one-launch mode (see BlockArgs::fused).  It also splits the
-// issue: the state products get their own issuer (warp 18) and the score of
-// an item goes ahead of the previous item's products only when its tiles are
-// ready; otherwise one issuer works in a fixed order (score t, the state
-// product of its chunk, then item t-1's P V and phi(Q)[S|z]).  A compile-time
-// flag keeps each instantiation's code to its own mode (the instruction
-// working set of the warp roles matters).
-template <int NQ, int NSOP, bool kFused>
-__global__ void __launch_bounds__(kThreadsFor(kFused), 1)
+// NQ Q stages and NSOP state operand buffers (shared-memory layout).  The
+// main issuer (warp 17) polls, so that a product whose inputs are ready never
+// waits behind one whose inputs are late; the state products have their own
+// issuer (warp 18).
+template <int NQ, int NSOP>
+__global__ void __launch_bounds__(kThreads, 1)
     lt_fused_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const FusedArgs a) {
@@ -223,21 +214,17 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
   }
   const int nc = (ntok + kChunk - 1) / kChunk;
   const int c0 = blk * a.bc, c1 = min(c0 + a.bc, nc);
-  if (c1 <= c0) return;  // nothing in this block (uniform over the CTA; never in fused mode)
+  if (c1 <= c0) return;  // never: the host plans no empty block (every CTA must arrive at the grid barrier)
   const int Ri = c1 - c0;  // chunks of this block, walked in order
   const int G = a.G;
   const bool causal = a.causal != 0;
   const int n_items = Ri * G;
   // non-causal with a workspace: the state is the sum of all blocks and this
   // CTA reads only Q
-  constexpr bool fused = kFused, kSplit = kFused;
-  const bool nc_from_ws = !causal && a.ws != nullptr && !fused;
-  // fused mode: this CTA first reduces its block's K, V to the aggregate
-  // (phase A) and publishes it, then gathers the carry from the aggregates
-  // the other CTAs of the launch publish; the K/V ring holds every chunk of
-  // the block, so each tile is loaded once
-  // non-causal and the whole state comes from the carry
-  const bool nc_carry = !causal && (nc_from_ws || fused);
+  // this CTA first reduces its block's K, V to the aggregate (phase A) and
+  // publishes it, then gathers the carry from the aggregates the other CTAs
+  // publish; the K/V ring holds every chunk of the block, so each tile is
+  // loaded once.  Non-causal: the whole state is the carry.
 
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* sK = smem + L::OFF_KV;
@@ -255,8 +242,8 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
     }
     for (int i = 0; i < NKV; ++i) {
       mbar_init(&bars.kv_full[i], 1);
-      // split causal: released by the main issuer (scores, P V) and the state issuer
-      mbar_init(&bars.kv_empty[i], (kSplit && causal) ? 2 : 1);
+      // causal: released by the main issuer (scores, P V) and the state issuer
+      mbar_init(&bars.kv_empty[i], causal ? 2 : 1);
       mbar_init(&bars.kv_xf[i], 1);
     }
     for (int i = 0; i < NSOP; ++i) {
@@ -276,7 +263,7 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
     mbar_init(bars.drain2, 1);
     fence_mbar_init();
   }
-  init_ones_block(smem + L::OFF_ONES, tid, kThreadsFor(kFused));
+  init_ones_block(smem + L::OFF_ONES, tid, kThreads);
   fence_proxy_async_smem();
   if (warp == 17) tmem_alloc(tmem_slot, TM_COLS);
   tc_fence_before();
@@ -299,16 +286,11 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
                       : reinterpret_cast<const float4*>(a.ws) + (size_t)(s * a.Hkv + g) * a.nb * (E / 4);
   float* carry_stage = reinterpret_cast<float*>(smem + L::OFF_SOP);
   float* carry_stage_z = reinterpret_cast<float*>(smem + L::OFF_Z);
-  if (!fused && nprev > 0 && warp < 16) {
-    // two-launch mode: the aggregates are complete; warps 0-15 sum them
-    sum_aggregates<512>(agg_base, nprev, carry_stage, carry_stage_z, tid);
-    named_bar_sync(4, 512);
-  }
-  // fused mode: the transform warps and the state warps (384 threads) sum the
-  // aggregates between two barriers 5, once the state warps have seen every
-  // needed flag.  Both groups pass both barriers on every path (an abort
-  // skips only the loads), so no barrier is left waiting.
-  const bool gather = fused && nprev > 0;
+  // The transform warps and the state warps (384 threads) sum the aggregates
+  // between two barriers 5, once the state warps have passed the grid
+  // barrier.  Both groups pass both barriers on every path (an abort skips
+  // only the loads), so no barrier is left waiting.
+  const bool gather = nprev > 0;
   auto gather_part = [&](int u) {
     named_bar_sync(5, 384);
     if (!*abort_flag) sum_aggregates<384>(agg_base, nprev, carry_stage, carry_stage_z, u);
@@ -342,16 +324,9 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
         ++q_issued;
         return true;
       };
-      if (causal && !fused) {
-        for (int r = 0; r < Ri && ok; ++r) {
-          ok = load_kv(r);
-          for (int h = 0; h < G && ok; ++h) ok = load_q(r * G + h);
-        }
-      } else {  // every K/V tile first (non-causal, or phase A of fused mode)
-        if (!nc_from_ws)
-          for (int r = 0; r < Ri && ok; ++r) ok = load_kv(r);
-        for (int j = 0; j < n_items && ok; ++j) ok = load_q(j);
-      }
+      // every K/V tile first (phase A needs them), then the Q tiles
+      for (int r = 0; r < Ri && ok; ++r) ok = load_kv(r);
+      for (int j = 0; j < n_items && ok; ++j) ok = load_q(j);
       if (!ok) {  // drain copies in flight (bounded, ignoring the abort flag)
         int dummy = 0;
         for (int r = (kv_issued > NKV ? kv_issued - NKV : 0); r < kv_issued; ++r)
@@ -483,16 +458,7 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
           }
         }
       } else {
-        if (!nc_carry) {
-          for (int r = 0; r < Ri && ok; ++r) {
-            ok = mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs);
-            if (!ok) break;
-            tc_fence_after();
-            issue_ds(r, tmem + TM_S, r > 0);
-            umma_commit(&bars.kv_empty[r % NKV]);
-          }
-          if (ok) umma_commit(bars.s_full);
-        }
+        // non-causal: the whole state is the carry, staged once
         if (ok) ok = mbar_wait(&bars.sop_full[0], 0, abort_flag, a.err, kWaitLimitNs);
         for (int j = 0; j < n_items && ok; ++j) {
           const int qs = j % NQ, as = j & 1;
@@ -517,7 +483,7 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
     // aggregate).  Causal: S_acc += phi(K_r)^T [V_r | 1] for each chunk but
     // the last, once the state warps have read S_<r (phase r of s_empty),
     // then this issuer's share of the K/V stage release.
-    if (lane == 0 && (fused || (kSplit && causal))) {
+    if (lane == 0) {
       constexpr uint32_t ID_SV = idesc_bf16_f32(D, DV + 16, 1, 1);
       const uint64_t dKmn = smem_desc_sw128(smem_u32(sK), kBox, 1024);  // MN-major phi(K)
       const uint32_t ones = smem_u32(smem + L::OFF_ONES);
@@ -532,16 +498,14 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
                       (accumulate || kk > 0) ? 1u : 0u);
       };
       bool ok = true;
-      if (fused) {
-        for (int r = 0; r < Ri && ok; ++r) {
-          ok = mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs);
-          if (!ok) break;
-          tc_fence_after();
-          issue_ds(r, r > 0);
-        }
-        if (ok) umma_commit(bars.agg_full);
+      for (int r = 0; r < Ri && ok; ++r) {
+        ok = mbar_wait(&bars.kv_xf[r % NKV], (r / NKV) & 1, abort_flag, a.err, kWaitLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+        issue_ds(r, r > 0);
       }
-      if (kSplit && causal) {
+      if (ok) umma_commit(bars.agg_full);
+      if (causal) {
         for (int r = 0; r < Ri && ok; ++r) {
           if (r + 1 < Ri) {
             ok = mbar_wait(bars.s_empty, r & 1, abort_flag, a.err, kWaitLimitNs) &&
@@ -565,28 +529,17 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
     // ---------------------------------------------- transform warps
     const int x = tid;  // 0..255
     bool ok = true;
-    // One loop over the tiles in arrival order (causal: K_r then the Q of
-    // each head of chunk r; non-causal: every K, then every Q), so that the
-    // transform code exists once in the kernel image.
-    const int nkv = nc_from_ws ? 0 : Ri;
-    const int T = (causal && !fused) ? Ri * (G + 1) : nkv + n_items;
-    // fused mode: the Q tiles past the ring wait for a product that needs the
-    // carry, so the gather comes after the first NQ of them
+    // One loop over the tiles in arrival order (every K, then every Q), so
+    // that the transform code exists once in the kernel image.  The gather
+    // comes after the first NQ Q tiles (those loaded without waiting on a
+    // product, some of which need the carry).
+    const int nkv = Ri;
+    const int T = nkv + n_items;
     const int join_t = nkv + min(n_items, NQ) - 1;
     bool joined = !gather;
     for (int t = 0; t < T && ok; ++t) {
-      bool is_kv;
-      int r, j;
-      if (causal && !fused) {
-        r = t / (G + 1);
-        const int k = t - r * (G + 1);
-        is_kv = k == 0;
-        j = r * G + k - 1;
-      } else {
-        is_kv = t < nkv;
-        r = t;
-        j = t - nkv;
-      }
+      const bool is_kv = t < nkv;
+      const int r = t, j = t - nkv;
       const int st = is_kv ? r % NKV : j % NQ;
       const uint32_t par = is_kv ? (r / NKV) & 1 : (j / NQ) & 1;
       ok = mbar_wait(is_kv ? &bars.kv_full[st] : &bars.q_full[st], par, abort_flag, a.err,
@@ -841,14 +794,12 @@ __global__ void __launch_bounds__(kThreadsFor(kFused), 1)
     // waits only for the last product that read chunk r - NSOP's operand.
     // Step 0 reads the carry from the operand buffers themselves: barrier 3
     // below orders every thread's read before the first operand write.
-    if (fused) {
-      // causal block 0 has no carry but publishes its aggregate
-      publish_and_gather(gather);
-      ok = !*abort_flag;
-    }
+    // causal block 0 has no carry but publishes its aggregate
+    publish_and_gather(gather);
+    ok = !*abort_flag;
     const int nsteps = causal ? Ri : 1;
     for (int r = 0; r < nsteps && ok; ++r) {
-      if (r == 0 && (causal || nc_carry)) {
+      if (r == 0) {
         load_carry();
       } else {
         ok = mbar_wait(bars.s_full, (causal ? r - 1 : 0) & 1, abort_flag, a.err, kWaitLimitNs);
@@ -919,15 +870,14 @@ cudaError_t launch_fwd_bf16_block_fused(const FwdLaunch& p, int nb, float* ws,
   a.eps = p.eps;
   a.total_tokens = (int)p.total_tokens;
   a.err = p.err;
-  a.fused = 1;
   // four Q stages (every Q tile of a block is loaded at once), one operand buffer
   using L = Layout<4, 1>;
-  auto fk = lt_fused_fwd_kernel<4, 1, true>;
+  auto fk = lt_fused_fwd_kernel<4, 1>;
   cudaError_t e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nb, p.Hkv, p.B);
-  cfg.blockDim = dim3(kThreadsFor(true), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = L::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute at[1];
