@@ -531,11 +531,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     // One loop over the tiles in arrival order (every K, then every Q), so
     // that the transform code exists once in the kernel image.  The gather
-    // comes after the first NQ Q tiles (those loaded without waiting on a
-    // product, some of which need the carry).
+    // comes before the last Q tile that is loaded without waiting on a
+    // product: by then the grid barrier has usually passed, and that tile's
+    // item waits for an accumulator that needs the carry anyway.
     const int nkv = Ri;
     const int T = nkv + n_items;
-    const int join_t = nkv + min(n_items, NQ) - 1;
+    const int join_t = nkv + max(0, min(n_items, NQ) - 2);
     bool joined = !gather;
     for (int t = 0; t < T && ok; ++t) {
       const bool is_kv = t < nkv;
@@ -736,7 +737,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      __threadfence();
+      // the group barrier orders every thread's aggregate writes before the
+      // arriving thread's release at gpu scope (release is cumulative)
       named_bar_sync(3, 128);
       if (y == 0) grid_barrier(do_gather, abort_flag, a.err, kWaitLimitNs);
       if (do_gather) gather_part(256 + y);

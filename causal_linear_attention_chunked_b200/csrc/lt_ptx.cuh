@@ -458,7 +458,7 @@ __device__ __forceinline__ bool grid_barrier(bool wait, volatile int* abort, int
       report_error(err, kDevErrTimeout);
       return false;
     }
-    __nanosleep(32);
+    __nanosleep(128);  // one poller per CTA on one word: keep its line cool
   }
 }
 
