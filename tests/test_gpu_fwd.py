@@ -295,6 +295,25 @@ def test_fused_launch_in_cuda_graph_replays_with_new_inputs(monkeypatch):
         assert row_rel_err(got, ref) <= TOL_BF16
 
 
+def test_fused_launch_many_back_to_back(monkeypatch):
+    """Forty one-launch calls in a row on one stream, alternating two input
+    sets without synchronising: each meets the grid barrier of its own
+    launch, so every output equals the first output of its input set."""
+    import causal_linear_attention_chunked_b200 as L
+    monkeypatch.delenv("LT_BLOCKS", raising=False)
+    monkeypatch.delenv("LT_KERNEL", raising=False)
+    B, Hq, Hkv, N = 2, 8, 8, 4096
+    assert L.linear_attn_fwd_plan(B, Hq, Hkv, N, 64, 64, causal=True)[1] == 1
+    sets = [tuple(t.cuda() for t in inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16,
+                                                      0.125, seed=sd)) for sd in (31, 32)]
+    outs = [L.linear_attn_fwd(*sets[i % 2], causal=True) for i in range(40)]
+    torch.cuda.synchronize()
+    assert L.get_last_device_error() == 0
+    for i, o in enumerate(outs):
+        assert torch.equal(o, outs[i % 2]), i
+    assert not torch.equal(outs[0], outs[1])
+
+
 def test_block_kernel_deterministic_across_block_counts(monkeypatch):
     """Every block count computes the same function; results agree to a few
     bf16 ulps (only the summation order of the carried state differs)."""
