@@ -517,58 +517,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto stage_state = [&](int buf, int use, int src, int s_parity) -> bool {
       const bool has_row = (D == 128) || (lane < 16);
       const int row = (D == 128) ? x : (sp * 16 + lane);
-      float r[DV + 16];
+      // this thread's row of [S | z 0 ..], rounded to packed bf16 16 columns
+      // at a time (the fp32 row never lives in registers whole)
+      uint32_t w[(DV + 16) / 2];
+      const uint32_t t_s = tmem + K::TM_S + lane_base;
       if (src == kFromTmem) {
         if (!mbar_wait(bars.s_full, s_parity, abort_flag, a.err, kWaitLimitNs)) return false;
         tc_fence_after();
-        const uint32_t t_s = tmem + K::TM_S + lane_base;
 #pragma unroll
-        for (int cb = 0; cb < DV / 32; ++cb) {
-          float t32[32];
-          tmem_ld32(t_s + cb * 32, t32);
+        for (int cb = 0; cb < (DV + 16) / 16; ++cb) {
+          float t16[16];
+          tmem_ld16(t_s + cb * 16, t16);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[cb * 32 + e] = t32[e];
+          for (int e = 0; e < 8; ++e) w[cb * 8 + e] = pack_bf16x2(t16[2 * e], t16[2 * e + 1]);
         }
-        float t16[16];
-        tmem_ld16(t_s + DV, t16);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r[DV + e] = t16[e];
         tc_fence_before();
       } else {
+        constexpr int E = D * DV + D;
+        const float* base = a.ws != nullptr ? a.ws + (size_t)(s * a.Hkv + g) * a.nb * E : nullptr;
+        const int nsum = src == kFromCarry ? (a.causal ? blk : a.nb) : 0;
 #pragma unroll
-        for (int e = 0; e < DV + 16; ++e) r[e] = 0.0f;
-        if (src == kFromCarry) {
+        for (int cb = 0; cb < (DV + 16) / 16; ++cb) {
+          float c16[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) c16[e] = 0.0f;
           if (has_row) {
-            constexpr int E = D * DV + D;
-            const float* base = a.ws + (size_t)(s * a.Hkv + g) * a.nb * E;
-            const int nsum = a.causal ? blk : a.nb;
             for (int bb = 0; bb < nsum; ++bb) {
-              const float4* r4 = reinterpret_cast<const float4*>(base + (size_t)bb * E + row * DV);
+              if (cb < DV / 16) {
+                const float4* r4 =
+                    reinterpret_cast<const float4*>(base + (size_t)bb * E + row * DV + cb * 16);
 #pragma unroll
-              for (int q4 = 0; q4 < DV / 4; ++q4) {
-                const float4 v4 = r4[q4];
-                r[4 * q4] += v4.x;
-                r[4 * q4 + 1] += v4.y;
-                r[4 * q4 + 2] += v4.z;
-                r[4 * q4 + 3] += v4.w;
+                for (int u = 0; u < 4; ++u) {
+                  const float4 v4 = r4[u];
+                  c16[4 * u] += v4.x;
+                  c16[4 * u + 1] += v4.y;
+                  c16[4 * u + 2] += v4.z;
+                  c16[4 * u + 3] += v4.w;
+                }
+              } else {
+                c16[0] += base[(size_t)bb * E + D * DV + row];
               }
-              r[DV] += base[(size_t)bb * E + D * DV + row];
             }
           }
-          if (a.causal) {
-            const uint32_t t_s = tmem + K::TM_S + lane_base;
+          if (src == kFromCarry && a.causal) {
+            uint32_t u16[16];
 #pragma unroll
-            for (int cb = 0; cb < (DV + 16) / 16; ++cb) {
-              uint32_t w16[16];
-#pragma unroll
-              for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(r[cb * 16 + e]);
-              tmem_st16(t_s + cb * 16, w16);
-            }
-            tmem_wait_st();
-            tc_fence_before();
+            for (int e = 0; e < 16; ++e) u16[e] = __float_as_uint(c16[e]);
+            tmem_st16(t_s + cb * 16, u16);
           }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[cb * 8 + e] = pack_bf16x2(c16[2 * e], c16[2 * e + 1]);
+        }
+        if (src == kFromCarry && a.causal) {
+          tmem_wait_st();
+          tc_fence_before();
         }
       }
       named_bar_sync(2, 128);
@@ -580,11 +583,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q8 = 0; q8 < (DV + 16) / 8; ++q8) {
           const int grp = q8 >> 3, jj = q8 & 7;
-          const uint4 w = make_uint4(pack_bf16x2(r[q8 * 8 + 0], r[q8 * 8 + 1]),
-                                     pack_bf16x2(r[q8 * 8 + 2], r[q8 * 8 + 3]),
-                                     pack_bf16x2(r[q8 * 8 + 4], r[q8 * 8 + 5]),
-                                     pack_bf16x2(r[q8 * 8 + 6], r[q8 * 8 + 7]));
-          *reinterpret_cast<uint4*>(sop + grp * (D * kRowBytes) + sw128_off(row, jj)) = w;
+          *reinterpret_cast<uint4*>(sop + grp * (D * kRowBytes) + sw128_off(row, jj)) =
+              make_uint4(w[4 * q8], w[4 * q8 + 1], w[4 * q8 + 2], w[4 * q8 + 3]);
         }
       }
       fence_proxy_async_smem();
