@@ -21,14 +21,17 @@
 // served from the same K/V tiles and the same state.  With more than one
 // block per sequence the state of a block starts from the carry summed from
 // the block aggregates of the state launch (earlier blocks when causal,
-// every block when not), written into the TMEM state accumulator.  Warp roles (320 threads):
-//   warps 0-3  transform warpgroup: phi applied in place to the TMA-loaded
-//              K and Q tiles, tail rows zeroed; causal mask of the score
-//              tile, conversion to bf16, staging as the A operand of P V.
-//   warps 4-7  state/epilogue warpgroup: TMEM state -> bf16 operand;
-//              TMEM accumulator -> normalised bf16 rows -> global memory.
-//   warp 8     TMA producer.
-//   warp 9     TMEM allocator and single-thread MMA issuer.
+// every block when not), written into the TMEM state accumulator.  Warp roles (448 threads):
+//   warps 0-3   phi warpgroup: phi applied in place to the TMA-loaded K and
+//               Q tiles, tail rows zeroed.
+//   warps 4-7   mask warpgroup: causal mask of the score tile, conversion
+//               to bf16, staging as the A operand of P V.
+//   warps 8-11  state/epilogue warpgroup: TMEM state -> bf16 operand;
+//               TMEM accumulator -> normalised bf16 rows, transposed through
+//               a small shared-memory tile per warp so that every store
+//               instruction writes whole 64-byte row segments.
+//   warp 12     TMA producer.
+//   warp 13     TMEM allocator and single-thread MMA issuer.
 // Non-causal mode (phi(Q)(phi(K)^T V) normalised the same way): first the
 // state over all chunks (K, V only; taken from the block aggregates when the
 // sequence is split into blocks), then every output row as phi(Q_i) [S|z]_n
@@ -46,7 +49,7 @@
 namespace lt {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 using namespace fwd;
 
 template <int D, int DV>
@@ -56,8 +59,8 @@ struct Cfg {
   static constexpr int VT = kChunk * DV * 2;
   static constexpr int PBT = kChunk * kChunk * 2;
   static constexpr int SOPT = (DV / 64 + 1) * D * kRowBytes;  // [S | z 0..] operand
-  static constexpr int ONEST = kChunk * kRowBytes;
-  static constexpr bool kBig = (D == 128);
+  static constexpr int ONEST = 16 * kRowBytes;  // K-major [1 | 0..] block, N = 16 rows
+  static constexpr int OSTT = 4 * 32 * 64;  // epilogue staging: 32 rows x 64 B per warp
   static constexpr int NQ = (D == 64 && DV == 64) ? 3 : 2;
   static constexpr int NKV = (D == 128) ? 1 : 2;
   static constexpr int NPB = (DV == 128) ? 1 : 2;
@@ -77,7 +80,8 @@ struct Cfg {
   static constexpr int OFF_PB = OFF_V + NKV * VT;
   static constexpr int OFF_SOP = OFF_PB + NPB * PBT;
   static constexpr int OFF_ONES = OFF_SOP + NSOP * SOPT;
-  static constexpr int OFF_BAR = OFF_ONES + ONEST;
+  static constexpr int OFF_OST = OFF_ONES + 1024 * ((ONEST + 1023) / 1024);
+  static constexpr int OFF_BAR = OFF_OST + OSTT;
   static constexpr int NBARS = 4 * NQ + 3 * NKV + 2 * NP + 2 * NPB + 2 * NSOP + 2 + 2 * NA + 1;
   static constexpr int SMEM = OFF_BAR + NBARS * 8 + 16 + 1024;  // + tmem slot + align slack
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -176,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sPB = smem + K::OFF_PB;
   uint8_t* sSOP = smem + K::OFF_SOP;
   uint8_t* sONES = smem + K::OFF_ONES;
+  uint8_t* sOST = smem + K::OFF_OST;
   Bars bars = carve_bars<D, DV>(smem + K::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + K::OFF_BAR + K::NBARS * 8);
 
@@ -213,16 +218,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bars.drain, 1);
     fence_mbar_init();
   }
-  init_ones_block(sONES, tid, kThreads);
+  // [1 | 0 ..] as a K-major B operand: row n = 0 all ones, rows 1..15 zero
+  // (uniform rows, so the swizzle leaves them unchanged); every 16-key step
+  // of a 64-key atom and both atoms of a chunk read the same 2 KB
+  for (int ch = tid; ch < K::ONEST / 16; ch += kThreads)
+    reinterpret_cast<uint4*>(sONES)[ch] =
+        ch < 8 ? make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u)
+               : make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_smem();
-  if (warp == 9) tmem_alloc(tmem_slot, K::TM_COLS);
+  if (warp == 13) tmem_alloc(tmem_slot, K::TM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int* abort_flag = &s_abort;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -275,14 +286,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&bars.q_full[i % K::NQ], (i / K::NQ) & 1, &dummy, nullptr, kWaitLimitNs);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t ID_P = idesc_bf16_f32(kChunk, kChunk, 0, 0);
       constexpr uint32_t ID_SV = idesc_bf16_f32(D, DV, 1, 1);
-      constexpr uint32_t ID_S1 = idesc_bf16_f32(D, 16, 1, 1);
+      constexpr uint32_t ID_S1 = idesc_bf16_f32(D, 16, 1, 0);
       constexpr uint32_t ID_PV = idesc_bf16_f32(kChunk, DV, 0, 1);
-      constexpr uint32_t ID_P1 = idesc_bf16_f32(kChunk, 16, 0, 1);
+      constexpr uint32_t ID_P1 = idesc_bf16_f32(kChunk, 16, 0, 0);
       constexpr uint32_t ID_QS = idesc_bf16_f32(kChunk, DV + 16, 0, 1);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       const uint32_t sPBa = smem_u32(sPB), sSOPa = smem_u32(sSOP), sONESa = smem_u32(sONES);
@@ -297,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t ad = smem_desc_sw128(kb + kk * 2048, kBox, 1024);
           umma_f16_ss(t_s, ad, smem_desc_sw128(vb + kk * 2048, kBox, 1024), ID_SV,
                       (accumulate || kk > 0) ? 1u : 0u);
-          umma_f16_ss(t_s + DV, ad, smem_desc_sw128(sONESa + kk * 2048, kBox, 1024), ID_S1,
+          umma_f16_ss(t_s + DV, ad, smem_desc_sw128(sONESa + (kk & 3) * 32, 16, 1024), ID_S1,
                       (accumulate || kk > 0) ? 1u : 0u);
         }
       };
@@ -330,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t ad = smem_desc_sw128(pb + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024);
             umma_f16_ss(t_acc, ad, smem_desc_sw128(vb + kk * 2048, kBox, 1024), ID_PV,
                         kk > 0 ? 1u : 0u);
-            umma_f16_ss(t_acc + DV, ad, smem_desc_sw128(sONESa + kk * 2048, kBox, 1024), ID_P1,
+            umma_f16_ss(t_acc + DV, ad, smem_desc_sw128(sONESa + (kk & 3) * 32, 16, 1024), ID_P1,
                         kk > 0 ? 1u : 0u);
           }
           issue_qs(t_acc, sQa + qs * K::QT, sSOPa + (c % K::NSOP) * K::SOPT, true);
@@ -411,31 +422,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(bars.drain, 0, &dummy, nullptr, kWaitLimitNs);
     }
   } else if (warp < 4) {
-    // ----------------------------------------------- transform warpgroup
-    const int x = tid;  // 0..127 == TMEM lane == chunk row
+    // ------------------------------------------------------ phi warpgroup
+    const int x = tid;  // 0..127
     bool ok = true;
     auto xf_kv = [&](int c) -> bool {
       const int st = c % K::NKV;
       if (!mbar_wait(&bars.kv_full[st], (c / K::NKV) & 1, abort_flag, a.err, kWaitLimitNs))
         return false;
       const int valid = min(kChunk, n - c * kChunk);
-      xf_tile<D / 64>(sK + st * K::KT, valid, true, x);
-      if (valid < kChunk) xf_tile<DV / 64>(sV + st * K::VT, valid, false, x);
+      prep_tile<D / 64, 128>(sK + st * K::KT, valid, true, x);
+      prep_tile<DV / 64, 128>(sV + st * K::VT, valid, false, x);
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
       if (x == 0) mbar_arrive(&bars.kv_xf[st]);
       return true;
     };
+    // rows past the end of the sequence only reach their own (unstored) outputs
     auto xf_q = [&](int i) -> bool {
       const int st = i % K::NQ;
       if (!mbar_wait(&bars.q_full[st], (i / K::NQ) & 1, abort_flag, a.err, kWaitLimitNs))
         return false;
-      xf_tile<D / 64>(sQ + st * K::QT, kChunk, true, x);
+      phi_tile_full<D / 64, 128>(sQ + st * K::QT, x);
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
       if (x == 0) mbar_arrive(&bars.q_xf[st]);
       return true;
     };
+    if (a.causal) {
+      for (int i = 0; i < n_items && ok; ++i) {
+        if (i % G == 0) ok = xf_kv(i / G);
+        if (ok) ok = xf_q(i);
+      }
+    } else {
+      if (!carried_state)
+        for (int c = 0; c < nc && ok; ++c) ok = xf_kv(c);
+      for (int i = 0; i < n_items && ok; ++i) ok = xf_q(i);
+    }
+  } else if (warp < 8) {
+    // ----------------------------------------------------- mask warpgroup
+    const int x = tid - 128;  // 0..127 == TMEM lane == chunk row
+    const int sp = warp & 3;  // TMEM sub-partition of this warp
+    bool ok = true;
     // mask + convert the score tile of item j into the bf16 A operand
     auto mask_p = [&](int j) -> bool {
       const int ps = j % K::NP, pbs = j % K::NPB;
@@ -445,13 +472,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                      kWaitLimitNs))
         return false;
       tc_fence_after();
-      const uint32_t t_p = tmem + K::TM_P + ps * kChunk + ((uint32_t)(warp * 32) << 16);
+      const uint32_t t_p = tmem + K::TM_P + ps * kChunk + ((uint32_t)(sp * 32) << 16);
       uint8_t* pb = sPB + pbs * K::PBT;
       const int row = x;
 #pragma unroll 1
       for (int b = 0; b < kChunk / 32; ++b) {
         uint4 w[4];
-        if (b <= warp) {  // warp-uniform: blocks right of the diagonal are all zero
+        if (b <= sp) {  // warp-uniform: blocks right of the diagonal are all zero
           float r[32];
           tmem_ld32(t_p + b * 32, r);
           tmem_wait_ld();
@@ -477,32 +504,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
+      named_bar_sync(3, 128);
       if (x == 0) {
         mbar_arrive(&bars.p_empty[ps]);
         mbar_arrive(&bars.pb_full[pbs]);
       }
       return true;
     };
-    if (a.causal) {
-      for (int i = 0; i < n_items && ok; ++i) {
-        // With a single K/V stage the next chunk's tiles arrive only after
-        // the previous chunk's last score tile has been consumed.
-        const bool flush_first = (K::NKV == 1) && (i % G == 0) && i > 0;
-        if (flush_first) ok = mask_p(i - 1);
-        if (ok && i % G == 0) ok = xf_kv(i / G);
-        if (ok) ok = xf_q(i);
-        if (ok && i > 0 && !flush_first) ok = mask_p(i - 1);
-      }
-      if (ok && n_items > 0) ok = mask_p(n_items - 1);
-    } else {
-      if (!carried_state)
-        for (int c = 0; c < nc && ok; ++c) ok = xf_kv(c);
-      for (int i = 0; i < n_items && ok; ++i) ok = xf_q(i);
-    }
+    if (a.causal)
+      for (int j = 0; j < n_items && ok; ++j) ok = mask_p(j);
   } else {
     // ----------------------------------------- state / epilogue warpgroup
-    const int x = tid - 128;          // 0..127
+    const int x = tid - 256;          // 0..127
     const int sp = warp & 3;          // TMEM sub-partition of this warp
     const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     bool ok = true;
@@ -517,29 +530,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto stage_state = [&](int buf, int use, int src, int s_parity) -> bool {
       const bool has_row = (D == 128) || (lane < 16);
       const int row = (D == 128) ? x : (sp * 16 + lane);
-      // this thread's row of [S | z 0 ..], rounded to packed bf16 16 columns
-      // at a time (the fp32 row never lives in registers whole)
-      uint32_t w[(DV + 16) / 2];
-      const uint32_t t_s = tmem + K::TM_S + lane_base;
+      // With one operand buffer (D = 128) the buffer frees only after the
+      // chunk's last accumulator MMA, which also frees the single K/V stage
+      // that the next state MMA needs: waiting for it first costs nothing,
+      // and the row goes to shared memory 16 columns at a time.  With two,
+      // the row is read (and the state released) before the buffer frees.
+      constexpr bool kStream = K::NSOP == 1;
+      uint8_t* sop = sSOP + buf * K::SOPT;
+      if (kStream && !mbar_wait(&bars.sop_empty[buf], (use & 1) ^ 1, abort_flag, a.err,
+                                kWaitLimitNs))
+        return false;
       if (src == kFromTmem) {
         if (!mbar_wait(bars.s_full, s_parity, abort_flag, a.err, kWaitLimitNs)) return false;
         tc_fence_after();
+      }
+      // this thread's row of [S | z 0 ..], rounded to packed bf16
+      uint32_t w[kStream ? 8 : (DV + 16) / 2];
+      const uint32_t t_s = tmem + K::TM_S + lane_base;
+      constexpr int E = D * DV + D;
+      const float* base = a.ws != nullptr ? a.ws + (size_t)(s * a.Hkv + g) * a.nb * E : nullptr;
+      const int nsum = src == kFromCarry ? (a.causal ? blk : a.nb) : 0;
 #pragma unroll
-        for (int cb = 0; cb < (DV + 16) / 16; ++cb) {
-          float t16[16];
-          tmem_ld16(t_s + cb * 16, t16);
+      for (int cb = 0; cb < (DV + 16) / 16; ++cb) {
+        float c16[16];
+        if (src == kFromTmem) {
+          tmem_ld16(t_s + cb * 16, c16);
           tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 8; ++e) w[cb * 8 + e] = pack_bf16x2(t16[2 * e], t16[2 * e + 1]);
-        }
-        tc_fence_before();
-      } else {
-        constexpr int E = D * DV + D;
-        const float* base = a.ws != nullptr ? a.ws + (size_t)(s * a.Hkv + g) * a.nb * E : nullptr;
-        const int nsum = src == kFromCarry ? (a.causal ? blk : a.nb) : 0;
-#pragma unroll
-        for (int cb = 0; cb < (DV + 16) / 16; ++cb) {
-          float c16[16];
+        } else {
 #pragma unroll
           for (int e = 0; e < 16; ++e) c16[e] = 0.0f;
           if (has_row) {
@@ -566,32 +583,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 16; ++e) u16[e] = __float_as_uint(c16[e]);
             tmem_st16(t_s + cb * 16, u16);
           }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) w[cb * 8 + e] = pack_bf16x2(c16[2 * e], c16[2 * e + 1]);
         }
-        if (src == kFromCarry && a.causal) {
-          tmem_wait_st();
-          tc_fence_before();
+        uint32_t* wp = w + (kStream ? 0 : cb * 8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) wp[e] = pack_bf16x2(c16[2 * e], c16[2 * e + 1]);
+        if (kStream && has_row) {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int q8 = cb * 2 + h2, grp = q8 >> 3, jj = q8 & 7;
+            *reinterpret_cast<uint4*>(sop + grp * (D * kRowBytes) + sw128_off(row, jj)) =
+                make_uint4(wp[4 * h2], wp[4 * h2 + 1], wp[4 * h2 + 2], wp[4 * h2 + 3]);
+          }
         }
       }
-      named_bar_sync(2, 128);
-      if (x == 0) mbar_arrive(bars.s_empty);
-      if (!mbar_wait(&bars.sop_empty[buf], (use & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
-        return false;
-      if (has_row) {
-        uint8_t* sop = sSOP + buf * K::SOPT;
+      if (src == kFromCarry && a.causal) tmem_wait_st();
+      if (src != kFromZero) tc_fence_before();
+      if (!kStream) {
+        named_bar_sync(2, 128);
+        if (x == 0) mbar_arrive(bars.s_empty);
+        if (!mbar_wait(&bars.sop_empty[buf], (use & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+          return false;
+        if (has_row) {
 #pragma unroll
-        for (int q8 = 0; q8 < (DV + 16) / 8; ++q8) {
-          const int grp = q8 >> 3, jj = q8 & 7;
-          *reinterpret_cast<uint4*>(sop + grp * (D * kRowBytes) + sw128_off(row, jj)) =
-              make_uint4(w[4 * q8], w[4 * q8 + 1], w[4 * q8 + 2], w[4 * q8 + 3]);
+          for (int q8 = 0; q8 < (DV + 16) / 8; ++q8) {
+            const int grp = q8 >> 3, jj = q8 & 7;
+            *reinterpret_cast<uint4*>(sop + grp * (D * kRowBytes) + sw128_off(row, jj)) =
+                make_uint4(w[4 * q8], w[4 * q8 + 1], w[4 * q8 + 2], w[4 * q8 + 3]);
+          }
         }
       }
       fence_proxy_async_smem();
       named_bar_sync(2, 128);
-      if (x == 0) mbar_arrive(&bars.sop_full[buf]);
+      if (x == 0) {
+        if (kStream) mbar_arrive(bars.s_empty);
+        mbar_arrive(&bars.sop_full[buf]);
+      }
       return true;
     };
+    // Output rows of item j.  Each warp owns 32 rows; per 32-column block a
+    // thread packs its row into the warp's staging tile (16-byte pieces
+    // XOR-swizzled by row so neither the writes nor the reads conflict), and
+    // the warp then stores 8 rows x 64 bytes per instruction.
+    uint8_t* const stg = sOST + sp * (32 * 64);
     auto epilogue = [&](int j) -> bool {
       const int c = j / G, h = j % G, as = j % K::NA;
       if (!mbar_wait(&bars.acc_full[as], (j / K::NA) & 1, abort_flag, a.err, kWaitLimitNs))
@@ -603,24 +636,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_ld();
       const float inv = 1.0f / (t16[0] + a.eps);
       const int valid = min(kChunk, n - c * kChunk);
-      const bool store = x < valid;
-      __nv_bfloat16* orow =
-          a.out + ((size_t)(t0 + c * kChunk + x) * a.Hq + (size_t)(g * G + h)) * DV;
+      const size_t ostride = (size_t)a.Hq * DV;
+      __nv_bfloat16* const obase =
+          a.out + ((size_t)(t0 + c * kChunk + sp * 32) * a.Hq + (size_t)(g * G + h)) * DV;
+      const int rd_row = lane >> 2, rd_piece = lane & 3;
 #pragma unroll 1
       for (int cb = 0; cb < DV / 32; ++cb) {
         float r[32];
         tmem_ld32(t_acc + cb * 32, r);
         tmem_wait_ld();
-        if (store) {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const uint4 w = make_uint4(pack_bf16x2(r[q4 * 8 + 0] * inv, r[q4 * 8 + 1] * inv),
-                                       pack_bf16x2(r[q4 * 8 + 2] * inv, r[q4 * 8 + 3] * inv),
-                                       pack_bf16x2(r[q4 * 8 + 4] * inv, r[q4 * 8 + 5] * inv),
-                                       pack_bf16x2(r[q4 * 8 + 6] * inv, r[q4 * 8 + 7] * inv));
-            *reinterpret_cast<uint4*>(orow + cb * 32 + q4 * 8) = w;
-          }
+        for (int q4 = 0; q4 < 4; ++q4)
+          *reinterpret_cast<uint4*>(stg + lane * 64 + ((q4 ^ ((lane >> 1) & 3)) << 4)) =
+              make_uint4(pack_bf16x2(r[q4 * 8 + 0] * inv, r[q4 * 8 + 1] * inv),
+                         pack_bf16x2(r[q4 * 8 + 2] * inv, r[q4 * 8 + 3] * inv),
+                         pack_bf16x2(r[q4 * 8 + 4] * inv, r[q4 * 8 + 5] * inv),
+                         pack_bf16x2(r[q4 * 8 + 6] * inv, r[q4 * 8 + 7] * inv));
+        __syncwarp();
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8) {
+          const int rr = k8 * 8 + rd_row;  // row within the warp's 32
+          const uint4 v = *reinterpret_cast<const uint4*>(
+              stg + rr * 64 + ((rd_piece ^ ((rr >> 1) & 3)) << 4));
+          if (sp * 32 + rr < valid)
+            *reinterpret_cast<uint4*>(obase + (size_t)rr * ostride + cb * 32 + rd_piece * 8) = v;
         }
+        __syncwarp();
       }
       tc_fence_before();
       named_bar_sync(2, 128);
@@ -653,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, K::TM_COLS);
   }
