@@ -322,63 +322,72 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
 
       if (a.causal) {
-        auto issue_acc = [&](int j) -> bool {
-          const int c = j / G, h = j % G;
-          const int pbs = j % K::NPB, as = j % K::NA, qs = j % K::NQ;
-          if (!mbar_wait(&bars.pb_full[pbs], (j / K::NPB) & 1, abort_flag, a.err, kWaitLimitNs))
-            return false;
-          if (h == 0 && !mbar_wait(&bars.sop_full[c % K::NSOP], (c / K::NSOP) & 1, abort_flag,
-                                   a.err, kWaitLimitNs))
-            return false;
-          if (!mbar_wait(&bars.acc_empty[as], ((j / K::NA) & 1) ^ 1, abort_flag, a.err,
-                         kWaitLimitNs))
-            return false;
-          tc_fence_after();
-          const uint32_t t_acc = tmem + K::TM_ACC + as * K::ACCW;
-          const uint32_t pb = sPBa + pbs * K::PBT;
-          const uint32_t vb = sVa + (c % K::NKV) * K::VT;
-          for (int kk = 0; kk < kChunk / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(pb + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024);
-            umma_f16_ss(t_acc, ad, smem_desc_sw128(vb + kk * 2048, kBox, 1024), ID_PV,
-                        kk > 0 ? 1u : 0u);
-            umma_f16_ss(t_acc + DV, ad, smem_desc_sw128(sONESa + (kk & 3) * 32, 16, 1024), ID_P1,
-                        kk > 0 ? 1u : 0u);
-          }
-          issue_qs(t_acc, sQa + qs * K::QT, sSOPa + (c % K::NSOP) * K::SOPT, true);
-          umma_commit(&bars.acc_full[as]);
-          umma_commit(&bars.pb_empty[pbs]);
-          umma_commit(&bars.q_empty[qs]);
-          if (h == G - 1) {
-            umma_commit(&bars.kv_empty[c % K::NKV]);
-            umma_commit(&bars.sop_empty[c % K::NSOP]);
-          }
-          return true;
-        };
-        for (int i = 0; i < n_items && ok; ++i) {
-          const int c = i / G;
-          // single K/V stage: the previous chunk's last accumulator MMA must
-          // be issued (it releases the stage) before waiting for new tiles
-          const bool flush_first = (K::NKV == 1) && (i % G == 0) && i > 0;
-          if (flush_first) {
-            ok = issue_acc(i - 1);
-            if (!ok) break;
-          }
-          if (i % G == 0) {
-            const int st = c % K::NKV;
-            ok = mbar_wait(&bars.kv_xf[st], (c / K::NKV) & 1, abort_flag, a.err, kWaitLimitNs) &&
-                 mbar_wait(bars.s_empty, c & 1, abort_flag, a.err, kWaitLimitNs);
-            if (!ok) break;
+        // Per item j (chunk c = j / G, head h = j % G) four groups of MMAs,
+        // issued by polling so that a group whose inputs are ready never
+        // waits behind one whose inputs are late (a Q tile still landing,
+        // the carry still being summed):
+        //   ST(c)  S_acc += phi(K_c)^T [V_c | 1], once K_c is transformed
+        //          and [S|z]_<c has been read out of TMEM
+        //   SC(j)  score tile phi(Q) phi(K_c)^T, once both tiles are
+        //          transformed and the mask warps have read the last one
+        //   PV(j)  Acc = P [V | 1], once P is masked and staged and the
+        //          epilogue has drained the accumulator
+        //   QS(j)  Acc += phi(Q) [S|z]_<c, after PV(j), once the chunk's
+        //          operand is staged
+        // Each barrier is tested only after the previous phase of the same
+        // barrier has been consumed in program order, so a parity test never
+        // sees a stale phase.  The K/V stage is released after PV of the
+        // chunk's last item, which therefore also waits for ST(c).
+        const int last_h = G - 1;
+        int st = 0, sc = 0, pv = 0, qn = 0;
+        uint32_t idle = 0;
+        uint64_t idle_t0 = 0;
+        while (qn < n_items && ok) {
+          bool did = false;
+          if (qn < pv && (qn % G != 0 || mbar_test(&bars.sop_full[(qn / G) % K::NSOP],
+                                                     ((qn / G) / K::NSOP) & 1))) {
             tc_fence_after();
-            issue_state(c, c > 0 || has_carry);
+            const int c = qn / G, as = qn % K::NA, qs = qn % K::NQ;
+            issue_qs(tmem + K::TM_ACC + as * K::ACCW, sQa + qs * K::QT,
+                     sSOPa + (c % K::NSOP) * K::SOPT, true);
+            umma_commit(&bars.acc_full[as]);
+            umma_commit(&bars.q_empty[qs]);
+            if (qn % G == last_h) umma_commit(&bars.sop_empty[c % K::NSOP]);
+            ++qn;
+            did = true;
+          } else if (st < nc && st * G <= sc &&
+                     mbar_test(&bars.kv_xf[st % K::NKV], (st / K::NKV) & 1) &&
+                     mbar_test(bars.s_empty, st & 1)) {
+            tc_fence_after();
+            issue_state(st, st > 0 || has_carry);
             umma_commit(bars.s_full);
-          }
-          const int qs = i % K::NQ, ps = i % K::NP;
-          ok = mbar_wait(&bars.q_xf[qs], (i / K::NQ) & 1, abort_flag, a.err, kWaitLimitNs) &&
-               mbar_wait(&bars.p_empty[ps], ((i / K::NP) & 1) ^ 1, abort_flag, a.err,
-                         kWaitLimitNs);
-          if (!ok) break;
-          tc_fence_after();
-          {
+            ++st;
+            did = true;
+          } else if (pv < sc && (pv % G != last_h || st > pv / G) &&
+                     mbar_test(&bars.pb_full[pv % K::NPB], (pv / K::NPB) & 1) &&
+                     mbar_test(&bars.acc_empty[pv % K::NA], ((pv / K::NA) & 1) ^ 1)) {
+            tc_fence_after();
+            const int c = pv / G, pbs = pv % K::NPB, as = pv % K::NA;
+            const uint32_t t_acc = tmem + K::TM_ACC + as * K::ACCW;
+            const uint32_t pb = sPBa + pbs * K::PBT;
+            const uint32_t vb = sVa + (c % K::NKV) * K::VT;
+            for (int kk = 0; kk < kChunk / 16; ++kk) {
+              const uint64_t ad = smem_desc_sw128(pb + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024);
+              umma_f16_ss(t_acc, ad, smem_desc_sw128(vb + kk * 2048, kBox, 1024), ID_PV,
+                          kk > 0 ? 1u : 0u);
+              umma_f16_ss(t_acc + DV, ad, smem_desc_sw128(sONESa + (kk & 3) * 32, 16, 1024), ID_P1,
+                          kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars.pb_empty[pbs]);
+            if (pv % G == last_h) umma_commit(&bars.kv_empty[c % K::NKV]);
+            ++pv;
+            did = true;
+          } else if (sc < n_items &&
+                     mbar_test(&bars.kv_xf[(sc / G) % K::NKV], ((sc / G) / K::NKV) & 1) &&
+                     mbar_test(&bars.q_xf[sc % K::NQ], (sc / K::NQ) & 1) &&
+                     mbar_test(&bars.p_empty[sc % K::NP], ((sc / K::NP) & 1) ^ 1)) {
+            tc_fence_after();
+            const int c = sc / G, qs = sc % K::NQ, ps = sc % K::NP;
             const uint32_t t_p = tmem + K::TM_P + ps * kChunk;
             const uint32_t qb = sQa + qs * K::QT, kb = sKa + (c % K::NKV) * K::KT;
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -387,10 +396,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                           smem_desc_sw128(kb + o, 16, 1024), ID_P, kk > 0 ? 1u : 0u);
             }
             umma_commit(&bars.p_full[ps]);
+            ++sc;
+            did = true;
           }
-          if (i > 0 && !flush_first) ok = issue_acc(i - 1);
+          if (did) {
+            idle = 0;
+          } else if ((++idle & 255u) == 0) {
+            if (*abort_flag) {
+              ok = false;
+            } else if (idle == 256) {
+              idle_t0 = global_timer_ns();
+            } else if (global_timer_ns() - idle_t0 > kWaitLimitNs) {
+              *abort_flag = 1;
+              report_error(a.err, kDevErrTimeout);
+              ok = false;
+            }
+          }
         }
-        if (ok && n_items > 0) ok = issue_acc(n_items - 1);
       } else {
         if (!carried_state) {
           for (int c = 0; c < nc && ok; ++c) {
@@ -560,7 +582,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) c16[e] = 0.0f;
           if (has_row) {
-            for (int bb = 0; bb < nsum; ++bb) {
+            // in block order; kU aggregates' loads in flight at a time
+            constexpr int kU = kStream ? 4 : 2;
+            int bb = 0;
+            for (; bb + kU <= nsum; bb += kU) {
+              if (cb < DV / 16) {
+                float4 v4[kU][4];
+#pragma unroll
+                for (int u2 = 0; u2 < kU; ++u2) {
+                  const float4* r4 = reinterpret_cast<const float4*>(
+                      base + (size_t)(bb + u2) * E + row * DV + cb * 16);
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) v4[u2][u] = r4[u];
+                }
+#pragma unroll
+                for (int u2 = 0; u2 < kU; ++u2)
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) {
+                    c16[4 * u] += v4[u2][u].x;
+                    c16[4 * u + 1] += v4[u2][u].y;
+                    c16[4 * u + 2] += v4[u2][u].z;
+                    c16[4 * u + 3] += v4[u2][u].w;
+                  }
+              } else {
+                float zv[kU];
+#pragma unroll
+                for (int u2 = 0; u2 < kU; ++u2) zv[u2] = base[(size_t)(bb + u2) * E + D * DV + row];
+#pragma unroll
+                for (int u2 = 0; u2 < kU; ++u2) c16[0] += zv[u2];
+              }
+            }
+            for (; bb < nsum; ++bb) {
               if (cb < DV / 16) {
                 const float4* r4 =
                     reinterpret_cast<const float4*>(base + (size_t)bb * E + row * DV + cb * 16);
