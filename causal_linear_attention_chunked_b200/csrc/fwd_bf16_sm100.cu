@@ -21,17 +21,20 @@
 // served from the same K/V tiles and the same state.  With more than one
 // block per sequence the state of a block starts from the carry summed from
 // the block aggregates of the state launch (earlier blocks when causal,
-// every block when not), written into the TMEM state accumulator.  Warp roles (448 threads):
+// every block when not), written into the TMEM state accumulator.  Warp roles (480 threads):
 //   warps 0-3   phi warpgroup: phi applied in place to the TMA-loaded K and
 //               Q tiles, tail rows zeroed.
-//   warps 4-7   mask warpgroup: causal mask of the score tile, conversion
-//               to bf16, staging as the A operand of P V.
+//   warps 4-7   mask warpgroup: causal mask of the score tile and
+//               conversion to bf16, in place in TMEM, where P V reads it as
+//               its A operand.
 //   warps 8-11  state/epilogue warpgroup: TMEM state -> bf16 operand;
 //               TMEM accumulator -> normalised bf16 rows, transposed through
 //               a small shared-memory tile per warp so that every store
 //               instruction writes whole 64-byte row segments.
-//   warp 12     TMA producer.
+//   warp 12     TMA producer of the K/V tiles.
 //   warp 13     TMEM allocator and single-thread MMA issuer.
+//   warp 14     TMA producer of the Q tiles (a Q tile never waits behind a
+//               K/V stage that is still in use).
 // Non-causal mode (phi(Q)(phi(K)^T V) normalised the same way): first the
 // state over all chunks (K, V only; taken from the block aggregates when the
 // sequence is split into blocks), then every output row as phi(Q_i) [S|z]_n
@@ -49,7 +52,7 @@
 namespace lt {
 namespace {
 
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 using namespace fwd;
 
 template <int D, int DV>
@@ -57,13 +60,11 @@ struct Cfg {
   static constexpr int QT = kChunk * D * 2;
   static constexpr int KT = kChunk * D * 2;
   static constexpr int VT = kChunk * DV * 2;
-  static constexpr int PBT = kChunk * kChunk * 2;
   static constexpr int SOPT = (DV / 64 + 1) * D * kRowBytes;  // [S | z 0..] operand
   static constexpr int ONEST = 16 * kRowBytes;  // K-major [1 | 0..] block, N = 16 rows
   static constexpr int OSTT = 4 * 32 * 64;  // epilogue staging: 32 rows x 64 B per warp
-  static constexpr int NQ = (D == 64 && DV == 64) ? 3 : 2;
+  static constexpr int NQ = 3;
   static constexpr int NKV = (D == 128) ? 1 : 2;
-  static constexpr int NPB = (DV == 128) ? 1 : 2;
   static constexpr int NSOP = (D == 128) ? 1 : 2;
   static constexpr int ACCW = DV + 16;  // numerator columns + normaliser block
   static constexpr int NP = (D == 64 && DV == 128) ? 1 : (DV == 64 ? 2 : 1);
@@ -77,12 +78,11 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * QT;
   static constexpr int OFF_V = OFF_K + NKV * KT;
-  static constexpr int OFF_PB = OFF_V + NKV * VT;
-  static constexpr int OFF_SOP = OFF_PB + NPB * PBT;
+  static constexpr int OFF_SOP = OFF_V + NKV * VT;
   static constexpr int OFF_ONES = OFF_SOP + NSOP * SOPT;
   static constexpr int OFF_OST = OFF_ONES + 1024 * ((ONEST + 1023) / 1024);
   static constexpr int OFF_BAR = OFF_OST + OSTT;
-  static constexpr int NBARS = 4 * NQ + 3 * NKV + 2 * NP + 2 * NPB + 2 * NSOP + 2 + 2 * NA + 1;
+  static constexpr int NBARS = 4 * NQ + 3 * NKV + 2 * NP + 2 * NSOP + 2 + 2 * NA + 1;
   static constexpr int SMEM = OFF_BAR + NBARS * 8 + 16 + 1024;  // + tmem slot + align slack
   static_assert(SMEM <= 232448, "shared memory budget");
 };
@@ -90,8 +90,7 @@ struct Cfg {
 struct Bars {
   uint64_t *q_full, *q_empty, *q_xf, *q_spare;
   uint64_t *kv_full, *kv_empty, *kv_xf;
-  uint64_t *p_full, *p_empty;
-  uint64_t *pb_full, *pb_empty;
+  uint64_t *p_full, *pb_full;
   uint64_t *sop_full, *sop_empty;
   uint64_t *s_full, *s_empty;
   uint64_t *acc_full, *acc_empty;
@@ -111,9 +110,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
   r.kv_empty = b; b += K::NKV;
   r.kv_xf = b; b += K::NKV;
   r.p_full = b; b += K::NP;
-  r.p_empty = b; b += K::NP;
-  r.pb_full = b; b += K::NPB;
-  r.pb_empty = b; b += K::NPB;
+  r.pb_full = b; b += K::NP;
   r.sop_full = b; b += K::NSOP;
   r.sop_empty = b; b += K::NSOP;
   r.s_full = b; b += 1;
@@ -177,7 +174,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem + K::OFF_Q;
   uint8_t* sK = smem + K::OFF_K;
   uint8_t* sV = smem + K::OFF_V;
-  uint8_t* sPB = smem + K::OFF_PB;
   uint8_t* sSOP = smem + K::OFF_SOP;
   uint8_t* sONES = smem + K::OFF_ONES;
   uint8_t* sOST = smem + K::OFF_OST;
@@ -199,11 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < K::NP; ++i) {
       mbar_init(&bars.p_full[i], 1);
-      mbar_init(&bars.p_empty[i], 1);
-    }
-    for (int i = 0; i < K::NPB; ++i) {
       mbar_init(&bars.pb_full[i], 1);
-      mbar_init(&bars.pb_empty[i], 1);
     }
     for (int i = 0; i < K::NSOP; ++i) {
       mbar_init(&bars.sop_full[i], 1);
@@ -233,13 +225,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   volatile int* abort_flag = &s_abort;
 
-  if (warp == 12) {
-    // ------------------------------------------------------------ producer
+  if (warp == 12 || warp == 14) {
+    // ----------------------------------------------- producers (K/V, Q)
     if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      int q_issued = 0, kv_issued = 0;
+      const bool q_side = warp == 14;
+      if (q_side) {
+        prefetch_tmap(&tm_q);
+      } else {
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+      }
+      int issued = 0;
       bool ok = true;
       auto load_kv = [&](int c) -> bool {
         const int st = c % K::NKV;
@@ -252,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int bx = 0; bx < DV / 64; ++bx)
           tma_load_3d(sV + st * K::VT + bx * kBox, &tm_v, &bars.kv_full[st], bx * 64, g,
                       t0 + c * kChunk);
-        ++kv_issued;
+        ++issued;
         return true;
       };
       auto load_q = [&](int i) -> bool {
@@ -264,26 +260,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int bx = 0; bx < D / 64; ++bx)
           tma_load_3d(sQ + st * K::QT + bx * kBox, &tm_q, &bars.q_full[st], bx * 64,
                       g * G + h, t0 + c * kChunk);
-        ++q_issued;
+        ++issued;
         return true;
       };
-      if (a.causal) {
-        for (int i = 0; i < n_items && ok; ++i) {
-          if (i % G == 0) ok = load_kv(i / G);
-          if (ok) ok = load_q(i);
-        }
-      } else {
-        if (!carried_state)
-          for (int c = 0; c < nc && ok; ++c) ok = load_kv(c);
+      if (q_side) {
         for (int i = 0; i < n_items && ok; ++i) ok = load_q(i);
+      } else if (a.causal || !carried_state) {
+        for (int c = 0; c < nc && ok; ++c) ok = load_kv(c);
       }
       if (!ok) {
         // drain: wait (bounded, ignoring the abort flag) for copies in flight
         int dummy = 0;
-        for (int c = (kv_issued > K::NKV ? kv_issued - K::NKV : 0); c < kv_issued; ++c)
-          mbar_wait(&bars.kv_full[c % K::NKV], (c / K::NKV) & 1, &dummy, nullptr, kWaitLimitNs);
-        for (int i = (q_issued > K::NQ ? q_issued - K::NQ : 0); i < q_issued; ++i)
-          mbar_wait(&bars.q_full[i % K::NQ], (i / K::NQ) & 1, &dummy, nullptr, kWaitLimitNs);
+        const int depth = q_side ? K::NQ : K::NKV;
+        uint64_t* full = q_side ? bars.q_full : bars.kv_full;
+        for (int u = (issued > depth ? issued - depth : 0); u < issued; ++u)
+          mbar_wait(&full[u % depth], (u / depth) & 1, &dummy, nullptr, kWaitLimitNs);
       }
     }
   } else if (warp == 13) {
@@ -296,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t ID_P1 = idesc_bf16_f32(kChunk, 16, 0, 0);
       constexpr uint32_t ID_QS = idesc_bf16_f32(kChunk, DV + 16, 0, 1);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      const uint32_t sPBa = smem_u32(sPB), sSOPa = smem_u32(sSOP), sONESa = smem_u32(sONES);
+      const uint32_t sSOPa = smem_u32(sSOP), sONESa = smem_u32(sONES);
       const uint32_t t_s = tmem + K::TM_S;
       bool ok = true;
 
@@ -364,28 +355,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++st;
             did = true;
           } else if (pv < sc && (pv % G != last_h || st > pv / G) &&
-                     mbar_test(&bars.pb_full[pv % K::NPB], (pv / K::NPB) & 1) &&
+                     mbar_test(&bars.pb_full[pv % K::NP], (pv / K::NP) & 1) &&
                      mbar_test(&bars.acc_empty[pv % K::NA], ((pv / K::NA) & 1) ^ 1)) {
             tc_fence_after();
-            const int c = pv / G, pbs = pv % K::NPB, as = pv % K::NA;
+            const int c = pv / G, as = pv % K::NA;
             const uint32_t t_acc = tmem + K::TM_ACC + as * K::ACCW;
-            const uint32_t pb = sPBa + pbs * K::PBT;
+            // A = the masked bf16 scores, in place in TMEM: 16 keys (8
+            // columns) per MMA
+            const uint32_t t_pb = tmem + K::TM_P + (pv % K::NP) * kChunk;
             const uint32_t vb = sVa + (c % K::NKV) * K::VT;
             for (int kk = 0; kk < kChunk / 16; ++kk) {
-              const uint64_t ad = smem_desc_sw128(pb + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024);
-              umma_f16_ss(t_acc, ad, smem_desc_sw128(vb + kk * 2048, kBox, 1024), ID_PV,
+              umma_f16_ts(t_acc, t_pb + kk * 8, smem_desc_sw128(vb + kk * 2048, kBox, 1024), ID_PV,
                           kk > 0 ? 1u : 0u);
-              umma_f16_ss(t_acc + DV, ad, smem_desc_sw128(sONESa + (kk & 3) * 32, 16, 1024), ID_P1,
-                          kk > 0 ? 1u : 0u);
+              umma_f16_ts(t_acc + DV, t_pb + kk * 8, smem_desc_sw128(sONESa + (kk & 3) * 32, 16, 1024),
+                          ID_P1, kk > 0 ? 1u : 0u);
             }
-            umma_commit(&bars.pb_empty[pbs]);
             if (pv % G == last_h) umma_commit(&bars.kv_empty[c % K::NKV]);
             ++pv;
             did = true;
-          } else if (sc < n_items &&
+          } else if (sc < n_items && pv > sc - K::NP &&
                      mbar_test(&bars.kv_xf[(sc / G) % K::NKV], ((sc / G) / K::NKV) & 1) &&
-                     mbar_test(&bars.q_xf[sc % K::NQ], (sc / K::NQ) & 1) &&
-                     mbar_test(&bars.p_empty[sc % K::NP], ((sc / K::NP) & 1) ^ 1)) {
+                     mbar_test(&bars.q_xf[sc % K::NQ], (sc / K::NQ) & 1)) {
             tc_fence_after();
             const int c = sc / G, qs = sc % K::NQ, ps = sc % K::NP;
             const uint32_t t_p = tmem + K::TM_P + ps * kChunk;
@@ -485,52 +475,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int x = tid - 128;  // 0..127 == TMEM lane == chunk row
     const int sp = warp & 3;  // TMEM sub-partition of this warp
     bool ok = true;
-    // mask + convert the score tile of item j into the bf16 A operand
+    // Causal mask and bf16 rounding of the score tile of item j, in place in
+    // TMEM (the A operand of P [V | 1]): fp32 columns [32b, 32b+32) become
+    // packed bf16 columns [16b, 16b+16), which only overwrites columns this
+    // thread has already read.  The buffer is reused by the score MMA of
+    // item j + NP, which the issuer orders after P V(j) (the pipe is in order).
     auto mask_p = [&](int j) -> bool {
-      const int ps = j % K::NP, pbs = j % K::NPB;
+      const int ps = j % K::NP;
       if (!mbar_wait(&bars.p_full[ps], (j / K::NP) & 1, abort_flag, a.err, kWaitLimitNs))
-        return false;
-      if (!mbar_wait(&bars.pb_empty[pbs], ((j / K::NPB) & 1) ^ 1, abort_flag, a.err,
-                     kWaitLimitNs))
         return false;
       tc_fence_after();
       const uint32_t t_p = tmem + K::TM_P + ps * kChunk + ((uint32_t)(sp * 32) << 16);
-      uint8_t* pb = sPB + pbs * K::PBT;
       const int row = x;
 #pragma unroll 1
       for (int b = 0; b < kChunk / 32; ++b) {
-        uint4 w[4];
+        uint32_t pk[16];
         if (b <= sp) {  // warp-uniform: blocks right of the diagonal are all zero
           float r[32];
           tmem_ld32(t_p + b * 32, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (b * 32 + e > row) r[e] = 0.0f;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            w[q4] = make_uint4(pack_bf16x2(r[q4 * 8 + 0], r[q4 * 8 + 1]),
-                               pack_bf16x2(r[q4 * 8 + 2], r[q4 * 8 + 3]),
-                               pack_bf16x2(r[q4 * 8 + 4], r[q4 * 8 + 5]),
-                               pack_bf16x2(r[q4 * 8 + 6], r[q4 * 8 + 7]));
+          for (int e = 0; e < 16; ++e) {
+            const float lo = (b * 32 + 2 * e > row) ? 0.0f : r[2 * e];
+            const float hi = (b * 32 + 2 * e + 1 > row) ? 0.0f : r[2 * e + 1];
+            pk[e] = pack_bf16x2(lo, hi);
+          }
         } else {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) w[q4] = make_uint4(0u, 0u, 0u, 0u);
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
         }
-        const int kb = b >> 1;  // 64-key block
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int jj = (b & 1) * 4 + q4;
-          *reinterpret_cast<uint4*>(pb + kb * kBox + sw128_off(row, jj)) = w[q4];
-        }
+        tmem_st16(t_p + b * 16, pk);
       }
+      tmem_wait_st();
       tc_fence_before();
-      fence_proxy_async_smem();
       named_bar_sync(3, 128);
-      if (x == 0) {
-        mbar_arrive(&bars.p_empty[ps]);
-        mbar_arrive(&bars.pb_full[pbs]);
-      }
+      if (x == 0) mbar_arrive(&bars.pb_full[ps]);
       return true;
     };
     if (a.causal)
@@ -572,7 +551,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int E = D * DV + D;
       const float* base = a.ws != nullptr ? a.ws + (size_t)(s * a.Hkv + g) * a.nb * E : nullptr;
       const int nsum = src == kFromCarry ? (a.causal ? blk : a.nb) : 0;
-#pragma unroll
+      // streamed: a loop (the first staging runs cold, while every CTA's
+      // first tiles are in flight, and straight-line code would miss the
+      // instruction cache line after line); held: unrolled, w stays in
+      // registers
+      constexpr int kStageUnroll = kStream ? 1 : (DV + 16) / 16;
+#pragma unroll kStageUnroll
       for (int cb = 0; cb < (DV + 16) / 16; ++cb) {
         float c16[16];
         if (src == kFromTmem) {
