@@ -55,6 +55,31 @@ namespace {
 constexpr int kThreads = 480;
 using namespace fwd;
 
+// phi in place over a full [kChunk x (NBOX*64)] bf16 tile by 128 threads, as
+// a loop with four 16-byte pieces in flight per thread (compact code: this
+// kernel's warp roles share each sub-partition's instruction cache)
+template <int NBOX>
+__device__ __forceinline__ void phi_tile_loop(uint8_t* tile, int tid) {
+  constexpr int kIt = kChunk * NBOX * 8 / 128;
+  static_assert(kIt % 4 == 0, "pieces per thread");
+  uint4* p = reinterpret_cast<uint4*>(tile) + tid;
+#pragma unroll 1
+  for (int i = 0; i < kIt; i += 4) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = p[(i + u) * 128];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      v[u].x = phi_bf16x2(v[u].x);
+      v[u].y = phi_bf16x2(v[u].y);
+      v[u].z = phi_bf16x2(v[u].z);
+      v[u].w = phi_bf16x2(v[u].w);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) p[(i + u) * 128] = v[u];
+  }
+}
+
 template <int D, int DV>
 struct Cfg {
   static constexpr int QT = kChunk * D * 2;
@@ -442,7 +467,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&bars.kv_full[st], (c / K::NKV) & 1, abort_flag, a.err, kWaitLimitNs))
         return false;
       const int valid = min(kChunk, n - c * kChunk);
-      prep_tile<D / 64, 128>(sK + st * K::KT, valid, true, x);
+      if (valid >= kChunk)
+        phi_tile_loop<D / 64>(sK + st * K::KT, x);
+      else
+        xf_tile<D / 64, 128>(sK + st * K::KT, valid, true, x);
       prep_tile<DV / 64, 128>(sV + st * K::VT, valid, false, x);
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
@@ -454,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = i % K::NQ;
       if (!mbar_wait(&bars.q_full[st], (i / K::NQ) & 1, abort_flag, a.err, kWaitLimitNs))
         return false;
-      phi_tile_full<D / 64, 128>(sQ + st * K::QT, x);
+      phi_tile_loop<D / 64>(sQ + st * K::QT, x);
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
       if (x == 0) mbar_arrive(&bars.q_xf[st]);
