@@ -31,7 +31,8 @@
 //               TMEM accumulator -> normalised bf16 rows, transposed through
 //               a small shared-memory tile per warp so that every store
 //               instruction writes whole 64-byte row segments.
-//   warp 12     TMA producer of the K/V tiles.
+//   warp 12     TMA producer of the K and V tiles (separate stages: K
+//               frees a chunk earlier than V).
 //   warp 13     TMEM allocator and single-thread MMA issuer.
 //   warp 14     TMA producer of the Q tiles (a Q tile never waits behind a
 //               K/V stage that is still in use).
@@ -107,14 +108,15 @@ struct Cfg {
   static constexpr int OFF_ONES = OFF_SOP + NSOP * SOPT;
   static constexpr int OFF_OST = OFF_ONES + 1024 * ((ONEST + 1023) / 1024);
   static constexpr int OFF_BAR = OFF_OST + OSTT;
-  static constexpr int NBARS = 4 * NQ + 3 * NKV + 2 * NP + 2 * NSOP + 2 + 2 * NA + 1;
+  static constexpr int NBARS = 4 * NQ + 6 * NKV + 2 * NP + 2 * NSOP + 2 + 2 * NA + 1;
   static constexpr int SMEM = OFF_BAR + NBARS * 8 + 16 + 1024;  // + tmem slot + align slack
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 struct Bars {
   uint64_t *q_full, *q_empty, *q_xf, *q_spare;
-  uint64_t *kv_full, *kv_empty, *kv_xf;
+  uint64_t *k_full, *k_empty, *k_xf;
+  uint64_t *v_full, *v_empty, *v_xf;
   uint64_t *p_full, *pb_full;
   uint64_t *sop_full, *sop_empty;
   uint64_t *s_full, *s_empty;
@@ -131,9 +133,12 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
   r.q_empty = b; b += K::NQ;
   r.q_xf = b; b += K::NQ;
   r.q_spare = b; b += K::NQ;
-  r.kv_full = b; b += K::NKV;
-  r.kv_empty = b; b += K::NKV;
-  r.kv_xf = b; b += K::NKV;
+  r.k_full = b; b += K::NKV;
+  r.k_empty = b; b += K::NKV;
+  r.k_xf = b; b += K::NKV;
+  r.v_full = b; b += K::NKV;
+  r.v_empty = b; b += K::NKV;
+  r.v_xf = b; b += K::NKV;
   r.p_full = b; b += K::NP;
   r.pb_full = b; b += K::NP;
   r.sop_full = b; b += K::NSOP;
@@ -214,9 +219,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.q_spare[i], 1);
     }
     for (int i = 0; i < K::NKV; ++i) {
-      mbar_init(&bars.kv_full[i], 1);
-      mbar_init(&bars.kv_empty[i], 1);
-      mbar_init(&bars.kv_xf[i], 1);
+      mbar_init(&bars.k_full[i], 1);
+      mbar_init(&bars.k_empty[i], 1);
+      mbar_init(&bars.k_xf[i], 1);
+      mbar_init(&bars.v_full[i], 1);
+      mbar_init(&bars.v_empty[i], 1);
+      mbar_init(&bars.v_xf[i], 1);
     }
     for (int i = 0; i < K::NP; ++i) {
       mbar_init(&bars.p_full[i], 1);
@@ -260,20 +268,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
       }
-      int issued = 0;
+      int issued = 0, v_issued = 0;
       bool ok = true;
-      auto load_kv = [&](int c) -> bool {
+      // K and V have stages of their own: K frees once the chunk's last score
+      // and its state MMA are done, V only after the chunk's last P V
+      auto load_kv = [&](int c, bool is_v) -> bool {
         const int st = c % K::NKV;
-        if (!mbar_wait(&bars.kv_empty[st], ((c / K::NKV) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
+        uint64_t* empty = is_v ? bars.v_empty : bars.k_empty;
+        uint64_t* full = is_v ? bars.v_full : bars.k_full;
+        if (!mbar_wait(&empty[st], ((c / K::NKV) & 1) ^ 1, abort_flag, a.err, kWaitLimitNs))
           return false;
-        mbar_arrive_expect_tx(&bars.kv_full[st], K::KT + K::VT);
-        for (int bx = 0; bx < D / 64; ++bx)
-          tma_load_3d(sK + st * K::KT + bx * kBox, &tm_k, &bars.kv_full[st], bx * 64, g,
-                      t0 + c * kChunk);
-        for (int bx = 0; bx < DV / 64; ++bx)
-          tma_load_3d(sV + st * K::VT + bx * kBox, &tm_v, &bars.kv_full[st], bx * 64, g,
-                      t0 + c * kChunk);
-        ++issued;
+        mbar_arrive_expect_tx(&full[st], is_v ? K::VT : K::KT);
+        for (int bx = 0; bx < (is_v ? DV : D) / 64; ++bx)
+          tma_load_3d((is_v ? sV + st * K::VT : sK + st * K::KT) + bx * kBox, is_v ? &tm_v : &tm_k,
+                      &full[st], bx * 64, g, t0 + c * kChunk);
+        ++(is_v ? v_issued : issued);
         return true;
       };
       auto load_q = [&](int i) -> bool {
@@ -291,15 +300,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (q_side) {
         for (int i = 0; i < n_items && ok; ++i) ok = load_q(i);
       } else if (a.causal || !carried_state) {
-        for (int c = 0; c < nc && ok; ++c) ok = load_kv(c);
+        for (int c = 0; c < nc && ok; ++c) {
+          ok = load_kv(c, false);
+          if (ok) ok = load_kv(c, true);
+        }
       }
       if (!ok) {
         // drain: wait (bounded, ignoring the abort flag) for copies in flight
         int dummy = 0;
         const int depth = q_side ? K::NQ : K::NKV;
-        uint64_t* full = q_side ? bars.q_full : bars.kv_full;
+        uint64_t* full = q_side ? bars.q_full : bars.k_full;
         for (int u = (issued > depth ? issued - depth : 0); u < issued; ++u)
           mbar_wait(&full[u % depth], (u / depth) & 1, &dummy, nullptr, kWaitLimitNs);
+        for (int u = (v_issued > depth ? v_issued - depth : 0); u < v_issued; ++u)
+          mbar_wait(&bars.v_full[u % depth], (u / depth) & 1, &dummy, nullptr, kWaitLimitNs);
       }
     }
   } else if (warp == 13) {
@@ -356,6 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // chunk's last item, which therefore also waits for ST(c).
         const int last_h = G - 1;
         int st = 0, sc = 0, pv = 0, qn = 0;
+        // V of chunk c is ready as loaded, except in a ragged chunk, whose
+        // tail rows the phi warps zero first (only the block's last chunk
+        // can be ragged, so its v_xf barrier completes exactly one phase)
+        auto v_ready = [&](int c) {
+          const int vs = c % K::NKV;
+          return n - c * kChunk < kChunk ? mbar_test(&bars.v_xf[vs], 0)
+                                         : mbar_test(&bars.v_full[vs], (c / K::NKV) & 1);
+        };
         uint32_t idle = 0;
         uint64_t idle_t0 = 0;
         while (qn < n_items && ok) {
@@ -372,14 +394,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++qn;
             did = true;
           } else if (st < nc && st * G <= sc &&
-                     mbar_test(&bars.kv_xf[st % K::NKV], (st / K::NKV) & 1) &&
+                     mbar_test(&bars.k_xf[st % K::NKV], (st / K::NKV) & 1) && v_ready(st) &&
                      mbar_test(bars.s_empty, st & 1)) {
             tc_fence_after();
             issue_state(st, st > 0 || has_carry);
             umma_commit(bars.s_full);
+            // K is released by whichever of ST(c) and the chunk's last score comes last
+            if (sc > st * G + last_h) umma_commit(&bars.k_empty[st % K::NKV]);
             ++st;
             did = true;
-          } else if (pv < sc && (pv % G != last_h || st > pv / G) &&
+          } else if (pv < sc && (pv % G != last_h || st > pv / G) && v_ready(pv / G) &&
                      mbar_test(&bars.pb_full[pv % K::NP], (pv / K::NP) & 1) &&
                      mbar_test(&bars.acc_empty[pv % K::NA], ((pv / K::NA) & 1) ^ 1)) {
             tc_fence_after();
@@ -395,11 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_f16_ts(t_acc + DV, t_pb + kk * 8, smem_desc_sw128(sONESa + (kk & 3) * 32, 16, 1024),
                           ID_P1, kk > 0 ? 1u : 0u);
             }
-            if (pv % G == last_h) umma_commit(&bars.kv_empty[c % K::NKV]);
+            if (pv % G == last_h) umma_commit(&bars.v_empty[c % K::NKV]);
             ++pv;
             did = true;
           } else if (sc < n_items && pv > sc - K::NP &&
-                     mbar_test(&bars.kv_xf[(sc / G) % K::NKV], ((sc / G) / K::NKV) & 1) &&
+                     mbar_test(&bars.k_xf[(sc / G) % K::NKV], ((sc / G) / K::NKV) & 1) &&
                      mbar_test(&bars.q_xf[sc % K::NQ], (sc / K::NQ) & 1)) {
             tc_fence_after();
             const int c = sc / G, qs = sc % K::NQ, ps = sc % K::NP;
@@ -411,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           smem_desc_sw128(kb + o, 16, 1024), ID_P, kk > 0 ? 1u : 0u);
             }
             umma_commit(&bars.p_full[ps]);
+            if (sc % G == last_h && st > c) umma_commit(&bars.k_empty[c % K::NKV]);
             ++sc;
             did = true;
           }
@@ -432,11 +457,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!carried_state) {
           for (int c = 0; c < nc && ok; ++c) {
             const int st = c % K::NKV;
-            ok = mbar_wait(&bars.kv_xf[st], (c / K::NKV) & 1, abort_flag, a.err, kWaitLimitNs);
+            const uint32_t par = (c / K::NKV) & 1;
+            ok = mbar_wait(&bars.k_xf[st], par, abort_flag, a.err, kWaitLimitNs) &&
+                 (n - c * kChunk < kChunk
+                      ? mbar_wait(&bars.v_xf[st], 0, abort_flag, a.err, kWaitLimitNs)
+                      : mbar_wait(&bars.v_full[st], par, abort_flag, a.err, kWaitLimitNs));
             if (!ok) break;
             tc_fence_after();
             issue_state(c, c > 0);
-            umma_commit(&bars.kv_empty[st]);
+            umma_commit(&bars.k_empty[st]);
+            umma_commit(&bars.v_empty[st]);
           }
           if (ok) umma_commit(bars.s_full);
         }
@@ -462,19 +492,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------ phi warpgroup
     const int x = tid;  // 0..127
     bool ok = true;
+    // phi(K_c) in place (tail rows zeroed); in a ragged chunk also the V
+    // tail rows zeroed, signalled separately
     auto xf_kv = [&](int c) -> bool {
       const int st = c % K::NKV;
-      if (!mbar_wait(&bars.kv_full[st], (c / K::NKV) & 1, abort_flag, a.err, kWaitLimitNs))
-        return false;
+      const uint32_t par = (c / K::NKV) & 1;
+      if (!mbar_wait(&bars.k_full[st], par, abort_flag, a.err, kWaitLimitNs)) return false;
       const int valid = min(kChunk, n - c * kChunk);
       if (valid >= kChunk)
         phi_tile_loop<D / 64>(sK + st * K::KT, x);
       else
         xf_tile<D / 64, 128>(sK + st * K::KT, valid, true, x);
-      prep_tile<DV / 64, 128>(sV + st * K::VT, valid, false, x);
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
-      if (x == 0) mbar_arrive(&bars.kv_xf[st]);
+      if (x == 0) mbar_arrive(&bars.k_xf[st]);
+      if (valid < kChunk) {
+        if (!mbar_wait(&bars.v_full[st], par, abort_flag, a.err, kWaitLimitNs)) return false;
+        xf_tile<DV / 64, 128>(sV + st * K::VT, valid, false, x);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (x == 0) mbar_arrive(&bars.v_xf[st]);
+      }
       return true;
     };
     // rows past the end of the sequence only reach their own (unstored) outputs
