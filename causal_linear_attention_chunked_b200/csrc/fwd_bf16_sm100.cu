@@ -527,9 +527,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
     if (a.causal) {
+      // A chunk's first Q tile is prefetched while the previous chunk still
+      // holds the K stage, so it goes first.  (Q(i) waits only for Q S of
+      // item i - NQ, an item of an earlier chunk: no cycle through phi(K_c).)
       for (int i = 0; i < n_items && ok; ++i) {
-        if (i % G == 0) ok = xf_kv(i / G);
-        if (ok) ok = xf_q(i);
+        ok = xf_q(i);
+        if (ok && i % G == 0) ok = xf_kv(i / G);
       }
     } else {
       if (!carried_state)
