@@ -353,3 +353,63 @@ def test_general_kernel_block_counts(monkeypatch, nb, case):
     got = run_dense(q, k, v, causal)
     ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
     assert row_rel_err(got, ref) <= TOL_BF16
+
+
+# A ragged last chunk loads the next packed sequence's (or the next batch
+# row's) first rows into its tiles, and the kernels zero those rows before any
+# product.  Here that neighbour holds NaN and Inf: every other sequence must
+# still match the oracle on clean data, with no non-finite output.  Covers the
+# one-launch kernel (dense d = dv = 64, three one-chunk blocks), the block
+# kernel (packed d = dv = 64), the general kernel (d = dv = 128, packed and
+# blocked) and the state launch (dense d = 128, non-causal aggregates).
+ISOLATION_CASES = [
+    # (layout, lengths, Hq, Hkv, d, dv, causal); dense layout: B = 2, N = lengths
+    ("packed", [130, 200, 77], 4, 2, 64, 64, True),
+    ("packed", [130, 200, 77], 4, 2, 64, 64, False),
+    ("packed", [130, 200, 77], 4, 2, 128, 128, True),
+    ("packed", [130, 200, 77], 4, 2, 128, 128, False),
+    ("dense", 300, 4, 2, 64, 64, True),
+    ("dense", 300, 4, 2, 64, 64, False),
+    ("dense", 300, 4, 2, 128, 128, True),
+    ("dense", 300, 4, 2, 128, 128, False),
+]
+
+
+def _poison(t, rows):
+    """q -> NaN, k -> +Inf, v -> NaN on the given token rows (first axis after
+    flattening the batch)."""
+    t = t.clone()
+    t.view(-1, *t.shape[-2:])[rows] = float("nan")
+    return t
+
+
+@pytest.mark.parametrize("case", ISOLATION_CASES, ids=lambda c: "%s_d%d_%s" % (
+    c[0], c[4], "c" if c[6] else "nc"))
+def test_nonfinite_neighbour_is_isolated(case):
+    layout, lens, Hq, Hkv, d, dv, causal = case
+    L = lt()
+    if layout == "packed":
+        w = inputs.Workload("t", len(lens), Hq, Hkv, 0, d, dv, torch.bfloat16, d ** -0.5, causal,
+                            sum(lens))
+        q, k, v, cu = inputs.make(w, lengths=lens)
+        bad = torch.arange(lens[0], lens[0] + lens[1])  # the middle sequence
+        keep = torch.cat([torch.arange(0, lens[0]), torch.arange(lens[0] + lens[1], sum(lens))])
+        cu_dev = cu.cuda()
+    else:
+        q, k, v = inputs.make_custom(2, Hq, Hkv, lens, d, dv, torch.bfloat16, d ** -0.5, seed=31)
+        bad = torch.arange(lens, 2 * lens)  # batch row 1, flattened tokens
+        keep = torch.arange(0, lens)
+        cu, cu_dev = None, None
+    ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6,
+                               cu_seqlens=None if cu is None else cu.numpy())
+    qp = _poison(q, bad)
+    kp = k.clone()
+    kp.view(-1, *k.shape[-2:])[bad] = float("inf")
+    vp = _poison(v, bad)
+    out = L.linear_attn_fwd(qp.cuda(), kp.cuda(), vp.cuda(), causal=causal, eps=1e-6,
+                            cu_seqlens=cu_dev)
+    torch.cuda.synchronize()
+    assert L.get_last_device_error() == 0
+    got = out.float().cpu().numpy().reshape(-1, Hq, dv)[keep.numpy()]
+    ref = np.asarray(ref).reshape(-1, Hq, dv)[keep.numpy()]
+    assert row_rel_err(got, ref) <= TOL_BF16
