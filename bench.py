@@ -66,22 +66,29 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def source_digest():
+FORWARD_SOURCES = (
+    "causal_linear_attention_chunked_b200/csrc/state_bf16_sm100.cu",
+    "causal_linear_attention_chunked_b200/csrc/fwd_bf16_block_sm100.cu",
+    "causal_linear_attention_chunked_b200/csrc/fwd_bf16_fused_sm100.cu",
+    "causal_linear_attention_chunked_b200/csrc/fwd_bf16_sm100.cu",
+    "causal_linear_attention_chunked_b200/csrc/fwd_common.cuh",
+    "causal_linear_attention_chunked_b200/csrc/lt_ptx.cuh")
+
+
+def source_digest(files=FORWARD_SOURCES):
     h = hashlib.sha256()
-    for rel in ("causal_linear_attention_chunked_b200/csrc/state_bf16_sm100.cu",
-                "causal_linear_attention_chunked_b200/csrc/fwd_bf16_block_sm100.cu",
-                "causal_linear_attention_chunked_b200/csrc/fwd_bf16_fused_sm100.cu",
-                "causal_linear_attention_chunked_b200/csrc/fwd_bf16_sm100.cu",
-                "causal_linear_attention_chunked_b200/csrc/fwd_common.cuh",
-                "causal_linear_attention_chunked_b200/csrc/lt_ptx.cuh"):
+    for rel in files:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def committed_traffic(workload):
+def committed_traffic(workload, kernel_label=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
+    on the current source of the kernel it names (else None).  The summary
+    lists the files its digest covers (`source_files`, default: every forward
+    source) and the kernel it measured (`kernel`), which must be the kernel
+    this run timed."""
     path = os.path.join(ROOT, "profiles", "traffic_lt_fwd_bf16_%s.txt" % workload)
     try:
         kv = {}
@@ -89,7 +96,10 @@ def committed_traffic(workload):
             if "=" in line and not line.startswith("#"):
                 a, b = line.split("=", 1)
                 kv[a.strip()] = b.strip()
-        if kv.get("source_digest") != source_digest():
+        files = kv["source_files"].split() if "source_files" in kv else FORWARD_SOURCES
+        if kv.get("source_digest") != source_digest(files):
+            return None
+        if "kernel" in kv and (kernel_label is None or kv["kernel"] not in kernel_label):
             return None
         return float(kv["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
@@ -399,7 +409,6 @@ def run_lt(args):
     value = whole_job_rate(units, world, ms_step)
     peak, peak_kind = peaks()
     achieved = nbytes / (ms_step * 1e-3) / 1e9
-    traffic = committed_traffic(w.name)
     packed = w.packed_len is not None
     nblk, per_step, ws_bytes = L.linear_attn_fwd_plan(w.B, w.Hq, w.Hkv, 1 if packed else w.N,
                                                       w.d, w.dv, causal=w.causal, packed=packed)
@@ -410,6 +419,7 @@ def run_lt(args):
         kern = "lt_fused_fwd_kernel (one cooperative launch)"
     else:
         kern = "lt_block_fwd_kernel" if d64 else "lt_fwd_bf16_kernel"
+    traffic = committed_traffic(w.name, kern)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
