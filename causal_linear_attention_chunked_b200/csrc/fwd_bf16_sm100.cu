@@ -21,9 +21,10 @@
 // served from the same K/V tiles and the same state.  With more than one
 // block per sequence the state of a block starts from the carry summed from
 // the block aggregates of the state launch (earlier blocks when causal,
-// every block when not), written into the TMEM state accumulator.  Warp roles (480 threads):
+// every block when not), written into the TMEM state accumulator.
+// Warp roles (480 threads):
 //   warps 0-3   phi warpgroup: phi applied in place to the TMA-loaded K and
-//               Q tiles, tail rows zeroed.
+//               Q tiles; rows past a ragged end of K, and of V, zeroed.
 //   warps 4-7   mask warpgroup: causal mask of the score tile and
 //               conversion to bf16, in place in TMEM, where P V reads it as
 //               its A operand.
