@@ -39,11 +39,13 @@ def _load():
                                                       ip, i32p, ip]
         lib.lt_oracle_decode_step.argtypes = [vp, vp, vp, ip, dp, dp, dp, ip, ip, ip, ip, ip,
                                               ctypes.c_double]
+        lib.lt_oracle_fwd_state.argtypes = fwd_args + [dp, dp, dp, dp]
         lib.lt_oracle_phi.argtypes = [ctypes.c_double]
         lib.lt_oracle_phi.restype = ctypes.c_double
         lib.lt_oracle_num_threads.restype = ctypes.c_int
         for name in ("lt_oracle_fwd_quadratic", "lt_oracle_fwd_recurrent", "lt_oracle_fwd_rows",
-                     "lt_oracle_noncausal_numerator", "lt_oracle_decode_step"):
+                     "lt_oracle_noncausal_numerator", "lt_oracle_decode_step",
+                     "lt_oracle_fwd_state"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -136,6 +138,27 @@ def fwd_quadratic(q, k, v, causal=True, eps=1e-6, cu_seqlens=None):
 def fwd_recurrent(q, k, v, causal=True, eps=1e-6, cu_seqlens=None):
     """Recurrent (RNN) form over the fixed-size state (S, z)."""
     return _fwd(_load().lt_oracle_fwd_recurrent, q, k, v, causal, eps, cu_seqlens)
+
+
+def fwd_state(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, S0=None, z0=None):
+    """Recurrent form continued from the state (S0, z0) (zero if None);
+    returns (out, S, z) with the state after each sequence's last token.
+    States are per (sequence, KV head): S [B][Hkv][d][dv], z [B][Hkv][d]."""
+    (rq, rk, rv), t = _same_type(q, k, v)
+    B, Hq, Hkv, N, d, dv, oshape = _geometry(rq, rk, rv, cu_seqlens)
+    out = np.zeros(oshape, dtype=np.float64)
+    S = np.zeros((B, Hkv, d, dv), dtype=np.float64)
+    z = np.zeros((B, Hkv, d), dtype=np.float64)
+    s0 = None if S0 is None else np.ascontiguousarray(np.asarray(S0, dtype=np.float64).reshape(S.shape))
+    z0_ = None if z0 is None else np.ascontiguousarray(np.asarray(z0, dtype=np.float64).reshape(z.shape))
+    cu, cup = _cu(cu_seqlens)
+    rc = _load().lt_oracle_fwd_state(
+        _ptr(rq), _ptr(rk), _ptr(rv), t, _dptr(out), B, Hq, Hkv, N, d, dv, int(bool(causal)),
+        float(eps), cup, None if s0 is None else _dptr(s0), None if z0_ is None else _dptr(z0_),
+        _dptr(S), _dptr(z))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out, S, z
 
 
 def fwd_rows(q, k, v, rows, causal=True, eps=1e-6, cu_seqlens=None):

@@ -149,15 +149,22 @@ int lt_oracle_fwd_quadratic(const void *q, const void *k, const void *v, int in_
 
 /*
  * Form 2: the recurrence over the fixed-size state (the RNN view).
- *     S <- 0 (d x dv), z <- 0 (d)
+ *     S <- S0 (d x dv), z <- z0 (d)          (zero unless a state is given)
  *     for i = 0..n-1:  S += phi(K_i)^T V_i;  z += phi(K_i);
  *                      O_i = phi(Q_i) S / (phi(Q_i) . z + eps)
  * Non-causal: run the state update over the whole sequence first, then
  * evaluate every O_i with the final (S, z).
+ * With S0/z0 the sequence continues from that state: the "RNN view" of the
+ * "Reference" section and the KV-cache reuse of "Features" (the cache is
+ * the state), so splitting a sequence and carrying (S, z) across the split
+ * reproduces the unsplit output.  S0, S_out: [B][Hkv][d][dv]; z0, z_out:
+ * [B][Hkv][d] (one state per sequence and KV head); any may be NULL.
+ * S_out/z_out receive the state after the sequence's last token.
  */
-int lt_oracle_fwd_recurrent(const void *q, const void *k, const void *v, int in_type,
-                            double *out, int B, int Hq, int Hkv, int N, int d, int dv,
-                            int causal, double eps, const int32_t *cu_seqlens) {
+static int recurrent_impl(const void *q, const void *k, const void *v, int in_type,
+                          double *out, int B, int Hq, int Hkv, int N, int d, int dv,
+                          int causal, double eps, const int32_t *cu_seqlens,
+                          const double *S0, const double *z0, double *S_out, double *z_out) {
     if (check_args(B, Hq, Hkv, N, d, dv, eps)) return 1;
     const int G = Hq / Hkv;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
@@ -171,6 +178,9 @@ int lt_oracle_fwd_recurrent(const void *q, const void *k, const void *v, int in_
             double *pq = malloc(sizeof(double) * d);
             double *pk = malloc(sizeof(double) * d);
             double *vv = malloc(sizeof(double) * dv);
+            const int64_t sg = (int64_t)s * Hkv + g;  /* this (sequence, KV head) state */
+            if (S0) memcpy(S, S0 + sg * d * dv, sizeof(double) * d * dv);
+            if (z0) memcpy(z, z0 + sg * d, sizeof(double) * d);
             if (!causal) {
                 for (int64_t i = 0; i < n; ++i) {
                     for (int c = 0; c < d; ++c) pk[c] = lt_oracle_phi(load_elem(k, off(t0 + i, g, Hkv, d, c), in_type));
@@ -199,6 +209,10 @@ int lt_oracle_fwd_recurrent(const void *q, const void *k, const void *v, int in_
                     out[off(t0 + i, h, Hq, dv, c)] = num / den;
                 }
             }
+            if (h % G == 0) {  /* one query head per group writes the group's state */
+                if (S_out) memcpy(S_out + sg * d * dv, S, sizeof(double) * d * dv);
+                if (z_out) memcpy(z_out + sg * d, z, sizeof(double) * d);
+            }
             free(S);
             free(z);
             free(pq);
@@ -207,6 +221,23 @@ int lt_oracle_fwd_recurrent(const void *q, const void *k, const void *v, int in_
         }
     }
     return 0;
+}
+
+int lt_oracle_fwd_recurrent(const void *q, const void *k, const void *v, int in_type,
+                            double *out, int B, int Hq, int Hkv, int N, int d, int dv,
+                            int causal, double eps, const int32_t *cu_seqlens) {
+    return recurrent_impl(q, k, v, in_type, out, B, Hq, Hkv, N, d, dv, causal, eps, cu_seqlens,
+                          NULL, NULL, NULL, NULL);
+}
+
+/* The forward pass continued from a given state and returning the final
+ * state (either may be NULL): form 2 with S0/z0 and S_out/z_out. */
+int lt_oracle_fwd_state(const void *q, const void *k, const void *v, int in_type,
+                        double *out, int B, int Hq, int Hkv, int N, int d, int dv,
+                        int causal, double eps, const int32_t *cu_seqlens,
+                        const double *S0, const double *z0, double *S_out, double *z_out) {
+    return recurrent_impl(q, k, v, in_type, out, B, Hq, Hkv, N, d, dv, causal, eps, cu_seqlens,
+                          S0, z0, S_out, z_out);
 }
 
 /*

@@ -248,6 +248,77 @@ def pin_value_scaling_and_key_permutation():
     assert np.abs(o - op).max() <= 1e-12 * np.abs(o).max()
 
 
+def pin_state_split_continuation():
+    """Cutting causal sequences at any point and continuing the second part
+    from the first part's final state reproduces the unsplit output (the
+    quadratic form) row by row, dense and packed, with GQA; the continued
+    run ends in the unsplit run's final state."""
+    B, N, Hq, Hkv, d, dv = 2, 23, 4, 2, 5, 6
+    q = _rand((B, N, Hq, d), 41)
+    k = _rand((B, N, Hkv, d), 42)
+    v = _rand((B, N, Hkv, dv), 43)
+    ref = oracle.fwd_quadratic(q, k, v, causal=True, eps=1e-6)
+    _, S_all, z_all = oracle.fwd_state(q, k, v, causal=True, eps=1e-6)
+    for n1 in (1, 9, 22):
+        o1, S1, z1 = oracle.fwd_state(q[:, :n1], k[:, :n1], v[:, :n1], causal=True, eps=1e-6)
+        o2, S2, z2 = oracle.fwd_state(q[:, n1:], k[:, n1:], v[:, n1:], causal=True, eps=1e-6,
+                                      S0=S1, z0=z1)
+        got = np.concatenate([o1, o2], axis=1)
+        assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+        assert np.abs(S2 - S_all).max() <= 1e-12 * np.abs(S_all).max()
+        assert np.abs(z2 - z_all).max() <= 1e-12 * np.abs(z_all).max()
+    # packed: sequence b of the second call continues sequence b of the first
+    lens1, lens2 = [4, 0, 7], [5, 3, 0]
+    g = np.random.default_rng(44)
+    n_all = [a + b for a, b in zip(lens1, lens2)]
+    qs = [g.standard_normal((n, Hq, d)) for n in n_all]
+    ks = [g.standard_normal((n, Hkv, d)) for n in n_all]
+    vs = [g.standard_normal((n, Hkv, dv)) for n in n_all]
+    cu1 = np.cumsum([0] + lens1).astype(np.int32)
+    cu2 = np.cumsum([0] + lens2).astype(np.int32)
+    part = lambda xs, lo, hi: np.concatenate([x[l:h] for x, l, h in zip(xs, lo, hi)])
+    hi1 = lens1
+    o1, S1, z1 = oracle.fwd_state(part(qs, [0] * 3, hi1), part(ks, [0] * 3, hi1),
+                                  part(vs, [0] * 3, hi1), causal=True, eps=1e-6, cu_seqlens=cu1)
+    o2, _, _ = oracle.fwd_state(part(qs, hi1, n_all), part(ks, hi1, n_all), part(vs, hi1, n_all),
+                                causal=True, eps=1e-6, cu_seqlens=cu2, S0=S1, z0=z1)
+    for b in range(3):
+        r = oracle.fwd_quadratic(qs[b][None], ks[b][None], vs[b][None], causal=True, eps=1e-6)[0]
+        got = np.concatenate([o1[cu1[b]:cu1[b + 1]], o2[cu2[b]:cu2[b + 1]]])
+        assert np.abs(got - r).max() <= 1e-12 * max(1.0, np.abs(r).max())
+
+
+def pin_state_final_equals_decode_chain():
+    """The final state of a forward pass from a given state equals the state
+    that as many decode steps from that state reach (prefill -> decode)."""
+    B, N, Hq, Hkv, d, dv = 2, 9, 4, 2, 5, 3
+    q = _rand((B, N, Hq, d), 45)
+    k = _rand((B, N, Hkv, d), 46)
+    v = _rand((B, N, Hkv, dv), 47)
+    S0 = np.abs(_rand((B, Hkv, d, dv), 48))
+    z0 = np.abs(_rand((B, Hkv, d), 49))
+    _, S_f, z_f = oracle.fwd_state(q, k, v, causal=True, eps=1e-6, S0=S0, z0=z0)
+    S, z = S0.copy(), z0.copy()
+    for t in range(N):
+        oracle.decode_step(np.ascontiguousarray(q[:, t]), np.ascontiguousarray(k[:, t]),
+                           np.ascontiguousarray(v[:, t]), S, z, eps=1e-6)
+    assert np.abs(S_f - S).max() <= 1e-12 * np.abs(S).max()
+    assert np.abs(z_f - z).max() <= 1e-12 * np.abs(z).max()
+
+
+def pin_state_noncausal_prefix():
+    """Non-causal from the state of a prefix p equals non-causal attention of
+    the rows of x over the keys of p and x together (quadratic form)."""
+    B, Hq, Hkv, d, dv = 1, 4, 2, 4, 5
+    p = [_rand((B, 6, H, w), 50 + i) for i, (H, w) in enumerate(((Hq, d), (Hkv, d), (Hkv, dv)))]
+    x = [_rand((B, 8, H, w), 60 + i) for i, (H, w) in enumerate(((Hq, d), (Hkv, d), (Hkv, dv)))]
+    _, Sp, zp = oracle.fwd_state(*p, causal=True, eps=1e-6)
+    got, _, _ = oracle.fwd_state(*x, causal=False, eps=1e-6, S0=Sp, z0=zp)
+    cat = [np.concatenate([a, b], axis=1) for a, b in zip(p, x)]
+    ref = oracle.fwd_quadratic(*cat, causal=False, eps=1e-6)[:, 6:]
+    assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
 ALL_PINS = [
     pin_phi_is_elu_plus_one,
     pin_hand_2x2,
@@ -262,4 +333,7 @@ ALL_PINS = [
     pin_packed_equals_independent,
     pin_decode_chain_equals_causal,
     pin_value_scaling_and_key_permutation,
+    pin_state_split_continuation,
+    pin_state_final_equals_decode_chain,
+    pin_state_noncausal_prefix,
 ]

@@ -27,6 +27,10 @@ MUTANTS = [
     ("decode reads state before update", "zg[a] += pk;", "zg[a] += 0.0 * pk;"),
     ("numerator sums V of the query row", "num[c] += a * load_elem(v, off(t0 + j,",
      "num[c] += a * load_elem(v, off(t0 + i,"),
+    ("initial state ignored", "if (S0) memcpy(", "if (0) memcpy("),
+    ("initial normaliser ignored", "if (z0) memcpy(", "if (0) memcpy("),
+    ("state indexed by query head", "const int64_t sg = (int64_t)s * Hkv + g;",
+     "const int64_t sg = (int64_t)s * Hkv + h % Hkv;"),
 ]
 
 
