@@ -19,8 +19,8 @@ LT_F32, LT_BF16 = 0, 1
 
 # every entry point declared in include/lt_linear_attn.h
 EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_fwd_noalloc", "lt_linear_attn_fwd_plan",
-            "lt_linear_attn_decode_step", "lt_status_string", "lt_get_last_device_error",
-            "lt_abi_version")
+            "lt_linear_attn_fwd_state", "lt_linear_attn_decode_step", "lt_status_string",
+            "lt_get_last_device_error", "lt_abi_version")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("liblt.so is not built (run `python -m "
@@ -38,6 +38,9 @@ lib.lt_linear_attn_fwd_plan.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                         ctypes.POINTER(_i), ctypes.POINTER(_i),
                                         ctypes.POINTER(ctypes.c_size_t)]
 lib.lt_linear_attn_fwd_plan.restype = _i
+lib.lt_linear_attn_fwd_state.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp,
+                                         _vp, _vp, _vp, _vp, _vp, _i]
+lib.lt_linear_attn_fwd_state.restype = _i
 lib.lt_linear_attn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f,
                                            _vp, _i]
 lib.lt_linear_attn_decode_step.restype = _i
@@ -104,6 +107,43 @@ def linear_attn_fwd(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, out=None, s
                                   int(bool(causal)), float(eps), _ptr(cu_seqlens),
                                   _stream_handle(stream, q.device), _dtype_code(q.dtype)))
     return out
+
+
+def linear_attn_fwd_state(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, S0=None, z0=None,
+                          return_state=True, out=None, stream=None):
+    """linear_attn_fwd continued from the state (S0, z0) (None: zero) and,
+    with return_state, also returning the final state: (out, S, z), states
+    fp32 [sequences, H_kv, d, dv] and [sequences, H_kv, d] (the layout of
+    linear_attn_decode_step).  See lt_linear_attn_fwd_state in
+    include/lt_linear_attn.h."""
+    if cu_seqlens is None:
+        B, N, Hq, d = q.shape
+        Hkv, dv = k.shape[2], v.shape[3]
+        oshape = (B, N, Hq, dv)
+    else:
+        N, Hq, d = q.shape
+        Hkv, dv = k.shape[1], v.shape[2]
+        B = cu_seqlens.numel() - 1
+        oshape = (N, Hq, dv)
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
+            raise TypeError("cu_seqlens must be a contiguous int32 tensor")
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+    for t in (S0, z0):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+            raise TypeError("S0 and z0 must be contiguous float32 tensors")
+    if out is None:
+        out = torch.empty(oshape, dtype=q.dtype, device=q.device)
+    S = z = None
+    if return_state:
+        S = torch.empty((B, Hkv, d, dv), dtype=torch.float32, device=q.device)
+        z = torch.empty((B, Hkv, d), dtype=torch.float32, device=q.device)
+    _check(lib.lt_linear_attn_fwd_state(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, Hq, Hkv, N, d,
+                                        dv, int(bool(causal)), float(eps), _ptr(cu_seqlens),
+                                        _ptr(S0), _ptr(z0), _ptr(S), _ptr(z),
+                                        _stream_handle(stream, q.device), _dtype_code(q.dtype)))
+    return (out, S, z) if return_state else out
 
 
 def linear_attn_fwd_plan(B, H_q, H_kv, N, d, dv, causal=True, packed=False,

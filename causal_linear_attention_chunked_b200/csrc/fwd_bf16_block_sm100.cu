@@ -39,6 +39,7 @@
 
 #include "fwd_common.cuh"
 #include "lt_internal.h"
+#include "lt_state.h"
 #include "lt_ptx.cuh"
 
 namespace lt {
@@ -57,6 +58,7 @@ struct BlockArgs {
   __nv_bfloat16* out;
   const int32_t* cu_seqlens;
   float* ws;        // block aggregates [lane][nb][E], or nullptr
+  int carry_pre;    // 1: slot b of ws already holds block b's carry (every block reads it)
   int Hq, Hkv, N, G, causal;
   int nb;           // blocks per sequence (lane)
   int bc;           // chunks per block
@@ -243,11 +245,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (non-causal), summed in fp32 in block order by warps 0-15 (the loads of
   // several blocks in flight at once) into the state operand buffer and the
   // z slot, which the state warps read after named barrier 4
-  const int nprev = (!kCarry || a.ws == nullptr) ? 0 : (causal ? blk : a.nb);
+  // (with a precomputed carry, slot blk alone)
+  const int nprev =
+      (!kCarry || a.ws == nullptr) ? 0 : (a.carry_pre ? 1 : (causal ? blk : a.nb));
   float* carry_s = reinterpret_cast<float*>(smem + OFF_SOP);
   float* carry_z = reinterpret_cast<float*>(smem + OFF_Z);
   if (kCarry && nprev > 0 && warp < 16) {
-    sum_aggregates<512>(reinterpret_cast<const float4*>(a.ws) + (size_t)(s * a.Hkv + g) * a.nb * (E / 4),
+    sum_aggregates<512>(reinterpret_cast<const float4*>(a.ws) +
+                            ((size_t)(s * a.Hkv + g) * a.nb + (a.carry_pre ? blk : 0)) * (E / 4),
                         nprev, carry_s, carry_z, tid);
     named_bar_sync(4, 512);
   }
@@ -665,8 +670,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool block_supported(const FwdLaunch& p) { return p.d == 64 && p.dv == 64; }
 
-cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, const float* ws,
-                                  cudaStream_t stream) {
+namespace {
+cudaError_t launch_block(const FwdLaunch& p, int nb, const float* ws, bool carry_pre,
+                         cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
   if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
       !make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64) ||
@@ -675,7 +681,8 @@ cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, const float* ws,
   BlockArgs a;
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
   a.cu_seqlens = p.cu_seqlens;
-  a.ws = nb > 1 ? const_cast<float*>(ws) : nullptr;
+  a.ws = (nb > 1 || carry_pre) ? const_cast<float*>(ws) : nullptr;
+  a.carry_pre = carry_pre ? 1 : 0;
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
   a.N = p.N;
@@ -686,11 +693,22 @@ cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, const float* ws,
   a.eps = p.eps;
   a.total_tokens = (int)p.total_tokens;
   a.err = p.err;
-  auto fk = (nb > 1 && ws != nullptr) ? lt_block_fwd_kernel<true> : lt_block_fwd_kernel<false>;
+  auto fk = a.ws != nullptr ? lt_block_fwd_kernel<true> : lt_block_fwd_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
   fk<<<dim3(nb, p.Hkv, p.B), kThreads, SMEM, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_fwd_bf16_block(const FwdLaunch& p, int nb, const float* ws,
+                                  cudaStream_t stream) {
+  return launch_block(p, nb, ws, false, stream);
+}
+
+cudaError_t launch_fwd_bf16_block_pre(const FwdLaunch& p, int nb, const float* ws,
+                                      cudaStream_t stream) {
+  return launch_block(p, nb, ws, true, stream);
 }
 
 }  // namespace lt

@@ -48,6 +48,7 @@
 #include <stdlib.h>
 
 #include "lt_internal.h"
+#include "lt_state.h"
 #include "lt_ptx.cuh"
 #include "fwd_common.cuh"
 
@@ -56,6 +57,12 @@ namespace {
 
 constexpr int kThreads = 480;
 using namespace fwd;
+
+// carry_pre: slot b of the workspace already holds block b's carry (the
+// forward pass continued from a given state), which every block reads
+struct GenArgs : FwdArgs {
+  int carry_pre;
+};
 
 // phi in place over a full [kChunk x (NBOX*64)] bf16 tile by 128 threads, as
 // a loop with four 16-byte pieces in flight per thread (compact code: this
@@ -156,7 +163,7 @@ template <int D, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     lt_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+                       const __grid_constant__ CUtensorMap tm_v, const GenArgs a) {
   using K = Cfg<D, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -198,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int G = a.G;
   // has_carry: the state starts from the block aggregates rather than zero;
   // carried_state: non-causal and the whole state comes from them
-  const bool has_carry = a.ws != nullptr && (!a.causal || blk > 0);
+  const bool has_carry = a.ws != nullptr && (a.carry_pre || !a.causal || blk > 0);
   const bool carried_state = a.ws != nullptr && !a.causal;
   const int n_items = nc * G;
 
@@ -619,8 +626,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t w[kStream ? 8 : (DV + 16) / 2];
       const uint32_t t_s = tmem + K::TM_S + lane_base;
       constexpr int E = D * DV + D;
-      const float* base = a.ws != nullptr ? a.ws + (size_t)(s * a.Hkv + g) * a.nb * E : nullptr;
-      const int nsum = src == kFromCarry ? (a.causal ? blk : a.nb) : 0;
+      const float* base =
+          a.ws != nullptr ? a.ws + ((size_t)(s * a.Hkv + g) * a.nb + (a.carry_pre ? blk : 0)) * E
+                          : nullptr;
+      const int nsum = src == kFromCarry ? (a.carry_pre ? 1 : (a.causal ? blk : a.nb)) : 0;
       // streamed: a loop (the first staging runs cold, while every CTA's
       // first tiles are in flight, and straight-line code would miss the
       // instruction cache line after line); held: unrolled, w stays in
@@ -807,7 +816,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, int DV>
-cudaError_t launch_fwd(const FwdLaunch& p, int nb, const float* ws, cudaStream_t stream) {
+cudaError_t launch_fwd(const FwdLaunch& p, int nb, const float* ws, bool carry_pre,
+                       cudaStream_t stream) {
   using K = Cfg<D, DV>;
   CUtensorMap tq, tk, tv;
   if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
@@ -817,10 +827,11 @@ cudaError_t launch_fwd(const FwdLaunch& p, int nb, const float* ws, cudaStream_t
   auto kern = lt_fwd_bf16_kernel<D, DV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
   if (e != cudaSuccess) return e;
-  FwdArgs a;
+  GenArgs a;
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
   a.cu_seqlens = p.cu_seqlens;
-  a.ws = nb > 1 ? ws : nullptr;
+  a.ws = (nb > 1 || carry_pre) ? ws : nullptr;
+  a.carry_pre = carry_pre ? 1 : 0;
   a.nb = nb;
   a.bc = block_chunks(p, nb);
   a.B = p.B;
@@ -839,13 +850,23 @@ cudaError_t launch_fwd(const FwdLaunch& p, int nb, const float* ws, cudaStream_t
 
 }  // namespace
 
+static cudaError_t launch_seq(const FwdLaunch& p, int nb, const float* ws, bool pre,
+                              cudaStream_t stream) {
+  if (p.d == 64 && p.dv == 64) return launch_fwd<64, 64>(p, nb, ws, pre, stream);
+  if (p.d == 128 && p.dv == 128) return launch_fwd<128, 128>(p, nb, ws, pre, stream);
+  if (p.d == 64 && p.dv == 128) return launch_fwd<64, 128>(p, nb, ws, pre, stream);
+  if (p.d == 128 && p.dv == 64) return launch_fwd<128, 64>(p, nb, ws, pre, stream);
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_fwd_bf16_seq(const FwdLaunch& p, int nb, const float* ws,
                                 cudaStream_t stream) {
-  if (p.d == 64 && p.dv == 64) return launch_fwd<64, 64>(p, nb, ws, stream);
-  if (p.d == 128 && p.dv == 128) return launch_fwd<128, 128>(p, nb, ws, stream);
-  if (p.d == 64 && p.dv == 128) return launch_fwd<64, 128>(p, nb, ws, stream);
-  if (p.d == 128 && p.dv == 64) return launch_fwd<128, 64>(p, nb, ws, stream);
-  return cudaErrorInvalidValue;
+  return launch_seq(p, nb, ws, false, stream);
+}
+
+cudaError_t launch_fwd_bf16_seq_pre(const FwdLaunch& p, int nb, const float* ws,
+                                    cudaStream_t stream) {
+  return launch_seq(p, nb, ws, true, stream);
 }
 
 // LT_KERNEL selects a forward kernel for every shape it supports (ablations):

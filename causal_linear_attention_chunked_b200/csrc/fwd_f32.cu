@@ -14,6 +14,7 @@
 #include <stdint.h>
 
 #include "lt_internal.h"
+#include "lt_state.h"
 #include "lt_ptx.cuh"
 
 namespace lt {
@@ -34,6 +35,12 @@ struct F32Args {
   float eps;
   int total_tokens;
   int* err;
+  // optional: initial state (else zero) and final state, per (sequence, KV
+  // head): S [.][Hkv][D][DV], z [.][Hkv][D]
+  const float* s0;
+  const float* z0;
+  float* s_out;
+  float* z_out;
 };
 
 template <int D, int DV>
@@ -64,9 +71,18 @@ __global__ void __launch_bounds__(kT) lt_fwd_f32_kernel(const F32Args a) {
     t0 = s * a.N;
     n = a.N;
   }
-  if (n <= 0) return;
-  for (int e = tid; e < D * DV; e += kT) S[e] = 0.0f;
-  for (int e = tid; e < D; e += kT) z[e] = 0.0f;
+  const size_t sg = (size_t)s * a.Hkv + g;  // this (sequence, KV head) state
+  // the CTA of the group's first query head writes the group's final state
+  const bool writes_state = a.s_out != nullptr && h % a.G == 0;
+  if (n <= 0) {
+    if (writes_state) {
+      for (int e = tid; e < D * DV; e += kT) a.s_out[sg * D * DV + e] = a.s0 ? a.s0[sg * D * DV + e] : 0.0f;
+      for (int e = tid; e < D; e += kT) a.z_out[sg * D + e] = a.z0 ? a.z0[sg * D + e] : 0.0f;
+    }
+    return;
+  }
+  for (int e = tid; e < D * DV; e += kT) S[e] = a.s0 ? a.s0[sg * D * DV + e] : 0.0f;
+  for (int e = tid; e < D; e += kT) z[e] = a.z0 ? a.z0[sg * D + e] : 0.0f;
   const int nc = (n + kC - 1) / kC;
 
   auto load_kv = [&](int c) {
@@ -157,10 +173,15 @@ __global__ void __launch_bounds__(kT) lt_fwd_f32_kernel(const F32Args a) {
       __syncthreads();
     }
   }
+  if (writes_state) {  // every state update is complete (barrier above)
+    for (int e = tid; e < D * DV; e += kT) a.s_out[sg * D * DV + e] = S[e];
+    for (int e = tid; e < D; e += kT) a.z_out[sg * D + e] = z[e];
+  }
 }
 
 template <int D, int DV>
-cudaError_t launch(const FwdLaunch& p, cudaStream_t stream) {
+cudaError_t launch(const FwdLaunch& p, const float* s0, const float* z0, float* s_out,
+                   float* z_out, cudaStream_t stream) {
   const int smem = (D * DV + D + 2 * kC * D + kC * DV + kC * kC + kC) * 4;
   auto kern = lt_fwd_f32_kernel<D, DV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -179,18 +200,27 @@ cudaError_t launch(const FwdLaunch& p, cudaStream_t stream) {
   a.eps = p.eps;
   a.total_tokens = (int)p.total_tokens;
   a.err = p.err;
+  a.s0 = s0;
+  a.z0 = z0;
+  a.s_out = s_out;
+  a.z_out = z_out;
   kern<<<dim3(p.Hq, p.B), kT, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_fwd_f32(const FwdLaunch& p, cudaStream_t stream) {
-  if (p.d == 64 && p.dv == 64) return launch<64, 64>(p, stream);
-  if (p.d == 128 && p.dv == 128) return launch<128, 128>(p, stream);
-  if (p.d == 64 && p.dv == 128) return launch<64, 128>(p, stream);
-  if (p.d == 128 && p.dv == 64) return launch<128, 64>(p, stream);
+cudaError_t launch_fwd_f32_state(const FwdLaunch& p, const float* s0, const float* z0,
+                                 float* s_out, float* z_out, cudaStream_t stream) {
+  if (p.d == 64 && p.dv == 64) return launch<64, 64>(p, s0, z0, s_out, z_out, stream);
+  if (p.d == 128 && p.dv == 128) return launch<128, 128>(p, s0, z0, s_out, z_out, stream);
+  if (p.d == 64 && p.dv == 128) return launch<64, 128>(p, s0, z0, s_out, z_out, stream);
+  if (p.d == 128 && p.dv == 64) return launch<128, 64>(p, s0, z0, s_out, z_out, stream);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fwd_f32(const FwdLaunch& p, cudaStream_t stream) {
+  return launch_fwd_f32_state(p, nullptr, nullptr, nullptr, nullptr, stream);
 }
 
 }  // namespace lt

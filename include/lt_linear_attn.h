@@ -25,6 +25,7 @@
  *     a stream-ordered workspace on `stream` (cudaMallocAsync, released by
  *     cudaFreeAsync on the same stream before the call returns) for the
  *     per-block partial states; lt_linear_attn_fwd_plan() gives its size.
+ *     lt_linear_attn_fwd_state with LT_BF16 allocates the same way (always).
  *     No other entry point allocates.
  *   - Layouts are token-major and dense (row-major, no padding):
  *       dense:   q [B][N][H_q][d],  k [B][N][H_kv][d],  v [B][N][H_kv][dv],
@@ -166,6 +167,47 @@ LT_API lt_status_t lt_linear_attn_fwd_plan(int B, int H_q, int H_kv, int N, int 
                                            int causal, int packed, lt_dtype_t dtype,
                                            int num_sms, int *blocks, int *launches,
                                            size_t *workspace_bytes);
+
+/*
+ * lt_linear_attn_fwd_state: the forward pass of lt_linear_attn_fwd continued
+ * from a given state and/or returning the final state (prefill -> decode
+ * handoff, a long sequence processed in pieces).  For linear attention the
+ * KV cache is the fixed-size state (lineartile page, "Features": KV-cache
+ * reuse; the recurrent view of the cited linear attention).
+ *
+ * With (S0, z0), sequence s starts from the state of its KV heads:
+ *     causal:     O_i = phi(Q_i)(S0 + S_i) / (phi(Q_i) . (z0 + z_i) + eps)
+ *     non-causal: the same with S_i, z_i summed over the whole sequence.
+ * (S_out, z_out) receive S0 + (the sum over the whole sequence): the state
+ * after the sequence's last token.  Cutting a sequence anywhere and passing
+ * the first call's (S_out, z_out) as the second call's (S0, z0) reproduces
+ * the uncut outputs; (S_out, z_out) can seed lt_linear_attn_decode_step.
+ *
+ * q .. cu_seqlens, stream, dtype   as for lt_linear_attn_fwd.
+ * S0     [B][H_kv][d][dv] fp32 device (16-byte aligned), or NULL: zero.
+ * z0     [B][H_kv][d] fp32 device, NULL exactly when S0 is.
+ * S_out  [B][H_kv][d][dv] fp32 device (16-byte aligned), or NULL: not returned.
+ * z_out  [B][H_kv][d] fp32 device, NULL exactly when S_out is.
+ *        B counts sequences (packed: the cu_seqlens entries minus one); an
+ *        empty sequence returns S0 (or zero).  S_out and z_out must not
+ *        overlap each other or any input (no in-place update); out must not
+ *        overlap S0 or z0.
+ * Scratch: LT_BF16 always allocates a stream-ordered workspace (every
+ * block's partial state, as lt_linear_attn_fwd; released before return).
+ * Evaluation (bf16): a state launch writes every block's partial state; a
+ * small kernel turns them, in block order, into each block's starting state
+ * S0 + (earlier blocks) and into the final state; the forward launch starts
+ * every block from its own.  With S0 = 0 the outputs equal lt_linear_attn_fwd's
+ * two-launch path bit for bit.
+ *
+ * Returns as lt_linear_attn_fwd.
+ */
+LT_API lt_status_t lt_linear_attn_fwd_state(const void *q, const void *k, const void *v,
+                                            void *out, int B, int H_q, int H_kv, int N, int d,
+                                            int dv, int causal, float eps,
+                                            const int32_t *cu_seqlens, const float *S0,
+                                            const float *z0, float *S_out, float *z_out,
+                                            lt_stream_t stream, lt_dtype_t dtype);
 
 /*
  * One recurrent decode step: the fixed-size state (S, z) plays the role of

@@ -89,6 +89,31 @@ def test_decode_rejects_invalid_arguments(case, expect):
     assert st == expect
 
 
+@pytest.mark.parametrize("case,expect", [
+    (dict(S0=FAKE), 1),             # S0 without z0
+    (dict(z0=FAKE), 1),             # z0 without S0
+    (dict(S_out=FAKE), 1),          # S_out without z_out
+    (dict(z_out=FAKE), 1),
+    (dict(q=None), 1),
+    (dict(B=0), 1),
+    (dict(Hkv=3, Hq=8), 1),
+    (dict(causal=2), 1),
+    (dict(eps=float("nan")), 1),
+    (dict(d=32), 2),
+    (dict(dtype=7), 2),
+])
+def test_fwd_state_rejects_invalid_arguments(case, expect):
+    from causal_linear_attention_chunked_b200 import _binding as b
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, B=1, Hq=8, Hkv=8, N=16, d=64, dv=64, causal=1,
+             eps=1e-6, cu=None, S0=None, z0=None, S_out=None, z_out=None, stream=None, dtype=1)
+    a.update(case)
+    st = b.lib.lt_linear_attn_fwd_state(a["q"], a["k"], a["v"], a["out"], a["B"], a["Hq"],
+                                        a["Hkv"], a["N"], a["d"], a["dv"], a["causal"], a["eps"],
+                                        a["cu"], a["S0"], a["z0"], a["S_out"], a["z_out"],
+                                        a["stream"], a["dtype"])
+    assert st == expect
+
+
 def test_oracle_and_library_share_no_code():
     """The oracle sources never include/import the CUDA path and vice versa."""
     osrc = open(os.path.join(ROOT, "oracle", "lt_oracle.c")).read()
