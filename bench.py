@@ -311,6 +311,42 @@ def measure_workload(L, w, K, W, stream, device, world, l2_bytes, rank=0):
     return units, ms_max / K, nbytes, R, window
 
 
+def measure_from_state(L, w, K, stream, device, l2_bytes, peak):
+    """The headline shape through lt_linear_attn_fwd_state: every pass starts
+    from a given state and returns the final state (prefill -> decode
+    handoff).  Bytes: Q, K, V, O plus the state read and written."""
+    total_tokens = w.B * w.N
+    state_bytes = w.B * w.Hkv * (w.d * w.dv + w.d) * 4
+    nbytes = algorithmic_bytes(w, total_tokens) + 2 * state_bytes
+    R = max(1, math.ceil(3 * l2_bytes / nbytes))
+    sets = make_sets(w, R, w.seed + 500, device)
+    g = inputs.generator(w.seed + 499)
+    S0 = torch.rand((w.B, w.Hkv, w.d, w.dv), generator=g).to(device)
+    z0 = torch.rand((w.B, w.Hkv, w.d), generator=g).to(device) + 1.0
+    S1 = torch.empty_like(S0)
+    z1 = torch.empty_like(z0)
+    fns = []
+    for (q, k, v, _, out) in sets:
+        def f(q=q, k=k, v=v, out=out):
+            L.linear_attn_fwd_state(q, k, v, causal=w.causal, eps=w.eps, S0=S0, z0=z0, out=out,
+                                    S_out=S1, z_out=z1, stream=stream)
+        fns.append(f)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            fns[i % R]()
+    torch.cuda.synchronize()
+    assert L.get_last_device_error(stream) == 0
+    ms, _, _ = timed_graph_steps(fns, K, stream, 1)
+    assert L.get_last_device_error(stream) == 0
+    ms /= K
+    ach = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": w.name + "_from_state", "tokens_per_s": total_tokens * w.Hq / (ms / 1e3),
+            "ms_per_step": ms, "achieved_gbs": ach, "roofline_frac": ach / peak,
+            "algorithmic_bytes": nbytes,
+            "note": "lt_linear_attn_fwd_state: given initial state, final state returned "
+                    "(state launch over every block, prefix kernel, forward launch)"}
+
+
 def measure_decode(L, stream, device, steps=1000, reps=3):
     c = inputs.DECODE
     B, Hq, Hkv, d, dv = c["B"], c["Hq"], c["Hkv"], c["d"], c["dv"]
@@ -458,6 +494,8 @@ def run_lt(args):
             extra.append({"workload": name, "tokens_per_s": u / (ms / 1e3), "ms_per_step": ms,
                           "achieved_gbs": ach, "roofline_frac": ach / peak,
                           "algorithmic_bytes": nb})
+        extra.append(measure_from_state(L, inputs.WORKLOADS[HEADLINE], args.extra_steps, stream,
+                                        device, l2, peak))
         extra.append(measure_decode(L, stream, device))
         line["extra"] = extra
     if rank == 0 and world == 1 and not args.profile:

@@ -110,12 +110,12 @@ def linear_attn_fwd(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, out=None, s
 
 
 def linear_attn_fwd_state(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, S0=None, z0=None,
-                          return_state=True, out=None, stream=None):
+                          return_state=True, out=None, S_out=None, z_out=None, stream=None):
     """linear_attn_fwd continued from the state (S0, z0) (None: zero) and,
     with return_state, also returning the final state: (out, S, z), states
     fp32 [sequences, H_kv, d, dv] and [sequences, H_kv, d] (the layout of
-    linear_attn_decode_step).  See lt_linear_attn_fwd_state in
-    include/lt_linear_attn.h."""
+    linear_attn_decode_step), written into S_out/z_out when given.  See
+    lt_linear_attn_fwd_state in include/lt_linear_attn.h."""
     if cu_seqlens is None:
         B, N, Hq, d = q.shape
         Hkv, dv = k.shape[2], v.shape[3]
@@ -137,8 +137,10 @@ def linear_attn_fwd_state(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, S0=No
         out = torch.empty(oshape, dtype=q.dtype, device=q.device)
     S = z = None
     if return_state:
-        S = torch.empty((B, Hkv, d, dv), dtype=torch.float32, device=q.device)
-        z = torch.empty((B, Hkv, d), dtype=torch.float32, device=q.device)
+        S = S_out if S_out is not None else torch.empty((B, Hkv, d, dv), dtype=torch.float32,
+                                                        device=q.device)
+        z = z_out if z_out is not None else torch.empty((B, Hkv, d), dtype=torch.float32,
+                                                        device=q.device)
     _check(lib.lt_linear_attn_fwd_state(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, Hq, Hkv, N, d,
                                         dv, int(bool(causal)), float(eps), _ptr(cu_seqlens),
                                         _ptr(S0), _ptr(z0), _ptr(S), _ptr(z),
