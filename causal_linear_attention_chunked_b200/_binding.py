@@ -20,7 +20,7 @@ LT_F32, LT_BF16 = 0, 1
 # every entry point declared in include/lt_linear_attn.h
 EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_fwd_noalloc", "lt_linear_attn_fwd_plan",
             "lt_linear_attn_fwd_state", "lt_linear_attn_decode_step", "lt_status_string",
-            "lt_get_last_device_error", "lt_abi_version")
+            "lt_get_last_device_error", "lt_abi_version", "lt_selftest_wait_timeout")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("liblt.so is not built (run `python -m "
@@ -49,6 +49,8 @@ lib.lt_status_string.restype = ctypes.c_char_p
 lib.lt_get_last_device_error.argtypes = [_vp]
 lib.lt_get_last_device_error.restype = _i
 lib.lt_abi_version.restype = _i
+lib.lt_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp]
+lib.lt_selftest_wait_timeout.restype = _i
 
 
 class LtError(RuntimeError):

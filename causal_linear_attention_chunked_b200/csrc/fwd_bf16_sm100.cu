@@ -48,6 +48,7 @@
 #include <stdlib.h>
 
 #include "lt_internal.h"
+#include "lt_fault.h"
 #include "lt_state.h"
 #include "lt_ptx.cuh"
 #include "fwd_common.cuh"
@@ -930,6 +931,7 @@ cudaError_t launch_fwd_bf16(const FwdLaunch& p, cudaStream_t stream) {
   plan_fwd_bf16(p, sms, &nb, &launches, &bytes);
   void* ws = nullptr;
   if (bytes) {
+    if (injected_workspace_alloc_failure()) return cudaErrorMemoryAllocation;
     cudaError_t e = cudaMallocAsync(&ws, bytes, stream);
     if (e != cudaSuccess) return e;
   }

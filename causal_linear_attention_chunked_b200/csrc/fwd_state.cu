@@ -23,6 +23,7 @@
 #include <stdint.h>
 
 #include "lt_internal.h"
+#include "lt_fault.h"
 #include "lt_state.h"
 
 namespace lt {
@@ -74,6 +75,7 @@ cudaError_t launch_fwd_state(const FwdLaunch& p, bool bf16, const float* s0, con
   const size_t E = (size_t)p.d * p.dv + p.d;
   const size_t bytes = (size_t)p.B * p.Hkv * nb * E * sizeof(float);
   void* ws = nullptr;
+  if (injected_workspace_alloc_failure()) return cudaErrorMemoryAllocation;
   cudaError_t e = cudaMallocAsync(&ws, bytes, stream);
   if (e != cudaSuccess) return e;
   float* w = static_cast<float*>(ws);

@@ -8,6 +8,7 @@
 
 #include "../../include/lt_linear_attn.h"
 #include "lt_internal.h"
+#include "lt_fault.h"
 #include "lt_state.h"
 #include "lt_ptx.cuh"
 
@@ -229,6 +230,15 @@ lt_status_t lt_linear_attn_fwd_state(const void* q, const void* k, const void* v
   p.err = err;
   const cudaError_t e =
       lt::launch_fwd_state(p, dtype == LT_BF16, S0, z0, S_out, z_out, (cudaStream_t)stream);
+  return e == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status_t lt_selftest_wait_timeout(unsigned int limit_us, lt_stream_t stream) {
+  if (limit_us == 0 || limit_us > 1000000u) return LT_ERR_INVALID_ARG;
+  int* err = device_error_word();
+  if (!err) return LT_ERR_CUDA;
+  const cudaError_t e =
+      lt::launch_selftest_wait(err, (uint64_t)limit_us * 1000u, (cudaStream_t)stream);
   return e == cudaSuccess ? LT_OK : LT_ERR_CUDA;
 }
 

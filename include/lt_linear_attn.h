@@ -229,6 +229,16 @@ LT_API lt_status_t lt_linear_attn_decode_step(const void *q, const void *k, cons
                                        float *z, void *out, int B, int H_q, int H_kv, int d,
                                        int dv, float eps, lt_stream_t stream, lt_dtype_t dtype);
 
+/*
+ * Diagnostic: enqueue one small kernel whose bounded wait (the pipeline
+ * wait every kernel uses) is on a barrier that nothing arrives on, so it
+ * gives up after limit_us microseconds (1 .. 1000000), records a timeout and
+ * returns.  lt_get_last_device_error(stream) then reports
+ * LT_ERR_DEVICE_TIMEOUT and the device stays usable.  It exists to test the
+ * timeout path without a GPU fault; the method has no counterpart.
+ */
+LT_API lt_status_t lt_selftest_wait_timeout(unsigned int limit_us, lt_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 LT_API const char *lt_status_string(lt_status_t status);
 

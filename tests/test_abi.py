@@ -114,6 +114,12 @@ def test_fwd_state_rejects_invalid_arguments(case, expect):
     assert st == expect
 
 
+def test_selftest_wait_rejects_invalid_limit():
+    from causal_linear_attention_chunked_b200 import _binding as b
+    assert b.lib.lt_selftest_wait_timeout(0, None) == 1
+    assert b.lib.lt_selftest_wait_timeout(2000000, None) == 1
+
+
 def test_oracle_and_library_share_no_code():
     """The oracle sources never include/import the CUDA path and vice versa."""
     osrc = open(os.path.join(ROOT, "oracle", "lt_oracle.c")).read()

@@ -49,3 +49,41 @@ def test_bad_cu_seqlens_reported_not_faulted():
     cu = torch.tensor([0, 60, 100, 140], dtype=torch.int32, device="cuda")  # beyond N
     L.linear_attn_fwd(q, q, q, cu_seqlens=cu, out=out)
     assert L.get_last_device_error() == b.LT_ERR_DEVICE_BAD_SEQLENS
+
+
+def test_injected_workspace_allocation_failure(monkeypatch):
+    """Host-side fault injection: the stream-ordered workspace allocation
+    reports failure; the call returns LT_ERR_CUDA with nothing enqueued or
+    written, and the next call (injection off) runs normally."""
+    from causal_linear_attention_chunked_b200 import _binding as b, inputs
+    L = b
+    q, k, v = inputs.make_custom(2, 8, 8, 1024, 64, 64, torch.bfloat16, 0.125, seed=3)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    assert L.linear_attn_fwd_plan(2, 8, 8, 1024, 64, 64)[2] > 0  # this shape needs a workspace
+    out = torch.full((2, 1024, 8, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    monkeypatch.setenv("LT_FAULT_WORKSPACE_ALLOC", "1")
+    for call in (lambda: L.linear_attn_fwd(q, k, v, out=out),
+                 lambda: L.linear_attn_fwd_state(q, k, v, out=out)):
+        with pytest.raises(L.LtError) as ei:
+            call()
+        assert ei.value.status == b.LT_ERR_CUDA
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all())
+    monkeypatch.delenv("LT_FAULT_WORKSPACE_ALLOC")
+    L.linear_attn_fwd(q, k, v, out=out)
+    assert L.get_last_device_error() == 0
+    assert bool(torch.isfinite(out.float()).all()) and not bool((out == 7.0).all())
+
+
+def test_stalled_wait_times_out_and_device_stays_usable():
+    """A bounded wait on a barrier nothing arrives on gives up after its
+    limit and reports LT_ERR_DEVICE_TIMEOUT; the error word is then clear and
+    the device runs a forward pass normally."""
+    from causal_linear_attention_chunked_b200 import _binding as b, inputs
+    assert b.lib.lt_selftest_wait_timeout(20000, None) == b.LT_OK  # 20 ms
+    assert b.get_last_device_error() == b.LT_ERR_DEVICE_TIMEOUT
+    assert b.get_last_device_error() == b.LT_OK
+    q, k, v = inputs.make_custom(1, 2, 2, 300, 64, 64, torch.bfloat16, 0.125, seed=4)
+    out = b.linear_attn_fwd(q.cuda(), k.cuda(), v.cuda())
+    assert b.get_last_device_error() == b.LT_OK
+    assert bool(torch.isfinite(out.float()).all())
