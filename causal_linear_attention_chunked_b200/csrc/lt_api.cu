@@ -53,6 +53,50 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 
 bool width_ok(int w) { return w == 64 || w == 128; }
 
+// The checks every forward entry point makes on its common arguments, in
+// order; on LT_OK, *tokens is the total token count and *p describes the call.
+lt_status_t check_fwd(const void* q, const void* k, const void* v, void* out, int B, int H_q,
+                      int H_kv, int N, int d, int dv, int causal, float eps,
+                      const int32_t* cu_seqlens, lt_dtype_t dtype, lt::FwdLaunch* p) {
+  if (dtype != LT_F32 && dtype != LT_BF16) return LT_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !out) return LT_ERR_INVALID_ARG;
+  if (B <= 0 || H_q <= 0 || H_kv <= 0 || N <= 0) return LT_ERR_INVALID_ARG;
+  if (H_q % H_kv != 0) return LT_ERR_INVALID_ARG;
+  if (B > 65535 || H_kv > 65535) return LT_ERR_INVALID_ARG;  // grid y/z extents
+  if (causal != 0 && causal != 1) return LT_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !isfinite(eps)) return LT_ERR_INVALID_ARG;
+  if (!width_ok(d) || !width_ok(dv)) return LT_ERR_UNSUPPORTED;
+  const long long tokens = cu_seqlens ? (long long)N : (long long)B * (long long)N;
+  if (tokens >= (1ll << 31)) return LT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return LT_ERR_INVALID_ARG;
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return LT_ERR_INVALID_ARG;
+  if (!is_device_ptr(q) || !is_device_ptr(k) || !is_device_ptr(v) || !is_device_ptr(out) ||
+      (cu_seqlens && !is_device_ptr(cu_seqlens)))
+    return LT_ERR_INVALID_ARG;
+  const size_t es = dtype == LT_BF16 ? 2 : 4;
+  const size_t nq = (size_t)tokens * H_q * d * es, nk = (size_t)tokens * H_kv * d * es;
+  const size_t nv = (size_t)tokens * H_kv * dv * es, no = (size_t)tokens * H_q * dv * es;
+  if (overlaps(out, no, q, nq) || overlaps(out, no, k, nk) || overlaps(out, no, v, nv))
+    return LT_ERR_INVALID_ARG;
+  *p = lt::FwdLaunch{};
+  p->q = q;
+  p->k = k;
+  p->v = v;
+  p->out = out;
+  p->cu_seqlens = cu_seqlens;
+  p->B = B;
+  p->Hq = H_q;
+  p->Hkv = H_kv;
+  p->N = N;
+  p->d = d;
+  p->dv = dv;
+  p->causal = causal;
+  p->eps = eps;
+  p->total_tokens = tokens;
+  return LT_OK;
+}
+
 }  // namespace
 
 namespace lt {
@@ -81,46 +125,12 @@ lt_status_t lt_linear_attn_fwd(const void* q, const void* k, const void* v, void
                                int H_q, int H_kv, int N, int d, int dv, int causal, float eps,
                                const int32_t* cu_seqlens, lt_stream_t stream,
                                lt_dtype_t dtype) {
-  if (dtype != LT_F32 && dtype != LT_BF16) return LT_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !out) return LT_ERR_INVALID_ARG;
-  if (B <= 0 || H_q <= 0 || H_kv <= 0 || N <= 0) return LT_ERR_INVALID_ARG;
-  if (H_q % H_kv != 0) return LT_ERR_INVALID_ARG;
-  if (B > 65535 || H_kv > 65535) return LT_ERR_INVALID_ARG;  // grid y/z extents
-  if (causal != 0 && causal != 1) return LT_ERR_INVALID_ARG;
-  if (!(eps >= 0.0f) || !isfinite(eps)) return LT_ERR_INVALID_ARG;
-  if (!width_ok(d) || !width_ok(dv)) return LT_ERR_UNSUPPORTED;
-  const long long tokens = cu_seqlens ? (long long)N : (long long)B * (long long)N;
-  if (tokens >= (1ll << 31)) return LT_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-    return LT_ERR_INVALID_ARG;
-  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return LT_ERR_INVALID_ARG;
-  if (!is_device_ptr(q) || !is_device_ptr(k) || !is_device_ptr(v) || !is_device_ptr(out) ||
-      (cu_seqlens && !is_device_ptr(cu_seqlens)))
-    return LT_ERR_INVALID_ARG;
-  const size_t es = dtype == LT_BF16 ? 2 : 4;
-  const size_t nq = (size_t)tokens * H_q * d * es, nk = (size_t)tokens * H_kv * d * es;
-  const size_t nv = (size_t)tokens * H_kv * dv * es, no = (size_t)tokens * H_q * dv * es;
-  if (overlaps(out, no, q, nq) || overlaps(out, no, k, nk) || overlaps(out, no, v, nv))
-    return LT_ERR_INVALID_ARG;
-  int* err = device_error_word();
-  if (!err) return LT_ERR_CUDA;
-
   lt::FwdLaunch p;
-  p.q = q;
-  p.k = k;
-  p.v = v;
-  p.out = out;
-  p.cu_seqlens = cu_seqlens;
-  p.B = B;
-  p.Hq = H_q;
-  p.Hkv = H_kv;
-  p.N = N;
-  p.d = d;
-  p.dv = dv;
-  p.causal = causal;
-  p.eps = eps;
-  p.total_tokens = tokens;
-  p.err = err;
+  const lt_status_t st =
+      check_fwd(q, k, v, out, B, H_q, H_kv, N, d, dv, causal, eps, cu_seqlens, dtype, &p);
+  if (st != LT_OK) return st;
+  p.err = device_error_word();
+  if (!p.err) return LT_ERR_CUDA;
   const cudaError_t e = dtype == LT_BF16 ? lt::launch_fwd_bf16(p, (cudaStream_t)stream)
                                          : lt::launch_fwd_f32(p, (cudaStream_t)stream);
   return e == cudaSuccess ? LT_OK : LT_ERR_CUDA;
@@ -171,35 +181,23 @@ lt_status_t lt_linear_attn_fwd_state(const void* q, const void* k, const void* v
                                      float eps, const int32_t* cu_seqlens, const float* S0,
                                      const float* z0, float* S_out, float* z_out,
                                      lt_stream_t stream, lt_dtype_t dtype) {
-  if (dtype != LT_F32 && dtype != LT_BF16) return LT_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !out) return LT_ERR_INVALID_ARG;
+  lt::FwdLaunch p;
+  const lt_status_t st =
+      check_fwd(q, k, v, out, B, H_q, H_kv, N, d, dv, causal, eps, cu_seqlens, dtype, &p);
+  if (st != LT_OK) return st;
   if ((S0 == nullptr) != (z0 == nullptr) || (S_out == nullptr) != (z_out == nullptr))
     return LT_ERR_INVALID_ARG;
-  if (B <= 0 || H_q <= 0 || H_kv <= 0 || N <= 0) return LT_ERR_INVALID_ARG;
-  if (H_q % H_kv != 0) return LT_ERR_INVALID_ARG;
-  if (B > 65535 || H_kv > 65535) return LT_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return LT_ERR_INVALID_ARG;
-  if (!(eps >= 0.0f) || !isfinite(eps)) return LT_ERR_INVALID_ARG;
-  if (!width_ok(d) || !width_ok(dv)) return LT_ERR_UNSUPPORTED;
-  const long long tokens = cu_seqlens ? (long long)N : (long long)B * (long long)N;
-  if (tokens >= (1ll << 31)) return LT_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-    return LT_ERR_INVALID_ARG;
-  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return LT_ERR_INVALID_ARG;
   if ((S0 && (!aligned16(S0) || (reinterpret_cast<uintptr_t>(z0) & 3u))) ||
       (S_out && (!aligned16(S_out) || (reinterpret_cast<uintptr_t>(z_out) & 3u))))
     return LT_ERR_INVALID_ARG;
-  if (!is_device_ptr(q) || !is_device_ptr(k) || !is_device_ptr(v) || !is_device_ptr(out) ||
-      (cu_seqlens && !is_device_ptr(cu_seqlens)) ||
-      (S0 && (!is_device_ptr(S0) || !is_device_ptr(z0))) ||
+  if ((S0 && (!is_device_ptr(S0) || !is_device_ptr(z0))) ||
       (S_out && (!is_device_ptr(S_out) || !is_device_ptr(z_out))))
     return LT_ERR_INVALID_ARG;
+  const long long tokens = p.total_tokens;
   const size_t es = dtype == LT_BF16 ? 2 : 4;
   const size_t nq = (size_t)tokens * H_q * d * es, nk = (size_t)tokens * H_kv * d * es;
   const size_t nv = (size_t)tokens * H_kv * dv * es, no = (size_t)tokens * H_q * dv * es;
   const size_t ns = (size_t)B * H_kv * d * dv * 4, nz = (size_t)B * H_kv * d * 4;
-  if (overlaps(out, no, q, nq) || overlaps(out, no, k, nk) || overlaps(out, no, v, nv))
-    return LT_ERR_INVALID_ARG;
   if (S0 && (overlaps(out, no, S0, ns) || overlaps(out, no, z0, nz))) return LT_ERR_INVALID_ARG;
   if (S_out) {
     // the final state is written while inputs may still be read: no overlap
@@ -210,24 +208,8 @@ lt_status_t lt_linear_attn_fwd_state(const void* q, const void* k, const void* v
         return LT_ERR_INVALID_ARG;
     if (overlaps(S_out, ns, z_out, nz)) return LT_ERR_INVALID_ARG;
   }
-  int* err = device_error_word();
-  if (!err) return LT_ERR_CUDA;
-  lt::FwdLaunch p = {};
-  p.q = q;
-  p.k = k;
-  p.v = v;
-  p.out = out;
-  p.cu_seqlens = cu_seqlens;
-  p.B = B;
-  p.Hq = H_q;
-  p.Hkv = H_kv;
-  p.N = N;
-  p.d = d;
-  p.dv = dv;
-  p.causal = causal;
-  p.eps = eps;
-  p.total_tokens = tokens;
-  p.err = err;
+  p.err = device_error_word();
+  if (!p.err) return LT_ERR_CUDA;
   const cudaError_t e =
       lt::launch_fwd_state(p, dtype == LT_BF16, S0, z0, S_out, z_out, (cudaStream_t)stream);
   return e == cudaSuccess ? LT_OK : LT_ERR_CUDA;
