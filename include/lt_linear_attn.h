@@ -116,7 +116,7 @@ LT_API lt_status_t lt_linear_attn_fwd(const void *q, const void *k, const void *
 /*
  * lt_linear_attn_fwd_noalloc: the bf16 forward pass of lt_linear_attn_fwd
  * (same arguments, dtype fixed to LT_BF16, same kernels and results) for
- * callers that cannot let a library allocate device memory.  The paper has
+ * callers that cannot let a library allocate device memory.  The method has
  * no counterpart; it exists for integration only.
  *
  * Who needs it: lt_linear_attn_fwd takes a stream-ordered workspace
