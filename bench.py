@@ -411,6 +411,43 @@ def measure_e2e(L, w, steps, stream, device):
                                     "buffers, copies + kernel on one stream)"}
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def measure_eager(L, w, stream, device, calls=200):
+    """Per-call cost of eager (not graph-captured) calls of the headline
+    shape: the host time to issue one call through the C ABI (argument
+    checks, plan, workspace, launch), and the device time per call when calls
+    are issued back to back without a graph."""
+    q, k, v, cu = inputs.make(w)
+    q, k, v = q.to(device), k.to(device), v.to(device)
+    out = torch.empty(q.shape[:-1] + (w.dv,), dtype=w.dtype, device=device)
+    for _ in range(5):
+        L.linear_attn_fwd(q, k, v, causal=w.causal, eps=w.eps, out=out, stream=stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        L.linear_attn_fwd(q, k, v, causal=w.causal, eps=w.eps, out=out, stream=stream)
+    t1 = time.perf_counter()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"workload": w.name + "_eager", "host_us_per_call": (t1 - t0) * 1e6 / calls,
+            "device_us_per_call": e0.elapsed_time(e1) * 1e3 / calls, "calls": calls,
+            "note": "eager calls through the Python binding and the C ABI, no CUDA graph; "
+                    "host time covers marshalling, argument checks, plan, workspace and launch"}
+
+
 def cpu_baseline(w, budget_s=10.0):
     import oracle  # the fp64 CPU oracle, as it stands (test infrastructure)
     q, k, v, _ = inputs.make(w)
@@ -422,7 +459,7 @@ def cpu_baseline(w, budget_s=10.0):
             break
     dt = time.time() - t0
     return {"value": reps * w.B * w.Hq * w.N / dt, "unit": "tokens/s",
-            "cores": oracle.num_threads(), "kind": "oracle",
+            "cores": oracle.num_threads(), "cpu_model": cpu_model(), "kind": "oracle",
             "sample": "%d full passes of %s (fp64 recurrent form, OpenMP over (sequence, head)) "
                       "in %.1f s" % (reps, w.name, dt)}
 
@@ -497,6 +534,7 @@ def run_lt(args):
         extra.append(measure_from_state(L, inputs.WORKLOADS[HEADLINE], args.extra_steps, stream,
                                         device, l2, peak))
         extra.append(measure_decode(L, stream, device))
+        extra.append(measure_eager(L, w, stream, device))
         line["extra"] = extra
     if rank == 0 and world == 1 and not args.profile:
         line["cpu_baseline"] = cpu_baseline(w)
@@ -543,7 +581,7 @@ def run_reference(args):
             "config": {"workload": w.name, "B": w.B, "H_q": w.Hq, "H_kv": w.Hkv, "N": w.N,
                        "d": w.d, "dv": w.dv, "causal": w.causal, "eps": w.eps},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
-                             "kind": "oracle", "sample": sample},
+                             "cpu_model": cpu_model(), "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

@@ -16,11 +16,14 @@ LIB_PATH = os.path.join(_HERE, "liblt.so")
 LT_OK, LT_ERR_INVALID_ARG, LT_ERR_UNSUPPORTED, LT_ERR_CUDA = 0, 1, 2, 3
 LT_ERR_DEVICE_TIMEOUT, LT_ERR_DEVICE_BAD_SEQLENS, LT_ERR_SCRATCH_TOO_SMALL = 4, 5, 6
 LT_F32, LT_BF16 = 0, 1
+LT_SCHED_AUTO, LT_SCHED_TWO_LAUNCH, LT_SCHED_GENERAL = 0, 1, 2
+_SCHED = {"auto": LT_SCHED_AUTO, "two_launch": LT_SCHED_TWO_LAUNCH, "general": LT_SCHED_GENERAL}
 
 # every entry point declared in include/lt_linear_attn.h
 EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_fwd_noalloc", "lt_linear_attn_fwd_plan",
             "lt_linear_attn_fwd_state", "lt_linear_attn_decode_step", "lt_status_string",
-            "lt_get_last_device_error", "lt_abi_version", "lt_selftest_wait_timeout")
+            "lt_get_last_device_error", "lt_abi_version", "lt_selftest_wait_timeout",
+            "lt_debug_set_schedule")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("liblt.so is not built (run `python -m "
@@ -51,6 +54,8 @@ lib.lt_get_last_device_error.restype = _i
 lib.lt_abi_version.restype = _i
 lib.lt_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp]
 lib.lt_selftest_wait_timeout.restype = _i
+lib.lt_debug_set_schedule.argtypes = [_i, _i]
+lib.lt_debug_set_schedule.restype = _i
 
 
 class LtError(RuntimeError):
@@ -179,6 +184,13 @@ def linear_attn_decode_step(q, k, v, S, z, eps=1e-6, out=None, stream=None):
                                           _stream_handle(stream, q.device),
                                           _dtype_code(q.dtype)))
     return out
+
+
+def set_schedule(kernel="auto", blocks=0):
+    """Diagnostic override of the forward schedule, process-wide (tests and
+    ablations): kernel "auto" | "two_launch" | "general", blocks 0 (the
+    library's choice) or a block count per dense sequence."""
+    _check(lib.lt_debug_set_schedule(_SCHED[kernel], int(blocks)))
 
 
 def get_last_device_error(stream=None):

@@ -6,6 +6,7 @@ Compiles every ``csrc/*.cu`` with nvcc for ``sm_100a`` and links one shared
 library with the C ABI of ``include/lt_linear_attn.h``.  The CUDA runtime is
 linked statically, so the library depends only on the driver.
 """
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -44,18 +45,24 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not (force or needs_build()):
         return LIB
     os.makedirs(OUT_DIR, exist_ok=True)
-    objs = []
-    for src in sources():
+
+    def compile_one(src):
         obj = os.path.join(OUT_DIR, os.path.basename(src) + ".o")
         cmd = [NVCC] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose else []) + \
             ["-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
-        if r.returncode != 0:
-            sys.stderr.write(r.stdout + r.stderr)
-            raise RuntimeError("nvcc failed on %s" % src)
-        if verbose:
-            sys.stderr.write(r.stdout + r.stderr)
-        objs.append(obj)
+        return src, obj, r
+
+    objs = []
+    workers = max(1, min(len(sources()), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as ex:
+        for src, obj, r in ex.map(compile_one, sources()):
+            if r.returncode != 0:
+                sys.stderr.write(r.stdout + r.stderr)
+                raise RuntimeError("nvcc failed on %s" % src)
+            if verbose:
+                sys.stderr.write(r.stdout + r.stderr)
+            objs.append(obj)
     tmp = LIB + ".tmp%d" % os.getpid()
     cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + objs + ["-cudart", "static"]
     r = subprocess.run(cmd, capture_output=True, text=True)

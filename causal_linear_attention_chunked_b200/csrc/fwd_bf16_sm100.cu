@@ -870,62 +870,39 @@ cudaError_t launch_fwd_bf16_seq_pre(const FwdLaunch& p, int nb, const float* ws,
   return launch_seq(p, nb, ws, true, stream);
 }
 
-// LT_KERNEL selects a forward kernel for every shape it supports (ablations):
-//   seq      the general kernel (one CTA per block of chunks) for d = dv = 64
-//            too; LT_BLOCKS=1 makes it fully sequential
-//   cluster  sequence split over a thread-block cluster (d = dv = 64)
-//   pair     the two-launch block scan (state launch, then forward launch)
-//            also where the one-launch cluster exchange applies
-static bool forced(char c) {
-  const char* force = getenv("LT_KERNEL");
-  return force && force[0] == c;
-}
-
+// The schedule override (lt_debug_set_schedule) can keep the two-launch
+// block scan where the one-launch path applies, or run the general kernel on
+// d = dv = 64 too (tests and ablations).
 static bool use_block_fused(const FwdLaunch& p, int nb, int num_sms) {
-  return !forced('s') && !forced('p') && block_fused_supported(p, nb, num_sms);
-}
-
-static int current_sms() {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return 0;
-  return sms;
+  return sched_kernel() == LT_SCHED_AUTO && block_fused_supported(p, nb, num_sms);
 }
 
 cudaError_t launch_fwd_bf16_ws(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream) {
-  if (use_block_fused(p, nb, current_sms())) return launch_fwd_bf16_block_fused(p, nb, ws, stream);
+  if (use_block_fused(p, nb, device_sm_count()))
+    return launch_fwd_bf16_block_fused(p, nb, ws, stream);
   cudaError_t e = cudaSuccess;
   if (nb > 1) {
     e = launch_block_state(p, nb, ws, stream);
     if (e != cudaSuccess) return e;
   }
-  if (!forced('s') && block_supported(p)) return launch_fwd_bf16_block(p, nb, ws, stream);
+  if (sched_kernel() != LT_SCHED_GENERAL && block_supported(p))
+    return launch_fwd_bf16_block(p, nb, ws, stream);
   return launch_fwd_bf16_seq(p, nb, ws, stream);
 }
 
 void plan_fwd_bf16(const FwdLaunch& p, int num_sms, int* nb, int* launches, size_t* ws_bytes) {
-  if (forced('c') && split_supported(p)) {
-    *nb = 1;
-    *launches = 1;
-    *ws_bytes = 0;
-    return;
-  }
   *nb = block_count(p, num_sms);
+  *ws_bytes = block_workspace_bytes(p, *nb);
   if (use_block_fused(p, *nb, num_sms)) {
     *launches = 1;
-    *ws_bytes = block_workspace_bytes(p, *nb);
     return;
   }
   *launches = *nb > 1 && (p.causal ? *nb - 1 : *nb) > 0 ? 2 : 1;
-  *ws_bytes = block_workspace_bytes(p, *nb);
 }
 
 cudaError_t launch_fwd_bf16(const FwdLaunch& p, cudaStream_t stream) {
-  if (forced('c') && split_supported(p)) return launch_fwd_bf16_split(p, stream);
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
   int nb = 1, launches = 1;
   size_t bytes = 0;
   plan_fwd_bf16(p, sms, &nb, &launches, &bytes);

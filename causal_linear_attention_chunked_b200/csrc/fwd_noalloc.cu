@@ -20,7 +20,6 @@
 // state (zeros for a block past the end of its sequence) before the forward
 // launch of the same call reads it.
 #include <cuda_runtime.h>
-#include <math.h>
 #include <stdint.h>
 
 #include <mutex>
@@ -60,22 +59,6 @@ cudaError_t scratch_address(float** addr) {
   return cudaSuccess;
 }
 
-bool on_device(const void* p) {
-  cudaPointerAttributes at;
-  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
-    cudaGetLastError();
-    return false;
-  }
-  return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-bool disjoint(const void* a, size_t na, const void* b, size_t nb) {
-  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-  return x >= y + nb || y >= x + na;
-}
-
 }  // namespace
 
 extern "C" {
@@ -84,52 +67,26 @@ lt_status_t lt_linear_attn_fwd_noalloc(const void* q, const void* k, const void*
                                        int B, int H_q, int H_kv, int N, int d, int dv,
                                        int causal, float eps, const int32_t* cu_seqlens,
                                        lt_stream_t stream) {
-  // sizes, widths and flags: the same rules as lt_linear_attn_fwd, and the
-  // block count and workspace size that call would use on this device
+  // the checks of lt_linear_attn_fwd, in the same order (so the same bad
+  // arguments give the same status), then the block count and workspace
+  // size that call would use on this device
+  lt::FwdLaunch p;
+  lt_status_t st = lt::check_fwd(q, k, v, out, B, H_q, H_kv, N, d, dv, causal, eps, cu_seqlens,
+                                 LT_BF16, &p);
+  if (st != LT_OK) return st;
   int nb = 1, launches = 1;
   size_t ws_bytes = 0;
-  const lt_status_t st = lt_linear_attn_fwd_plan(B, H_q, H_kv, N, d, dv, causal,
-                                                 cu_seqlens ? 1 : 0, LT_BF16, 0, &nb,
-                                                 &launches, &ws_bytes);
+  st = lt_linear_attn_fwd_plan(B, H_q, H_kv, N, d, dv, causal, cu_seqlens ? 1 : 0, LT_BF16, 0,
+                               &nb, &launches, &ws_bytes);
   if (st != LT_OK) return st;
-  if (!(eps >= 0.0f) || !isfinite(eps)) return LT_ERR_INVALID_ARG;
-  if (!q || !k || !v || !out) return LT_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-    return LT_ERR_INVALID_ARG;
-  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return LT_ERR_INVALID_ARG;
-  if (!on_device(q) || !on_device(k) || !on_device(v) || !on_device(out) ||
-      (cu_seqlens && !on_device(cu_seqlens)))
-    return LT_ERR_INVALID_ARG;
-  const long long tokens = cu_seqlens ? (long long)N : (long long)B * (long long)N;
-  const size_t nq = (size_t)tokens * H_q * d * 2, nk = (size_t)tokens * H_kv * d * 2;
-  const size_t nv = (size_t)tokens * H_kv * dv * 2, no = (size_t)tokens * H_q * dv * 2;
-  if (!disjoint(out, no, q, nq) || !disjoint(out, no, k, nk) || !disjoint(out, no, v, nv))
-    return LT_ERR_INVALID_ARG;
   if (ws_bytes > kScratchBytes) return LT_ERR_SCRATCH_TOO_SMALL;
-  int* err = lt::device_error_word_current();
-  if (!err) return LT_ERR_CUDA;
+  p.err = lt::device_error_word_current();
+  if (!p.err) return LT_ERR_CUDA;
   float* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) {
     cudaGetLastError();
     return LT_ERR_CUDA;
   }
-
-  lt::FwdLaunch p;
-  p.q = q;
-  p.k = k;
-  p.v = v;
-  p.out = out;
-  p.cu_seqlens = cu_seqlens;
-  p.B = B;
-  p.Hq = H_q;
-  p.Hkv = H_kv;
-  p.N = N;
-  p.d = d;
-  p.dv = dv;
-  p.causal = causal;
-  p.eps = eps;
-  p.total_tokens = tokens;
-  p.err = err;
   const cudaError_t e =
       lt::launch_fwd_bf16_ws(p, nb, ws_bytes ? scratch : nullptr, (cudaStream_t)stream);
   return e == cudaSuccess ? LT_OK : LT_ERR_CUDA;

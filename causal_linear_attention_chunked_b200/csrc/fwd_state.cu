@@ -68,9 +68,8 @@ __global__ void __launch_bounds__(kPrefixThreads)
 cudaError_t launch_fwd_state(const FwdLaunch& p, bool bf16, const float* s0, const float* z0,
                              float* s_out, float* z_out, cudaStream_t stream) {
   if (!bf16) return launch_fwd_f32_state(p, s0, z0, s_out, z_out, stream);
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
   const int nb = block_count(p, sms);  // 1 for packed sequences
   const size_t E = (size_t)p.d * p.dv + p.d;
   const size_t bytes = (size_t)p.B * p.Hkv * nb * E * sizeof(float);

@@ -4,6 +4,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/lt_linear_attn.h"
@@ -19,7 +20,12 @@ __device__ int g_device_error;
 
 constexpr int kMaxDevices = 64;
 int* g_err_ptr[kMaxDevices];
+int g_sm_count[kMaxDevices];
 std::mutex g_err_mu;
+
+// lt_debug_set_schedule's override (tests and ablations only)
+std::atomic<int> g_sched_kernel{LT_SCHED_AUTO};
+std::atomic<int> g_sched_blocks{0};
 
 // Device address of the error word on the current device (looked up once
 // per device).
@@ -54,8 +60,8 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 bool width_ok(int w) { return w == 64 || w == 128; }
 
 // The checks every forward entry point makes on its common arguments, in
-// order; on LT_OK, *tokens is the total token count and *p describes the call.
-lt_status_t check_fwd(const void* q, const void* k, const void* v, void* out, int B, int H_q,
+// order; on LT_OK, *p describes the call.
+lt_status_t check_fwd_impl(const void* q, const void* k, const void* v, void* out, int B, int H_q,
                       int H_kv, int N, int d, int dv, int causal, float eps,
                       const int32_t* cu_seqlens, lt_dtype_t dtype, lt::FwdLaunch* p) {
   if (dtype != LT_F32 && dtype != LT_BF16) return LT_ERR_UNSUPPORTED;
@@ -101,6 +107,33 @@ lt_status_t check_fwd(const void* q, const void* k, const void* v, void* out, in
 
 namespace lt {
 int* device_error_word_current() { return device_error_word(); }
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return 0;
+  }
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  if (g_sm_count[dev] <= 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    g_sm_count[dev] = sms;
+  }
+  return g_sm_count[dev];
+}
+
+int sched_kernel() { return g_sched_kernel.load(std::memory_order_relaxed); }
+int sched_blocks() { return g_sched_blocks.load(std::memory_order_relaxed); }
+
+lt_status_t check_fwd(const void* q, const void* k, const void* v, void* out, int B, int H_q,
+                      int H_kv, int N, int d, int dv, int causal, float eps,
+                      const int32_t* cu_seqlens, lt_dtype_t dtype, FwdLaunch* p) {
+  return check_fwd_impl(q, k, v, out, B, H_q, H_kv, N, d, dv, causal, eps, cu_seqlens, dtype, p);
+}
 }  // namespace lt
 
 extern "C" {
@@ -127,7 +160,7 @@ lt_status_t lt_linear_attn_fwd(const void* q, const void* k, const void* v, void
                                lt_dtype_t dtype) {
   lt::FwdLaunch p;
   const lt_status_t st =
-      check_fwd(q, k, v, out, B, H_q, H_kv, N, d, dv, causal, eps, cu_seqlens, dtype, &p);
+      check_fwd_impl(q, k, v, out, B, H_q, H_kv, N, d, dv, causal, eps, cu_seqlens, dtype, &p);
   if (st != LT_OK) return st;
   p.err = device_error_word();
   if (!p.err) return LT_ERR_CUDA;
@@ -155,12 +188,8 @@ lt_status_t lt_linear_attn_fwd_plan(int B, int H_q, int H_kv, int N, int d, int 
     return LT_OK;
   }
   if (num_sms <= 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-      cudaGetLastError();
-      return LT_ERR_CUDA;
-    }
+    num_sms = lt::device_sm_count();
+    if (num_sms <= 0) return LT_ERR_CUDA;
   }
   lt::FwdLaunch p = {};
   p.cu_seqlens = packed ? reinterpret_cast<const int32_t*>(16) : nullptr;  // only tested for null
@@ -183,7 +212,7 @@ lt_status_t lt_linear_attn_fwd_state(const void* q, const void* k, const void* v
                                      lt_stream_t stream, lt_dtype_t dtype) {
   lt::FwdLaunch p;
   const lt_status_t st =
-      check_fwd(q, k, v, out, B, H_q, H_kv, N, d, dv, causal, eps, cu_seqlens, dtype, &p);
+      check_fwd_impl(q, k, v, out, B, H_q, H_kv, N, d, dv, causal, eps, cu_seqlens, dtype, &p);
   if (st != LT_OK) return st;
   if ((S0 == nullptr) != (z0 == nullptr) || (S_out == nullptr) != (z_out == nullptr))
     return LT_ERR_INVALID_ARG;
@@ -213,6 +242,15 @@ lt_status_t lt_linear_attn_fwd_state(const void* q, const void* k, const void* v
   const cudaError_t e =
       lt::launch_fwd_state(p, dtype == LT_BF16, S0, z0, S_out, z_out, (cudaStream_t)stream);
   return e == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status_t lt_debug_set_schedule(lt_schedule_t kernel, int blocks) {
+  if (kernel != LT_SCHED_AUTO && kernel != LT_SCHED_TWO_LAUNCH && kernel != LT_SCHED_GENERAL)
+    return LT_ERR_INVALID_ARG;
+  if (blocks < 0) return LT_ERR_INVALID_ARG;
+  g_sched_kernel.store((int)kernel, std::memory_order_relaxed);
+  g_sched_blocks.store(blocks, std::memory_order_relaxed);
+  return LT_OK;
 }
 
 lt_status_t lt_selftest_wait_timeout(unsigned int limit_us, lt_stream_t stream) {

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/lt_linear_attn.h"
+
 namespace lt {
 
 struct FwdLaunch {
@@ -39,10 +41,6 @@ void plan_fwd_bf16(const FwdLaunch& p, int num_sms, int* nb, int* launches, size
 // the same with a caller-provided workspace of at least
 // block_workspace_bytes(p, nb) bytes (nullptr when that is 0)
 cudaError_t launch_fwd_bf16_ws(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream);
-// d = dv = 64: sequence split over a thread-block cluster (or one CTA per
-// (sequence, KV head) for packed inputs)
-bool split_supported(const FwdLaunch& p);
-cudaError_t launch_fwd_bf16_split(const FwdLaunch& p, cudaStream_t stream);
 // Block-parallel scan.  A dense sequence is cut into nb blocks of
 // block_chunks(p, nb) chunks; the state launch writes each block's aggregate
 // phi(K)^T [V | 1] (fp32, d x dv then d) to the workspace and the forward
@@ -68,6 +66,17 @@ cudaError_t launch_fwd_bf16_block_fused(const FwdLaunch& p, int nb, float* ws,
                                         cudaStream_t stream);
 // the per-device error word of the current device (looked up once per device)
 int* device_error_word_current();
+// SM count of the current device (queried once per device); 0 on failure
+int device_sm_count();
+// the schedule override of lt_debug_set_schedule (LT_SCHED_AUTO and 0 unless
+// a test or an ablation set them)
+int sched_kernel();
+int sched_blocks();
+// the argument checks every forward entry point makes, in order; on LT_OK
+// *p describes the call (its err field still unset)
+lt_status_t check_fwd(const void* q, const void* k, const void* v, void* out, int B, int H_q,
+                      int H_kv, int N, int d, int dv, int causal, float eps,
+                      const int32_t* cu_seqlens, lt_dtype_t dtype, FwdLaunch* p);
 cudaError_t launch_fwd_f32(const FwdLaunch& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeLaunch& p, cudaStream_t stream);
 

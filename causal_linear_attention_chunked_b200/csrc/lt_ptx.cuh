@@ -11,6 +11,13 @@
 #include <stdint.h>
 
 #include <cooperative_groups.h>
+#include <cuda_runtime_api.h>  // CUDART_VERSION
+
+// grid_barrier (below) uses the barrier word of the cooperative-groups grid
+// workspace and its arrive protocol as the CUDA 12.8 / 12.9 headers define
+// them; another toolkit may change either, so it must be re-checked there.
+static_assert(CUDART_VERSION >= 12080 && CUDART_VERSION < 12100,
+              "grid_barrier follows the cooperative-groups grid workspace of CUDA 12.8-12.9");
 
 namespace lt {
 

@@ -246,15 +246,12 @@ cudaError_t launch(const FwdLaunch& p, int nb, int nblocks_launch, float* ws,
 
 // Blocks per sequence: enough CTAs to cover the SMs about once.  Packed
 // sequences keep one block each (the sequences themselves give the
-// parallelism).  LT_BLOCKS overrides (ablations).
+// parallelism).  lt_debug_set_schedule can force a count (tests, ablations).
 int block_count(const FwdLaunch& p, int num_sms) {
   if (p.cu_seqlens) return 1;
   const int nc = (p.N + kChunk - 1) / kChunk;
-  const char* force = getenv("LT_BLOCKS");
-  if (force) {
-    const int f = atoi(force);
-    return f < 1 ? 1 : (f > nc ? nc : f);
-  }
+  const int f = sched_blocks();
+  if (f > 0) return f > nc ? nc : f;
   const int lanes = p.B * p.Hkv;
   int nb = num_sms / (lanes > 0 ? lanes : 1);
   if (nb < 1) nb = 1;

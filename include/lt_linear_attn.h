@@ -103,8 +103,12 @@ typedef enum {
  * dense products and the inter-chunk part through the carried state
  * ("Why Stream Wins at Ultra-Long Context", section 5.3: chunk-local work
  * plus a carry).  A dense sequence is cut into blocks of consecutive chunks
- * so that every SM has work: one launch writes each block's partial state
- * to the workspace, a second runs the blocks from the carry.
+ * so that every SM has work, and each block starts from the sum of the
+ * earlier blocks' partial states.  Short blocks (d = dv = 64, at most four
+ * chunks, every block resident at once) run as ONE cooperative launch whose
+ * blocks exchange their partial states through the workspace; otherwise one
+ * launch writes each block's partial state and a second runs the blocks
+ * from the carry.  lt_linear_attn_fwd_plan tells which.
  *
  * Returns LT_OK when the work was enqueued.
  */
@@ -228,6 +232,30 @@ LT_API lt_status_t lt_linear_attn_fwd_state(const void *q, const void *k, const 
 LT_API lt_status_t lt_linear_attn_decode_step(const void *q, const void *k, const void *v, float *S,
                                        float *z, void *out, int B, int H_q, int H_kv, int d,
                                        int dv, float eps, lt_stream_t stream, lt_dtype_t dtype);
+
+/*
+ * Diagnostic schedule override, for tests and ablations only: makes every
+ * later forward call of this process (every device, every thread) use a
+ * given kernel path and/or block count instead of the one the library picks.
+ * Results stay correct on every path; only the speed changes.  Not meant to
+ * be changed while forward calls run on other threads.
+ *
+ * kernel  LT_SCHED_AUTO: the library's choice (the default);
+ *         LT_SCHED_TWO_LAUNCH: the state launch plus the forward launch
+ *           also where one cooperative launch would run;
+ *         LT_SCHED_GENERAL: the general kernel (every width pair) also for
+ *           d = dv = 64.
+ * blocks  0: the library's choice; n > 0: n blocks per dense sequence (at
+ *         most its chunk count).
+ * Returns LT_OK, or LT_ERR_INVALID_ARG for an unknown kernel or blocks < 0.
+ * The method has no counterpart.
+ */
+typedef enum {
+  LT_SCHED_AUTO = 0,
+  LT_SCHED_TWO_LAUNCH = 1,
+  LT_SCHED_GENERAL = 2
+} lt_schedule_t;
+LT_API lt_status_t lt_debug_set_schedule(lt_schedule_t kernel, int blocks);
 
 /*
  * Diagnostic: enqueue one small kernel whose bounded wait (the pipeline

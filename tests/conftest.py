@@ -34,3 +34,24 @@ def cuda_available():
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture
+def sched():
+    """Set the library's diagnostic schedule override for one test:
+    ``sched(kernel=..., blocks=...)`` updates the given fields (kernel
+    "auto" | "two_launch" | "general"; blocks 0 = the library's choice); the
+    override is reset to the library's choice when the test ends."""
+    from causal_linear_attention_chunked_b200 import _binding as b
+    state = {"kernel": "auto", "blocks": 0}
+
+    def set_(kernel=None, blocks=None):
+        if kernel is not None:
+            state["kernel"] = kernel
+        if blocks is not None:
+            state["blocks"] = blocks
+        b.set_schedule(state["kernel"], state["blocks"])
+
+    set_()
+    yield set_
+    b.set_schedule("auto", 0)

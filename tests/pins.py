@@ -64,6 +64,10 @@ def pin_hand_2x2():
     rows = np.array([[0, 0, 0], [0, 1, 0]])
     got = oracle.fwd_rows(q, k, v, rows, causal=True, eps=0.0)
     assert np.allclose(got, g["causal_eps0"], rtol=0, atol=1e-15)
+    got = oracle.fwd_rows(q, k, v, rows, causal=False, eps=0.0)
+    assert np.allclose(got, g["noncausal_eps0"], rtol=0, atol=1e-15), got
+    got = oracle.fwd_rows(q, k, v, rows, causal=True, eps=1e-6)
+    assert np.allclose(got, g["causal_eps1e-6"], rtol=0, atol=1e-15), got
 
 
 def hand_3tok_inputs(d=64, dv=64, dtype=torch.float32):
@@ -218,6 +222,42 @@ def pin_packed_equals_independent():
                 assert np.abs(packed[a:b] - dense).max() <= 1e-12 * max(1.0, np.abs(dense).max())
 
 
+def pin_rows_equal_quadratic_packed_gqa():
+    """Selected rows (the full-size checker) equal the same rows of the
+    quadratic form, itself pinned above, on packed GQA sequences (an empty
+    one among them) and on a dense batch, causal and non-causal: every
+    sequence, the first and last position of each, and random heads."""
+    lens = [9, 0, 1, 17, 6]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T, Hq, Hkv, d, dv = int(cu[-1]), 6, 2, 5, 4
+    q = _rand((T, Hq, d), 70)
+    k = _rand((T, Hkv, d), 71)
+    v = _rand((T, Hkv, dv), 72)
+    g = np.random.default_rng(73)
+    rows = []
+    for s, n in enumerate(lens):
+        for i in sorted({0, n - 1, n // 2} if n else ()):
+            for h in (0, Hq - 1, int(g.integers(0, Hq))):
+                rows.append((s, i, h))
+    rows = np.array(rows, dtype=np.int64)
+    for causal in (True, False):
+        full = oracle.fwd_quadratic(q, k, v, causal=causal, eps=1e-6, cu_seqlens=cu)
+        want = np.stack([full[cu[s] + i, h] for s, i, h in rows])
+        got = oracle.fwd_rows(q, k, v, rows, causal=causal, eps=1e-6, cu_seqlens=cu)
+        assert np.abs(got - want).max() <= 1e-12 * np.abs(want).max(), causal
+    B, N = 2, 13
+    qd = _rand((B, N, Hq, d), 74)
+    kd = _rand((B, N, Hkv, d), 75)
+    vd = _rand((B, N, Hkv, dv), 76)
+    rows = np.array([(b, i, h) for b in range(B) for i in (0, 6, N - 1) for h in (1, Hq - 2)],
+                    dtype=np.int64)
+    for causal in (True, False):
+        full = oracle.fwd_quadratic(qd, kd, vd, causal=causal, eps=1e-6)
+        want = np.stack([full[b, i, h] for b, i, h in rows])
+        got = oracle.fwd_rows(qd, kd, vd, rows, causal=causal, eps=1e-6)
+        assert np.abs(got - want).max() <= 1e-12 * np.abs(want).max(), causal
+
+
 def pin_decode_chain_equals_causal():
     """N decode steps from a zero state reproduce the causal forward row by row."""
     B, N, Hq, Hkv, d, dv = 3, 11, 4, 2, 5, 6
@@ -331,6 +371,7 @@ ALL_PINS = [
     pin_convex_hull,
     pin_gqa_equals_replication,
     pin_packed_equals_independent,
+    pin_rows_equal_quadratic_packed_gqa,
     pin_decode_chain_equals_causal,
     pin_value_scaling_and_key_permutation,
     pin_state_split_continuation,

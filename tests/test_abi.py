@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 def test_abi_version_and_status_strings():
     from causal_linear_attention_chunked_b200 import _binding as b
     assert b.lib.lt_abi_version() == 1
-    for code in range(6):
+    for code in range(7):
         assert b.lib.lt_status_string(code).startswith(b"LT_")
     assert b.lib.lt_status_string(99) == b"unknown lt_status_t"
 
@@ -68,6 +68,42 @@ def test_fwd_rejects_invalid_arguments(case, expect):
                                   a["N"], a["d"], a["dv"], a["causal"], a["eps"], a["cu"],
                                   a["stream"], a["dtype"])
     assert st == expect
+
+
+@pytest.mark.parametrize("case", [
+    dict(q=None), dict(q=None, d=32), dict(B=0), dict(Hkv=3, Hq=8), dict(N=0), dict(causal=2),
+    dict(eps=-1.0), dict(eps=float("nan")), dict(d=32), dict(dv=96), dict(d=32, eps=-1.0),
+    dict(B=70000), dict(B=1 << 16, N=1 << 16), dict(Hkv=70000, Hq=70000),
+])
+def test_noalloc_returns_the_same_status_as_fwd(case):
+    """The no-allocation entry point makes lt_linear_attn_fwd's checks in the
+    same order, so the same bad arguments give the same status code."""
+    from causal_linear_attention_chunked_b200 import _binding as b
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, B=1, Hq=8, Hkv=8, N=16, d=64, dv=64, causal=1,
+             eps=1e-6)
+    a.update(case)
+    args = (a["q"], a["k"], a["v"], a["out"], a["B"], a["Hq"], a["Hkv"], a["N"], a["d"],
+            a["dv"], a["causal"], a["eps"], None, None)
+    st_fwd = b.lib.lt_linear_attn_fwd(*args, 1)
+    st_na = b.lib.lt_linear_attn_fwd_noalloc(*args)
+    assert st_fwd != 0 and st_na == st_fwd, (st_fwd, st_na)
+
+
+def test_schedule_override_validates_and_resets():
+    from causal_linear_attention_chunked_b200 import _binding as b
+    assert b.lib.lt_debug_set_schedule(3, 0) == 1
+    assert b.lib.lt_debug_set_schedule(0, -1) == 1
+    nb, nl, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    try:
+        assert b.lib.lt_debug_set_schedule(b.LT_SCHED_TWO_LAUNCH, 3) == 0
+        assert b.lib.lt_linear_attn_fwd_plan(2, 8, 8, 4096, 64, 64, 1, 0, 1, 148, ctypes.byref(nb),
+                                             ctypes.byref(nl), ctypes.byref(ws)) == 0
+        assert (nb.value, nl.value) == (3, 2)
+    finally:
+        assert b.lib.lt_debug_set_schedule(b.LT_SCHED_AUTO, 0) == 0
+    assert b.lib.lt_linear_attn_fwd_plan(2, 8, 8, 4096, 64, 64, 1, 0, 1, 148, ctypes.byref(nb),
+                                         ctypes.byref(nl), ctypes.byref(ws)) == 0
+    assert (nb.value, nl.value) == (8, 1)
 
 
 @pytest.mark.parametrize("case,expect", [
@@ -149,12 +185,10 @@ def test_oracle_and_library_share_no_code():
     ((2, 8, 8, 4096, 64, 64, 1, 0, 0), (1, 1, 0)),                           # fp32 path
     ((1, 2, 1, 8192, 64, 64, 1, 0, 1), (64, 1, 64 * (64 * 64 + 64) * 4)),  # 64 chunks, one launch
 ])
-def test_fwd_plan_host_arithmetic(monkeypatch, shape, expect):
+def test_fwd_plan_host_arithmetic(sched, shape, expect):
     """Blocks per sequence: the SM count over the (sequence, KV head) lanes,
     at most the chunk count; one launch when there is one block; the
     workspace holds one fp32 d x dv + d partial state per block."""
-    monkeypatch.delenv("LT_BLOCKS", raising=False)
-    monkeypatch.delenv("LT_KERNEL", raising=False)
     from causal_linear_attention_chunked_b200 import _binding as b
     B, Hq, Hkv, N, d, dv, causal, packed, dt = shape
     nb, nl, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
@@ -164,11 +198,10 @@ def test_fwd_plan_host_arithmetic(monkeypatch, shape, expect):
     assert (nb.value, nl.value, ws.value) == expect
 
 
-def test_fwd_plan_pair_forced(monkeypatch):
-    """LT_KERNEL=pair keeps the two-launch block scan where the one-launch
-    cluster exchange would apply."""
-    monkeypatch.delenv("LT_BLOCKS", raising=False)
-    monkeypatch.setenv("LT_KERNEL", "pair")
+def test_fwd_plan_pair_forced(sched):
+    """The two-launch override keeps the state launch plus the forward launch
+    where the one-launch path would apply."""
+    sched(kernel="two_launch")
     from causal_linear_attention_chunked_b200 import _binding as b
     nb, nl, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
     st = b.lib.lt_linear_attn_fwd_plan(2, 8, 8, 4096, 64, 64, 1, 0, 1, 148,

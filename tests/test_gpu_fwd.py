@@ -134,40 +134,14 @@ def test_bf16_deterministic():
     assert torch.equal(a, b)
 
 
-SPLIT_CASES = [
-    # (B, Hq, Hkv, N, causal)
-    (1, 2, 2, 1000, True),     # 8 chunks, ragged tail
-    (2, 4, 2, 777, True),      # GQA inside the split kernel
-    (1, 1, 1, 2049, False),    # 17 chunks, non-causal
-    (1, 2, 1, 130, True),      # 2 chunks: clusters larger than the chunk count
-    (1, 1, 1, 16 * 128 * 2 + 3, True),  # 33 chunks: inactive last round on most CTAs
-]
-
-
-@pytest.mark.parametrize("n_split", [1, 2, 3, 5, 8, 16])
-@pytest.mark.parametrize("case", SPLIT_CASES, ids=lambda c: "B%dHq%dHkv%dN%d%s" % (
-    c[0], c[1], c[2], c[3], "c" if c[4] else "nc"))
-def test_split_kernel_cluster_sizes(monkeypatch, n_split, case):
-    """The cluster variant (LT_KERNEL=cluster): a sequence split over a
-    cluster of n CTAs that exchange their chunk states through distributed
-    shared memory."""
-    monkeypatch.setenv("LT_KERNEL", "cluster")
-    monkeypatch.setenv("LT_SPLIT_N", str(n_split))
-    B, Hq, Hkv, N, causal = case
-    q, k, v = inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16, 0.125, seed=N + n_split)
-    got = run_dense(q, k, v, causal)
-    ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
-    assert row_rel_err(got, ref) <= TOL_BF16
-
-
 @pytest.mark.parametrize("case", DENSE_CASES[:8], ids=lambda c: "B%dHq%dHkv%dN%d%s" % (
     c[0], c[1], c[2], c[3], "c" if c[6] else "nc"))
-def test_sequential_kernel_forced(monkeypatch, case):
+def test_sequential_kernel_forced(sched, case):
     """The general kernel run fully sequentially (one CTA per (sequence,
     KV head)) on the d = dv = 64 shapes the specialised kernel normally
     takes."""
-    monkeypatch.setenv("LT_KERNEL", "seq")
-    monkeypatch.setenv("LT_BLOCKS", "1")
+    sched(kernel="general")
+    sched(blocks=1)
     B, Hq, Hkv, N, d, dv, causal = case
     q, k, v = inputs.make_custom(B, Hq, Hkv, N, d, dv, torch.bfloat16, d ** -0.5, seed=N)
     got = run_dense(q, k, v, causal)
@@ -175,14 +149,14 @@ def test_sequential_kernel_forced(monkeypatch, case):
     assert row_rel_err(got, ref) <= TOL_BF16
 
 
-def test_split_and_sequential_agree_closely(monkeypatch):
+def test_block_and_general_kernels_agree_closely(sched):
     """The two kernels differ only in rounding order (state operand, bf16
     output rounding of each); two independent bf16 roundings of the same
     value can differ by 2 ulp (0.78% of an entry), so their outputs must
     agree to 1e-2 in the row metric, well inside the 2e-2 bar."""
     q, k, v = inputs.make_custom(2, 8, 8, 4096, 64, 64, torch.bfloat16, 0.125, seed=9)
     a = run_dense(q, k, v, True)
-    monkeypatch.setenv("LT_KERNEL", "seq")
+    sched(kernel="general")
     b = run_dense(q, k, v, True)
     assert row_rel_err(a, b) <= 1e-2
 
@@ -202,17 +176,17 @@ BLOCK_CASES = [
 @pytest.mark.parametrize("nb", [1, 2, 3, 5, 8])
 @pytest.mark.parametrize("case", BLOCK_CASES, ids=lambda c: "B%dHq%dHkv%dN%d%s" % (
     c[0], c[1], c[2], c[3], "c" if c[4] else "nc"))
-def test_block_kernel_block_counts(monkeypatch, nb, case, mode):
-    """d = dv = 64, the sequence cut into nb blocks (LT_BLOCKS).  "pair": the
-    block aggregates in a first launch, then one CTA per block from the
-    carried prefix.  "auto": blocks of at most four chunks, at most eight of
-    them, run as one launch whose blocks form a cluster and exchange their
-    aggregates in shared memory; other shapes as "pair"."""
-    monkeypatch.setenv("LT_BLOCKS", str(nb))
+def test_block_kernel_block_counts(sched, nb, case, mode):
+    """d = dv = 64, the sequence cut into nb blocks (schedule override).
+    "pair": the block aggregates in a first launch, then one CTA per block
+    from the carried prefix.  "auto": blocks of at most four chunks run as
+    one cooperative launch whose blocks exchange their aggregates through the
+    workspace; other shapes as "pair"."""
+    sched(blocks=nb)
     if mode == "pair":
-        monkeypatch.setenv("LT_KERNEL", "pair")
+        sched(kernel="two_launch")
     else:
-        monkeypatch.delenv("LT_KERNEL", raising=False)
+        sched(kernel="auto")
     B, Hq, Hkv, N, causal = case
     q, k, v = inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16, 0.125, seed=N + 7 * nb)
     got = run_dense(q, k, v, causal)
@@ -236,22 +210,22 @@ FUSED_CASES = [
 
 @pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: "B%dHq%dHkv%dN%d%s%s" % (
     c[0], c[1], c[2], c[3], "c" if c[4] else "nc", "-nb%d" % c[5] if c[5] else ""))
-def test_fused_launch_matches_two_launches_bitwise(monkeypatch, case):
+def test_fused_launch_matches_two_launches_bitwise(sched, case):
     """The one-launch path and the two-launch path compute the same block
     aggregates with the same products and sum the carry in the same block
     order, so their outputs agree bit for bit; both match the oracle."""
     import causal_linear_attention_chunked_b200 as L
     B, Hq, Hkv, N, causal, nb_forced = case
-    monkeypatch.delenv("LT_KERNEL", raising=False)
+    sched(kernel="auto")
     if nb_forced:
-        monkeypatch.setenv("LT_BLOCKS", str(nb_forced))
+        sched(blocks=nb_forced)
     else:
-        monkeypatch.delenv("LT_BLOCKS", raising=False)
+        sched(blocks=0)
     nb, launches, ws = L.linear_attn_fwd_plan(B, Hq, Hkv, N, 64, 64, causal=causal)
     assert nb >= 2 and launches == 1 and ws > 0
     q, k, v = inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16, 0.125, seed=N + B)
     one = run_dense(q, k, v, causal)
-    monkeypatch.setenv("LT_KERNEL", "pair")
+    sched(kernel="two_launch")
     assert L.linear_attn_fwd_plan(B, Hq, Hkv, N, 64, 64, causal=causal)[1] == 2
     two = run_dense(q, k, v, causal)
     assert np.array_equal(one, two)
@@ -259,13 +233,11 @@ def test_fused_launch_matches_two_launches_bitwise(monkeypatch, case):
     assert row_rel_err(one, ref) <= TOL_BF16
 
 
-def test_fused_launch_in_cuda_graph_replays_with_new_inputs(monkeypatch):
+def test_fused_launch_in_cuda_graph_replays_with_new_inputs(sched):
     """A captured one-launch call replayed with new input contents: each
     replay publishes its own aggregates and meets at its own grid barrier,
     so no replay takes another replay's aggregates for its own."""
     import causal_linear_attention_chunked_b200 as L
-    monkeypatch.delenv("LT_BLOCKS", raising=False)
-    monkeypatch.delenv("LT_KERNEL", raising=False)
     B, Hq, Hkv, N = 2, 8, 8, 4096
     assert L.linear_attn_fwd_plan(B, Hq, Hkv, N, 64, 64, causal=True)[1] == 1
     q, k, v = (t.cuda() for t in inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16,
@@ -295,13 +267,11 @@ def test_fused_launch_in_cuda_graph_replays_with_new_inputs(monkeypatch):
         assert row_rel_err(got, ref) <= TOL_BF16
 
 
-def test_fused_launch_many_back_to_back(monkeypatch):
+def test_fused_launch_many_back_to_back(sched):
     """Forty one-launch calls in a row on one stream, alternating two input
     sets without synchronising: each meets the grid barrier of its own
     launch, so every output equals the first output of its input set."""
     import causal_linear_attention_chunked_b200 as L
-    monkeypatch.delenv("LT_BLOCKS", raising=False)
-    monkeypatch.delenv("LT_KERNEL", raising=False)
     B, Hq, Hkv, N = 2, 8, 8, 4096
     assert L.linear_attn_fwd_plan(B, Hq, Hkv, N, 64, 64, causal=True)[1] == 1
     sets = [tuple(t.cuda() for t in inputs.make_custom(B, Hq, Hkv, N, 64, 64, torch.bfloat16,
@@ -314,13 +284,13 @@ def test_fused_launch_many_back_to_back(monkeypatch):
     assert not torch.equal(outs[0], outs[1])
 
 
-def test_block_kernel_deterministic_across_block_counts(monkeypatch):
+def test_block_kernel_deterministic_across_block_counts(sched):
     """Every block count computes the same function; results agree to a few
     bf16 ulps (only the summation order of the carried state differs)."""
     q, k, v = inputs.make_custom(1, 4, 4, 3000, 64, 64, torch.bfloat16, 0.125, seed=4)
     outs = []
     for nb in (1, 4, 12):
-        monkeypatch.setenv("LT_BLOCKS", str(nb))
+        sched(blocks=nb)
         outs.append(run_dense(q, k, v, True))
     for o in outs[1:]:
         assert row_rel_err(o, outs[0]) <= 1e-2
@@ -340,13 +310,13 @@ GENERAL_BLOCK_CASES = [
 @pytest.mark.parametrize("nb", [1, 2, 3, 5])
 @pytest.mark.parametrize("case", GENERAL_BLOCK_CASES, ids=lambda c: "B%dHq%dHkv%dN%dd%ddv%d%s" % (
     c[0], c[1], c[2], c[3], c[4], c[5], "c" if c[6] else "nc"))
-def test_general_kernel_block_counts(monkeypatch, nb, case):
+def test_general_kernel_block_counts(sched, nb, case):
     """The general kernel (every width pair) with the sequence cut into nb
     blocks: the state launch's block aggregates are summed into the carry
     each block starts from (written into its TMEM state accumulator when
     causal, used as the whole state when not)."""
-    monkeypatch.setenv("LT_KERNEL", "seq")
-    monkeypatch.setenv("LT_BLOCKS", str(nb))
+    sched(kernel="general")
+    sched(blocks=nb)
     B, Hq, Hkv, N, d, dv, causal = case
     q, k, v = inputs.make_custom(B, Hq, Hkv, N, d, dv, torch.bfloat16, d ** -0.5,
                                  seed=N + 11 * nb)

@@ -31,6 +31,14 @@ MUTANTS = [
     ("initial normaliser ignored", "if (z0) memcpy(", "if (0) memcpy("),
     ("state indexed by query head", "const int64_t sg = (int64_t)s * Hkv + g;",
      "const int64_t sg = (int64_t)s * Hkv + h % Hkv;"),
+    # the selected-rows form only (8-space indentation is unique to it)
+    ("rows: non-causal stops at the diagonal",
+     "\n        const int64_t jend = causal ? i + 1 : n;",
+     "\n        const int64_t jend = i + 1;"),
+    ("rows: GQA head mapping h % Hkv", "\n        const int g = h / G;\n        double *pq",
+     "\n        const int g = h % Hkv;\n        double *pq"),
+    ("rows: packed offsets ignored", "\n        seq_range(s, N, cu_seqlens, &t0, &n);\n        if (i < 0",
+     "\n        seq_range(s, N, NULL, &t0, &n);\n        if (i < 0"),
 ]
 
 
@@ -38,6 +46,7 @@ def _build_mutant(tmp_path, idx, old, new):
     with open(obuild.SRC) as f:
         src = f.read()
     assert old in src, "mutation target not found: %r" % old
+    assert src.count(old) == 1 or not old.startswith("\n"), "ambiguous target: %r" % old
     src = src.replace(old, new)
     c = tmp_path / ("mutant%d.c" % idx)
     so = tmp_path / ("mutant%d.so" % idx)
@@ -57,7 +66,7 @@ def test_mutant_is_caught(tmp_path, monkeypatch, idx):
     for pin in pins.ALL_PINS:
         try:
             pin()
-        except AssertionError:
+        except (AssertionError, ValueError):  # a wrong value, or a rejected valid call
             failed.append(pin.__name__)
     monkeypatch.setattr(oracle, "_lib", None)
     assert failed, "no pin caught the planted mistake: %s" % name
