@@ -469,4 +469,49 @@ __device__ __forceinline__ bool grid_barrier(bool wait, volatile int* abort, int
   }
 }
 
+
+// The grid barrier above split in two, for a CTA that arrives early and
+// waits later.  grid_arrive: one thread per CTA, exactly once per CTA and
+// launch, on every path; it stores the barrier word's value before the
+// arrival in *old and returns false (after recording an error) when the
+// launch is not cooperative.  grid_wait(old): wait, bounded like mbar_wait,
+// until every CTA has arrived.
+__device__ __forceinline__ bool grid_arrive(unsigned int* old, volatile int* abort, int* err) {
+  cooperative_groups::details::grid_workspace* gw =
+      cooperative_groups::details::get_grid_workspace();
+  if (gw == nullptr) {
+    *abort = 1;
+    report_error(err, kDevErrTimeout);
+    return false;
+  }
+  const unsigned int ctas = gridDim.x * gridDim.y * gridDim.z;
+  const bool master = (blockIdx.x | blockIdx.y | blockIdx.z) == 0;
+  const unsigned int inc = master ? 0x80000000u - (ctas - 1u) : 1u;
+  unsigned int o;
+  asm volatile("atom.add.release.gpu.u32 %0, [%1], %2;" : "=r"(o) : "l"(&gw->barrier), "r"(inc)
+               : "memory");
+  *old = o;
+  return true;
+}
+
+__device__ __forceinline__ bool grid_wait(unsigned int old, volatile int* abort, int* err,
+                                          uint64_t limit_ns) {
+  cooperative_groups::details::grid_workspace* gw =
+      cooperative_groups::details::get_grid_workspace();
+  unsigned int* bar = &gw->barrier;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    unsigned int cur;
+    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(bar) : "memory");
+    if ((cur ^ old) & 0x80000000u) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      report_error(err, kDevErrTimeout);
+      return false;
+    }
+    __nanosleep(128);  // one poller per CTA on one word: keep its line cool
+  }
+}
+
 }  // namespace lt

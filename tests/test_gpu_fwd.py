@@ -200,20 +200,24 @@ FUSED_CASES = [
     (2, 8, 8, 4096, True, 0),        # the headline shape: 8 blocks of 4 chunks
     (4, 8, 8, 2000, True, 0),        # 4 blocks of 4 chunks, ragged last chunk
     (1, 4, 4, 7 * 128 + 117, True, 0),  # 8 blocks of 1 chunk
-    (2, 4, 1, 1000, True, 0),        # 4 query heads per KV head
-    (1, 8, 2, 3000, True, 6),        # GQA, 6 blocks of 4 chunks
+    (2, 4, 1, 1000, True, 0),        # 4 query heads per KV head: 8 blocks of 1 chunk
+    (1, 8, 4, 3000, True, 12),       # GQA, 12 blocks of 2 chunks x 2 query heads
+    (1, 8, 2, 3000, True, 0),        # GQA, 24 blocks of 1 chunk x 4 query heads
     (1, 2, 2, 1024, False, 0),
     (3, 2, 2, 900, False, 0),
-    (1, 4, 2, 1500, False, 3),       # 3 blocks of 4 chunks
+    (1, 4, 2, 1500, False, 6),       # 6 blocks of 2 chunks x 2 query heads
+    (1, 4, 1, 1000, False, 0),       # 8 blocks of 1 chunk x 4 query heads
 ]
 
 
 @pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: "B%dHq%dHkv%dN%d%s%s" % (
     c[0], c[1], c[2], c[3], "c" if c[4] else "nc", "-nb%d" % c[5] if c[5] else ""))
-def test_fused_launch_matches_two_launches_bitwise(sched, case):
-    """The one-launch path and the two-launch path compute the same block
-    aggregates with the same products and sum the carry in the same block
-    order, so their outputs agree bit for bit; both match the oracle."""
+def test_fused_launch_agrees_with_two_launches(sched, case):
+    """The one-launch path splits each chunk's starting state into the carry
+    of the earlier blocks and the block's own earlier chunks and rounds each
+    part to the bf16 operand separately; the two-launch path rounds their sum
+    once.  Both match the oracle, and they agree with each other to within
+    two bf16 roundings (1e-2 in the row metric)."""
     import causal_linear_attention_chunked_b200 as L
     B, Hq, Hkv, N, causal, nb_forced = case
     sched(kernel="auto")
@@ -228,9 +232,10 @@ def test_fused_launch_matches_two_launches_bitwise(sched, case):
     sched(kernel="two_launch")
     assert L.linear_attn_fwd_plan(B, Hq, Hkv, N, 64, 64, causal=causal)[1] == 2
     two = run_dense(q, k, v, causal)
-    assert np.array_equal(one, two)
+    assert row_rel_err(one, two) <= 1e-2
     ref = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6)
     assert row_rel_err(one, ref) <= TOL_BF16
+    assert row_rel_err(two, ref) <= TOL_BF16
 
 
 def test_fused_launch_in_cuda_graph_replays_with_new_inputs(sched):
