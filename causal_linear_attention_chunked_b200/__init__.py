@@ -13,7 +13,8 @@ The binding (and with it the library) is loaded on first use of one of the
 API names below; a missing library raises ImportError.
 """
 _API = ("linear_attn_fwd", "linear_attn_fwd_state", "linear_attn_fwd_plan",
-        "linear_attn_decode_step",
+        "linear_attn_decode_step", "linear_attn_state", "linear_attn_state_carry",
+        "set_schedule",
         "get_last_device_error",
         "linear_attn_fwd_host", "LtError")
 

@@ -23,7 +23,7 @@ _SCHED = {"auto": LT_SCHED_AUTO, "two_launch": LT_SCHED_TWO_LAUNCH, "general": L
 EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_fwd_noalloc", "lt_linear_attn_fwd_plan",
             "lt_linear_attn_fwd_state", "lt_linear_attn_decode_step", "lt_status_string",
             "lt_get_last_device_error", "lt_abi_version", "lt_selftest_wait_timeout",
-            "lt_debug_set_schedule")
+            "lt_debug_set_schedule", "lt_linear_attn_state", "lt_linear_attn_state_carry")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("liblt.so is not built (run `python -m "
@@ -54,6 +54,11 @@ lib.lt_get_last_device_error.restype = _i
 lib.lt_abi_version.restype = _i
 lib.lt_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp]
 lib.lt_selftest_wait_timeout.restype = _i
+lib.lt_linear_attn_state.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
+                                     _i]
+lib.lt_linear_attn_state.restype = _i
+lib.lt_linear_attn_state_carry.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]
+lib.lt_linear_attn_state_carry.restype = _i
 lib.lt_debug_set_schedule.argtypes = [_i, _i]
 lib.lt_debug_set_schedule.restype = _i
 
@@ -153,6 +158,57 @@ def linear_attn_fwd_state(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, S0=No
                                         _ptr(S0), _ptr(z0), _ptr(S), _ptr(z),
                                         _stream_handle(stream, q.device), _dtype_code(q.dtype)))
     return (out, S, z) if return_state else out
+
+
+def linear_attn_state(k, v, cu_seqlens=None, S0=None, z0=None, S_out=None, z_out=None,
+                      stream=None):
+    """The final state of every (sequence, KV head) without the outputs:
+    (S, z) = (S0, z0) + sum over the sequence of phi(K_t)^T V_t and phi(K_t);
+    fp32 [sequences, H_kv, d, dv] and [sequences, H_kv, d].  k, v as for
+    linear_attn_fwd.  See lt_linear_attn_state in include/lt_linear_attn.h."""
+    if cu_seqlens is None:
+        B, N, Hkv, d = k.shape
+        dv = v.shape[3]
+    else:
+        N, Hkv, d = k.shape
+        dv = v.shape[2]
+        B = cu_seqlens.numel() - 1
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
+            raise TypeError("cu_seqlens must be a contiguous int32 tensor")
+    for t in (k, v):
+        if not t.is_contiguous():
+            raise ValueError("k, v must be contiguous")
+    for t in (S0, z0):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+            raise TypeError("S0 and z0 must be contiguous float32 tensors")
+    S = S_out if S_out is not None else torch.empty((B, Hkv, d, dv), dtype=torch.float32,
+                                                    device=k.device)
+    z = z_out if z_out is not None else torch.empty((B, Hkv, d), dtype=torch.float32,
+                                                    device=k.device)
+    _check(lib.lt_linear_attn_state(_ptr(k), _ptr(v), B, Hkv, N, d, dv, _ptr(cu_seqlens), _ptr(S0),
+                                    _ptr(z0), _ptr(S), _ptr(z), _stream_handle(stream, k.device),
+                                    _dtype_code(k.dtype)))
+    return S, z
+
+
+def linear_attn_state_carry(S_all, z_all, rank, causal=True, S_out=None, z_out=None,
+                            stream=None):
+    """Segment `rank`'s starting state from every segment's state S_all
+    [world, B, H_kv, d, dv], z_all [world, B, H_kv, d] (fp32): the sum over
+    the earlier segments (causal) or the other segments (non-causal), in
+    rank order.  See lt_linear_attn_state_carry."""
+    world, B, Hkv, d, dv = S_all.shape
+    for t in (S_all, z_all):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise TypeError("S_all and z_all must be contiguous float32 tensors")
+    S = S_out if S_out is not None else torch.empty((B, Hkv, d, dv), dtype=torch.float32,
+                                                    device=S_all.device)
+    z = z_out if z_out is not None else torch.empty((B, Hkv, d), dtype=torch.float32,
+                                                    device=S_all.device)
+    _check(lib.lt_linear_attn_state_carry(_ptr(S_all), _ptr(z_all), world, int(rank),
+                                          int(bool(causal)), B, Hkv, d, dv, _ptr(S), _ptr(z),
+                                          _stream_handle(stream, S_all.device)))
+    return S, z
 
 
 def linear_attn_fwd_plan(B, H_q, H_kv, N, d, dv, causal=True, packed=False,

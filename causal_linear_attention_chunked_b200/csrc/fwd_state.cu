@@ -65,6 +65,16 @@ __global__ void __launch_bounds__(kPrefixThreads)
 
 }  // namespace
 
+cudaError_t launch_state_prefix(const FwdLaunch& p, int nb, float* ws, const float* s0,
+                                const float* z0, float* s_out, float* z_out,
+                                cudaStream_t stream) {
+  const size_t E = (size_t)p.d * p.dv + p.d;
+  const dim3 grid((unsigned)((E + kPrefixThreads - 1) / kPrefixThreads), p.Hkv, p.B);
+  lt_state_prefix_kernel<<<grid, kPrefixThreads, 0, stream>>>(ws, nb, p.Hkv, p.d, p.dv, p.causal,
+                                                              s0, z0, s_out, z_out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fwd_state(const FwdLaunch& p, bool bf16, const float* s0, const float* z0,
                              float* s_out, float* z_out, cudaStream_t stream) {
   if (!bf16) return launch_fwd_f32_state(p, s0, z0, s_out, z_out, stream);
@@ -83,12 +93,7 @@ cudaError_t launch_fwd_state(const FwdLaunch& p, bool bf16, const float* s0, con
   all.causal = 0;
   e = launch_block_state(all, nb, w, stream);
   // 2. carries and the final state
-  if (e == cudaSuccess) {
-    const dim3 grid((unsigned)((E + kPrefixThreads - 1) / kPrefixThreads), p.Hkv, p.B);
-    lt_state_prefix_kernel<<<grid, kPrefixThreads, 0, stream>>>(w, nb, p.Hkv, p.d, p.dv,
-                                                                p.causal, s0, z0, s_out, z_out);
-    e = cudaGetLastError();
-  }
+  if (e == cudaSuccess) e = launch_state_prefix(p, nb, w, s0, z0, s_out, z_out, stream);
   // 3. the forward launch from the precomputed carries
   if (e == cudaSuccess)
     e = (p.d == 64 && p.dv == 64) ? launch_fwd_bf16_block_pre(p, nb, w, stream)

@@ -27,4 +27,16 @@ cudaError_t launch_fwd_f32_state(const FwdLaunch& p, const float* s0, const floa
 cudaError_t launch_fwd_state(const FwdLaunch& p, bool bf16, const float* s0, const float* z0,
                              float* s_out, float* z_out, cudaStream_t stream);
 
+// Block states [lane][nb][d*dv + d] (the state launch's workspace) -> each
+// block's carry in place (causal: S0 + earlier blocks; non-causal: S0 + all)
+// and the final state S0 + all blocks into (s_out, z_out) (nullptr: not
+// written).  p.causal selects the carry.
+cudaError_t launch_state_prefix(const FwdLaunch& p, int nb, float* ws, const float* s0,
+                                const float* z0, float* s_out, float* z_out,
+                                cudaStream_t stream);
+
+// The final state alone, S0 + sum over each sequence (no outputs; q unused).
+cudaError_t launch_state_only(const FwdLaunch& p, bool bf16, const float* s0, const float* z0,
+                              float* s_out, float* z_out, cudaStream_t stream);
+
 }  // namespace lt

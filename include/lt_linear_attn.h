@@ -25,8 +25,8 @@
  *     a stream-ordered workspace on `stream` (cudaMallocAsync, released by
  *     cudaFreeAsync on the same stream before the call returns) for the
  *     per-block partial states; lt_linear_attn_fwd_plan() gives its size.
- *     lt_linear_attn_fwd_state with LT_BF16 allocates the same way (always).
- *     No other entry point allocates.
+ *     lt_linear_attn_fwd_state and lt_linear_attn_state with LT_BF16
+ *     allocate the same way (always).  No other entry point allocates.
  *   - Layouts are token-major and dense (row-major, no padding):
  *       dense:   q [B][N][H_q][d],  k [B][N][H_kv][d],  v [B][N][H_kv][dv],
  *                out [B][N][H_q][dv]
@@ -212,6 +212,57 @@ LT_API lt_status_t lt_linear_attn_fwd_state(const void *q, const void *k, const 
                                             const int32_t *cu_seqlens, const float *S0,
                                             const float *z0, float *S_out, float *z_out,
                                             lt_stream_t stream, lt_dtype_t dtype);
+
+/*
+ * lt_linear_attn_state: the final state of every (sequence, KV head) without
+ * the outputs -- for linear attention the whole past of a sequence is this
+ * fixed-size state (lineartile page, "Reference": the recurrent view;
+ * "Features": KV-cache reuse).  For sequence s and KV head g:
+ *     S_out = S0 + sum_t phi(K_t)^T V_t,   z_out = z0 + sum_t phi(K_t)
+ * over the sequence's tokens.  It reads only K and V: a prefill that needs
+ * just the state, or one segment's contribution when a sequence is cut into
+ * segments across devices (context parallelism, with
+ * lt_linear_attn_state_carry).
+ *
+ * k, v       as for lt_linear_attn_fwd (element type dtype, 16-byte aligned).
+ * B, H_kv, N, d, dv, cu_seqlens, stream, dtype   as for lt_linear_attn_fwd.
+ * S0, z0     [B][H_kv][d][dv] and [B][H_kv][d] fp32 device, or both NULL (zero).
+ * S_out, z_out  the same shapes, fp32 device (S_out 16-byte aligned); they
+ *            must not overlap the inputs or each other.
+ * Evaluation: bf16 as the first launch of the block-parallel forward pass
+ * (every block's partial state on the tensor cores, in a stream-ordered
+ * workspace released before return) plus a summation in block order; fp32
+ * with FMA arithmetic, one CTA per (sequence, KV head).
+ * Returns as lt_linear_attn_fwd.
+ */
+LT_API lt_status_t lt_linear_attn_state(const void *k, const void *v, int B, int H_kv, int N,
+                                        int d, int dv, const int32_t *cu_seqlens,
+                                        const float *S0, const float *z0, float *S_out,
+                                        float *z_out, lt_stream_t stream, lt_dtype_t dtype);
+
+/*
+ * lt_linear_attn_state_carry: the starting state of segment `rank` when every
+ * sequence of a batch is cut into `world` contiguous segments in rank order
+ * (context parallelism, lineartile page "Features": multi-GPU sharding; the
+ * inter-segment carry of "Why Stream Wins at Ultra-Long Context", section
+ * 5.3, across devices).  From the states of every segment computed from zero
+ * (lt_linear_attn_state, gathered from the ranks):
+ *     causal:     S_out = sum_{r < rank} S_all[r]   (z likewise)
+ *     non-causal: S_out = sum_{r != rank} S_all[r]
+ * summed in fp32 in rank order, so every rank and every run gets the same
+ * bits.  Passing (S_out, z_out) as (S0, z0) of lt_linear_attn_fwd_state over
+ * the rank's segment gives that segment's outputs of attention over the whole
+ * sequence.
+ *
+ * S_all  [world][B][H_kv][d][dv] fp32 device;  z_all  [world][B][H_kv][d].
+ * world >= 1, 0 <= rank < world, causal 0 or 1, d and dv 64 or 128.
+ * S_out  [B][H_kv][d][dv], z_out [B][H_kv][d] fp32 device; no overlaps.
+ * Returns LT_OK, LT_ERR_INVALID_ARG, LT_ERR_UNSUPPORTED or LT_ERR_CUDA.
+ */
+LT_API lt_status_t lt_linear_attn_state_carry(const float *S_all, const float *z_all, int world,
+                                              int rank, int causal, int B, int H_kv, int d,
+                                              int dv, float *S_out, float *z_out,
+                                              lt_stream_t stream);
 
 /*
  * One recurrent decode step: the fixed-size state (S, z) plays the role of

@@ -150,6 +150,37 @@ def test_fwd_state_rejects_invalid_arguments(case, expect):
     assert st == expect
 
 
+@pytest.mark.parametrize("case,expect", [
+    (dict(k=None), 1), (dict(S_out=None), 1), (dict(S0=FAKE), 1), (dict(z0=FAKE), 1),
+    (dict(B=0), 1), (dict(N=0), 1), (dict(Hkv=0), 1), (dict(d=32), 2), (dict(dv=96), 2),
+    (dict(dtype=4), 2), (dict(B=70000), 1),
+])
+def test_state_rejects_invalid_arguments(case, expect):
+    from causal_linear_attention_chunked_b200 import _binding as b
+    a = dict(k=FAKE, v=FAKE, B=1, Hkv=8, N=16, d=64, dv=64, cu=None, S0=None, z0=None,
+             S_out=FAKE, z_out=FAKE, stream=None, dtype=1)
+    a.update(case)
+    st = b.lib.lt_linear_attn_state(a["k"], a["v"], a["B"], a["Hkv"], a["N"], a["d"], a["dv"],
+                                    a["cu"], a["S0"], a["z0"], a["S_out"], a["z_out"],
+                                    a["stream"], a["dtype"])
+    assert st == expect
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(S_all=None), 1), (dict(z_out=None), 1), (dict(world=0), 1), (dict(rank=-1), 1),
+    (dict(rank=4), 1), (dict(causal=3), 1), (dict(B=0), 1), (dict(d=48), 2),
+])
+def test_state_carry_rejects_invalid_arguments(case, expect):
+    from causal_linear_attention_chunked_b200 import _binding as b
+    a = dict(S_all=FAKE, z_all=FAKE, world=4, rank=1, causal=1, B=1, Hkv=2, d=64, dv=64,
+             S_out=FAKE, z_out=FAKE)
+    a.update(case)
+    st = b.lib.lt_linear_attn_state_carry(a["S_all"], a["z_all"], a["world"], a["rank"],
+                                          a["causal"], a["B"], a["Hkv"], a["d"], a["dv"],
+                                          a["S_out"], a["z_out"], None)
+    assert st == expect
+
+
 def test_selftest_wait_rejects_invalid_limit():
     from causal_linear_attention_chunked_b200 import _binding as b
     assert b.lib.lt_selftest_wait_timeout(0, None) == 1

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle
-from parity import row_rel_err, TOL_BF16, TOL_F32
+from parity import row_rel_err, state_rel_err, TOL_BF16, TOL_F32, TOL_STATE_BF16, TOL_STATE_F32
 from causal_linear_attention_chunked_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -17,22 +17,6 @@ def lt():
     return L
 
 
-def state_rel_err(got, ref):
-    """Largest error of a state, relative to the largest magnitude of the
-    same (sequence, KV head) state."""
-    got = np.asarray(got, dtype=np.float64)
-    ref = np.asarray(ref, dtype=np.float64)
-    assert got.shape == ref.shape and np.all(np.isfinite(got))
-    g2 = got.reshape(got.shape[0] * got.shape[1], -1)
-    r2 = ref.reshape(ref.shape[0] * ref.shape[1], -1)
-    den = np.maximum(np.abs(r2).max(axis=1), 1e-30)
-    return float((np.abs(g2 - r2).max(axis=1) / den).max())
-
-
-# fp32 state accumulated from bf16-rounded phi(K): relative error of a state
-# well inside the bf16 rounding of its terms (2^-8)
-TOL_STATE_BF16 = 8e-3
-TOL_STATE_F32 = 1e-4
 
 
 def prefix_state(B, Hkv, d, dv, n, dtype, seed):
