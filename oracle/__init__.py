@@ -40,12 +40,17 @@ def _load():
         lib.lt_oracle_decode_step.argtypes = [vp, vp, vp, ip, dp, dp, dp, ip, ip, ip, ip, ip,
                                               ctypes.c_double]
         lib.lt_oracle_fwd_state.argtypes = fwd_args + [dp, dp, dp, dp]
+        bwd_args = [vp, vp, vp, vp, ip, dp, dp, dp, ip, ip, ip, ip, ip, ip, ip,
+                    ctypes.c_double, i32p]
+        lib.lt_oracle_bwd_quadratic.argtypes = bwd_args
+        lib.lt_oracle_bwd_recurrent.argtypes = bwd_args
         lib.lt_oracle_phi.argtypes = [ctypes.c_double]
         lib.lt_oracle_phi.restype = ctypes.c_double
         lib.lt_oracle_num_threads.restype = ctypes.c_int
         for name in ("lt_oracle_fwd_quadratic", "lt_oracle_fwd_recurrent", "lt_oracle_fwd_rows",
                      "lt_oracle_noncausal_numerator", "lt_oracle_decode_step",
-                     "lt_oracle_fwd_state"):
+                     "lt_oracle_fwd_state", "lt_oracle_bwd_quadratic",
+                     "lt_oracle_bwd_recurrent"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -213,3 +218,29 @@ def decode_step(q, k, v, S, z, eps=1e-6):
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return out
+
+
+def _bwd(fn, q, k, v, dout, causal, eps, cu_seqlens):
+    (rq, rk, rv, rdo), t = _same_type(q, k, v, dout)
+    B, Hq, Hkv, N, d, dv, oshape = _geometry(rq, rk, rv, cu_seqlens)
+    if tuple(rdo.shape) != tuple(oshape):
+        raise ValueError("dout must have the output's shape %s" % (oshape,))
+    dq = np.zeros(rq.shape, dtype=np.float64)
+    dk = np.zeros(rk.shape, dtype=np.float64)
+    dvv = np.zeros(rv.shape, dtype=np.float64)
+    cu, cup = _cu(cu_seqlens)
+    rc = fn(_ptr(rq), _ptr(rk), _ptr(rv), _ptr(rdo), t, _dptr(dq), _dptr(dk), _dptr(dvv), B, Hq,
+            Hkv, N, d, dv, int(bool(causal)), float(eps), cup)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return dq, dk, dvv
+
+
+def bwd_quadratic(q, k, v, dout, causal=True, eps=1e-6, cu_seqlens=None):
+    """Gradients (dQ, dK, dV) of sum(O * dout) by the quadratic definition."""
+    return _bwd(_load().lt_oracle_bwd_quadratic, q, k, v, dout, causal, eps, cu_seqlens)
+
+
+def bwd_recurrent(q, k, v, dout, causal=True, eps=1e-6, cu_seqlens=None):
+    """Gradients (dQ, dK, dV) by the forward and reverse state recurrences."""
+    return _bwd(_load().lt_oracle_bwd_recurrent, q, k, v, dout, causal, eps, cu_seqlens)

@@ -34,6 +34,15 @@
  * fp32 values are exactly representable in fp64, so the oracle sees the very
  * values the GPU sees.  All arithmetic is fp64.
  *
+ * Backward pass (the gradient of the forward above with respect to Q, K, V
+ * for an upstream gradient dO): the "lineartile 1.0.0" page lists one
+ * ("Project Structure": core/kernels/backward.py, tests/test_backward) but
+ * prints no formula; "Why Stream Wins at Ultra-Long Context", section 4.2,
+ * gives the reverse recurrence of a linear scan's backward pass.  Two
+ * independent forms below: the quadratic definition differentiated term by
+ * term, and a forward recurrence (for dQ) plus a reverse recurrence (for dK,
+ * dV) over the state.
+ *
  * Pins (tests in tests/test_oracle_pins.py): a hand-worked 2x2 example,
  * agreement of the two independent forms, associativity of the non-causal
  * product, closed forms (constant keys -> prefix mean of V), invariants
@@ -373,6 +382,194 @@ int lt_oracle_decode_step(const void *q, const void *k, const void *v, int in_ty
                     num += lt_oracle_phi(load_elem(q, ((int64_t)b * Hq + h) * d + a, in_type)) * Sg[a * dv + c];
                 out[((int64_t)b * Hq + h) * dv + c] = num / den;
             }
+        }
+    }
+    return 0;
+}
+
+/* phi'(x): 1 for x > 0, e^x for x <= 0 (both give 1 at x = 0). */
+static double phi_prime(double x) { return x > 0.0 ? 1.0 : exp(x); }
+
+/*
+ * Backward pass, form 1: the quadratic definition differentiated.  With
+ * a_ij = phi(Q_i).phi(K_j) over the kept pairs (j <= i causal, all j
+ * otherwise), den_i = sum_j a_ij + eps and O_i = sum_j a_ij V_j / den_i, an
+ * upstream gradient dO gives
+ *     g_i = dO_i / den_i,   h_i = -(dO_i . O_i) / den_i,
+ *     da_ij = g_i . V_j + h_i,
+ *     dphi(Q_i) = sum_j da_ij phi(K_j),   dphi(K_j) = sum_i da_ij phi(Q_i),
+ *     dV_j = sum_i a_ij g_i,
+ *     dQ = dphi(Q) * phi'(Q),   dK = dphi(K) * phi'(K)   (elementwise).
+ * A KV head's dK, dV sum the contributions of every query head of its group.
+ * dq [.][Hq][d], dk [.][Hkv][d], dv [.][Hkv][dv] fp64 (overwritten).
+ */
+int lt_oracle_bwd_quadratic(const void *q, const void *k, const void *v, const void *dout,
+                            int in_type, double *dq, double *dk, double *dv, int B, int Hq,
+                            int Hkv, int N, int d, int dvw, int causal, double eps,
+                            const int32_t *cu_seqlens) {
+    if (check_args(B, Hq, Hkv, N, d, dvw, eps)) return 1;
+    const int G = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int s = 0; s < B; ++s) {
+        for (int g = 0; g < Hkv; ++g) {
+            int64_t t0, n;
+            seq_range(s, N, cu_seqlens, &t0, &n);
+            double *pq = malloc(sizeof(double) * d), *pk = malloc(sizeof(double) * d);
+            double *o = malloc(sizeof(double) * dvw), *gi = malloc(sizeof(double) * dvw);
+            for (int64_t j = 0; j < n; ++j) {
+                for (int c = 0; c < d; ++c) dk[off(t0 + j, g, Hkv, d, c)] = 0.0;
+                for (int c = 0; c < dvw; ++c) dv[off(t0 + j, g, Hkv, dvw, c)] = 0.0;
+            }
+            for (int h = g * G; h < (g + 1) * G; ++h) {
+                for (int64_t i = 0; i < n; ++i) {
+                    for (int c = 0; c < d; ++c) pq[c] = lt_oracle_phi(load_elem(q, off(t0 + i, h, Hq, d, c), in_type));
+                    const int64_t jend = causal ? i + 1 : n;
+                    /* the forward row: den_i and O_i */
+                    double den = eps;
+                    for (int c = 0; c < dvw; ++c) o[c] = 0.0;
+                    for (int64_t j = 0; j < jend; ++j) {
+                        double a = 0.0;
+                        for (int c = 0; c < d; ++c) a += pq[c] * lt_oracle_phi(load_elem(k, off(t0 + j, g, Hkv, d, c), in_type));
+                        den += a;
+                        for (int c = 0; c < dvw; ++c) o[c] += a * load_elem(v, off(t0 + j, g, Hkv, dvw, c), in_type);
+                    }
+                    double go = 0.0;
+                    for (int c = 0; c < dvw; ++c) {
+                        o[c] /= den;
+                        gi[c] = load_elem(dout, off(t0 + i, h, Hq, dvw, c), in_type) / den;
+                        go += load_elem(dout, off(t0 + i, h, Hq, dvw, c), in_type) * o[c];
+                    }
+                    const double hi = -go / den;
+                    /* the gradient terms of every kept pair (i, j) */
+                    for (int c = 0; c < d; ++c) dq[off(t0 + i, h, Hq, d, c)] = 0.0;
+                    for (int64_t j = 0; j < jend; ++j) {
+                        double a = 0.0, gv = 0.0;
+                        for (int c = 0; c < d; ++c) {
+                            pk[c] = lt_oracle_phi(load_elem(k, off(t0 + j, g, Hkv, d, c), in_type));
+                            a += pq[c] * pk[c];
+                        }
+                        for (int c = 0; c < dvw; ++c) gv += gi[c] * load_elem(v, off(t0 + j, g, Hkv, dvw, c), in_type);
+                        const double da = gv + hi;
+                        for (int c = 0; c < d; ++c) {
+                            dq[off(t0 + i, h, Hq, d, c)] += da * pk[c];
+                            dk[off(t0 + j, g, Hkv, d, c)] += da * pq[c];
+                        }
+                        for (int c = 0; c < dvw; ++c) dv[off(t0 + j, g, Hkv, dvw, c)] += a * gi[c];
+                    }
+                    for (int c = 0; c < d; ++c)
+                        dq[off(t0 + i, h, Hq, d, c)] *= phi_prime(load_elem(q, off(t0 + i, h, Hq, d, c), in_type));
+                }
+            }
+            for (int64_t j = 0; j < n; ++j)
+                for (int c = 0; c < d; ++c)
+                    dk[off(t0 + j, g, Hkv, d, c)] *= phi_prime(load_elem(k, off(t0 + j, g, Hkv, d, c), in_type));
+            free(pq); free(pk); free(o); free(gi);
+        }
+    }
+    return 0;
+}
+
+/*
+ * Backward pass, form 2: recurrences over the state.  Per query head:
+ *   forward, i = 0..n-1 (causal; non-causal uses the final sums for every i):
+ *     S += phi(K_i)^T V_i,  z += phi(K_i)   (the forward pass's state)
+ *     O_i, den_i from phi(Q_i), S, z;  g_i, h_i as in form 1
+ *     dphi(Q_i) = S g_i + z h_i
+ *   reverse, j = n-1..0 (the backward recurrence of a linear scan):
+ *     R += phi(Q_j) g_j^T,  r += phi(Q_j) h_j     (sums over i >= j)
+ *     dphi(K_j) = R V_j + r,   dV_j = R^T phi(K_j)
+ *   (non-causal: R, r summed over the whole sequence before any j).
+ * Same outputs as form 1.
+ */
+int lt_oracle_bwd_recurrent(const void *q, const void *k, const void *v, const void *dout,
+                            int in_type, double *dq, double *dk, double *dv, int B, int Hq,
+                            int Hkv, int N, int d, int dvw, int causal, double eps,
+                            const int32_t *cu_seqlens) {
+    if (check_args(B, Hq, Hkv, N, d, dvw, eps)) return 1;
+    const int G = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int s = 0; s < B; ++s) {
+        for (int g = 0; g < Hkv; ++g) {
+            int64_t t0, n;
+            seq_range(s, N, cu_seqlens, &t0, &n);
+            double *S = malloc(sizeof(double) * d * dvw), *z = malloc(sizeof(double) * d);
+            double *R = malloc(sizeof(double) * d * dvw), *r = malloc(sizeof(double) * d);
+            double *pq = malloc(sizeof(double) * d), *pk = malloc(sizeof(double) * d);
+            double *vv = malloc(sizeof(double) * dvw), *o = malloc(sizeof(double) * dvw);
+            double *gs = malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * dvw);
+            double *hs = malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+            for (int64_t j = 0; j < n; ++j) {
+                for (int c = 0; c < d; ++c) dk[off(t0 + j, g, Hkv, d, c)] = 0.0;
+                for (int c = 0; c < dvw; ++c) dv[off(t0 + j, g, Hkv, dvw, c)] = 0.0;
+            }
+            for (int h = g * G; h < (g + 1) * G; ++h) {
+                /* forward recurrence: O_i, den_i, g_i, h_i and dphi(Q_i) */
+                memset(S, 0, sizeof(double) * d * dvw);
+                memset(z, 0, sizeof(double) * d);
+                for (int pass = causal ? 1 : 0; pass < 2; ++pass) {
+                    for (int64_t i = 0; i < n; ++i) {
+                        if (pass == 0 || causal) {
+                            for (int c = 0; c < d; ++c) pk[c] = lt_oracle_phi(load_elem(k, off(t0 + i, g, Hkv, d, c), in_type));
+                            for (int c = 0; c < dvw; ++c) vv[c] = load_elem(v, off(t0 + i, g, Hkv, dvw, c), in_type);
+                            for (int a = 0; a < d; ++a) {
+                                for (int c = 0; c < dvw; ++c) S[a * dvw + c] += pk[a] * vv[c];
+                                z[a] += pk[a];
+                            }
+                        }
+                        if (pass == 0) continue;  /* non-causal: the sums first */
+                        for (int c = 0; c < d; ++c) pq[c] = lt_oracle_phi(load_elem(q, off(t0 + i, h, Hq, d, c), in_type));
+                        double den = eps;
+                        for (int a = 0; a < d; ++a) den += pq[a] * z[a];
+                        double go = 0.0;
+                        for (int c = 0; c < dvw; ++c) {
+                            double num = 0.0;
+                            for (int a = 0; a < d; ++a) num += pq[a] * S[a * dvw + c];
+                            o[c] = num / den;
+                            const double d_o = load_elem(dout, off(t0 + i, h, Hq, dvw, c), in_type);
+                            gs[i * dvw + c] = d_o / den;
+                            go += d_o * o[c];
+                        }
+                        hs[i] = -go / den;
+                        for (int a = 0; a < d; ++a) {
+                            double acc = z[a] * hs[i];
+                            for (int c = 0; c < dvw; ++c) acc += S[a * dvw + c] * gs[i * dvw + c];
+                            dq[off(t0 + i, h, Hq, d, a)] =
+                                acc * phi_prime(load_elem(q, off(t0 + i, h, Hq, d, a), in_type));
+                        }
+                    }
+                }
+                /* reverse recurrence: dphi(K_j) and dV_j */
+                memset(R, 0, sizeof(double) * d * dvw);
+                memset(r, 0, sizeof(double) * d);
+                for (int pass = causal ? 1 : 0; pass < 2; ++pass) {
+                    for (int64_t j = n - 1; j >= 0; --j) {
+                        if (pass == 0 || causal) {
+                            for (int c = 0; c < d; ++c) pq[c] = lt_oracle_phi(load_elem(q, off(t0 + j, h, Hq, d, c), in_type));
+                            for (int a = 0; a < d; ++a) {
+                                for (int c = 0; c < dvw; ++c) R[a * dvw + c] += pq[a] * gs[j * dvw + c];
+                                r[a] += pq[a] * hs[j];
+                            }
+                        }
+                        if (pass == 0) continue;
+                        for (int c = 0; c < d; ++c) pk[c] = lt_oracle_phi(load_elem(k, off(t0 + j, g, Hkv, d, c), in_type));
+                        for (int c = 0; c < dvw; ++c) vv[c] = load_elem(v, off(t0 + j, g, Hkv, dvw, c), in_type);
+                        for (int a = 0; a < d; ++a) {
+                            double acc = r[a];
+                            for (int c = 0; c < dvw; ++c) acc += R[a * dvw + c] * vv[c];
+                            dk[off(t0 + j, g, Hkv, d, a)] += acc;
+                        }
+                        for (int c = 0; c < dvw; ++c) {
+                            double acc = 0.0;
+                            for (int a = 0; a < d; ++a) acc += R[a * dvw + c] * pk[a];
+                            dv[off(t0 + j, g, Hkv, dvw, c)] += acc;
+                        }
+                    }
+                }
+            }
+            for (int64_t j = 0; j < n; ++j)
+                for (int c = 0; c < d; ++c)
+                    dk[off(t0 + j, g, Hkv, d, c)] *= phi_prime(load_elem(k, off(t0 + j, g, Hkv, d, c), in_type));
+            free(S); free(z); free(R); free(r); free(pq); free(pk); free(vv); free(o); free(gs); free(hs);
         }
     }
     return 0;

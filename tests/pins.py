@@ -359,6 +359,111 @@ def pin_state_noncausal_prefix():
     assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max()
 
 
+def pin_bwd_hand_2x2():
+    """Hand-worked gradients of the 2x2 example (tests/golden/hand_2x2_backward.json)."""
+    g = _load("hand_2x2_backward.json")
+    q, k, v, do = (np.array(g[x], dtype=np.float64).reshape(1, 2, 1, 2)
+                   for x in ("q", "k", "v", "dout"))
+    for causal, key in ((True, "causal"), (False, "noncausal")):
+        for fn in (oracle.bwd_quadratic, oracle.bwd_recurrent):
+            dq, dk, dv = fn(q, k, v, do, causal=causal, eps=0.0)
+            for got, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+                assert np.allclose(got[0, :, 0], g[key][name], rtol=0, atol=1e-15), \
+                    (fn.__name__, key, name, got[0, :, 0])
+
+
+def _loss(q, k, v, do, causal, eps, cu=None):
+    return float((oracle.fwd_quadratic(q, k, v, causal=causal, eps=eps, cu_seqlens=cu) * do).sum())
+
+
+def pin_bwd_finite_differences():
+    """Both backward forms equal central finite differences of
+    L = sum(O * dO) through the (pinned) quadratic forward form: every entry
+    of Q, K and V, with negative inputs (phi' = e^x), GQA, eps > 0, causal and
+    non-causal, dense and packed."""
+    cases = [
+        # (B, N, Hq, Hkv, d, dv, causal, eps, packed lengths or None)
+        (1, 5, 2, 1, 3, 2, True, 1e-3, None),
+        (2, 4, 2, 2, 2, 3, False, 0.0, None),
+        (1, 0, 2, 1, 2, 2, True, 1e-2, [3, 0, 2]),
+    ]
+    h = 1e-5
+    for i, (B, N, Hq, Hkv, d, dv, causal, eps, lens) in enumerate(cases):
+        cu = None
+        if lens is not None:
+            cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+            T = int(cu[-1])
+            shapes = ((T, Hq, d), (T, Hkv, d), (T, Hkv, dv), (T, Hq, dv))
+        else:
+            shapes = ((B, N, Hq, d), (B, N, Hkv, d), (B, N, Hkv, dv), (B, N, Hq, dv))
+        q, k, v, do = (_rand(sh, 80 + 4 * i + j, 1.5) for j, sh in enumerate(shapes))
+        grads = [fn(q, k, v, do, causal=causal, eps=eps, cu_seqlens=cu)
+                 for fn in (oracle.bwd_quadratic, oracle.bwd_recurrent)]
+        for which, x in enumerate((q, k, v)):
+            fd = np.zeros_like(x)
+            for idx in np.ndindex(*x.shape):
+                xp, xm = x.copy(), x.copy()
+                xp[idx] += h
+                xm[idx] -= h
+                args_p = [q, k, v]
+                args_m = [q, k, v]
+                args_p[which], args_m[which] = xp, xm
+                fd[idx] = (_loss(*args_p, do, causal, eps, cu) -
+                           _loss(*args_m, do, causal, eps, cu)) / (2 * h)
+            scale = max(1e-12, np.abs(fd).max())
+            for gr in grads:
+                err = np.abs(gr[which] - fd).max() / scale
+                assert err <= 1e-6, (i, which, err)
+
+
+def pin_bwd_two_forms_agree():
+    """The differentiated quadratic form and the two recurrences agree to
+    1e-12 relative on random inputs (GQA, widths 64 and 128, non-causal)."""
+    cases = [(2, 30, 4, 2, 8, 5, True), (1, 40, 2, 2, 64, 64, True), (1, 25, 4, 1, 6, 128, False),
+             (2, 17, 2, 2, 64, 64, False)]
+    for i, (B, N, Hq, Hkv, d, dv, causal) in enumerate(cases):
+        q = _rand((B, N, Hq, d), 90 + i, 0.5)
+        k = _rand((B, N, Hkv, d), 100 + i, 0.5)
+        v = _rand((B, N, Hkv, dv), 110 + i)
+        do = _rand((B, N, Hq, dv), 120 + i)
+        a = oracle.bwd_quadratic(q, k, v, do, causal=causal, eps=1e-6)
+        b = oracle.bwd_recurrent(q, k, v, do, causal=causal, eps=1e-6)
+        for x, y in zip(a, b):
+            assert np.abs(x - y).max() <= 1e-12 * max(1e-300, np.abs(x).max()), i
+
+
+def pin_bwd_packed_and_gqa():
+    """Packed sequences give the gradients of independent dense calls; with
+    GQA, dK and dV of a KV head are the sums over its query heads of the
+    gradients with each KV head explicitly replicated."""
+    lens = [6, 0, 1, 9]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T, Hq, Hkv, d, dv = int(cu[-1]), 4, 2, 3, 4
+    q, k, v, do = (_rand(sh, 130 + j) for j, sh in
+                   enumerate(((T, Hq, d), (T, Hkv, d), (T, Hkv, dv), (T, Hq, dv))))
+    for causal in (True, False):
+        pk = oracle.bwd_recurrent(q, k, v, do, causal=causal, eps=1e-6, cu_seqlens=cu)
+        for s, n in enumerate(lens):
+            if n == 0:
+                continue
+            a, b = cu[s], cu[s + 1]
+            dense = oracle.bwd_quadratic(q[None, a:b], k[None, a:b], v[None, a:b],
+                                         do[None, a:b], causal=causal, eps=1e-6)
+            for x, y in zip(pk, dense):
+                assert np.abs(x[a:b] - y[0]).max() <= 1e-12 * max(1.0, np.abs(y).max())
+    B, N = 2, 11
+    q, k, v, do = (_rand(sh, 140 + j) for j, sh in
+                   enumerate(((B, N, Hq, d), (B, N, Hkv, d), (B, N, Hkv, dv), (B, N, Hq, dv))))
+    G = Hq // Hkv
+    for causal in (True, False):
+        dq, dk, dv_ = oracle.bwd_recurrent(q, k, v, do, causal=causal, eps=1e-6)
+        rq, rk, rv = oracle.bwd_quadratic(q, np.repeat(k, G, axis=2), np.repeat(v, G, axis=2),
+                                          do, causal=causal, eps=1e-6)
+        assert np.abs(dq - rq).max() <= 1e-12 * np.abs(rq).max()
+        assert np.abs(dk - rk.reshape(B, N, Hkv, G, d).sum(3)).max() <= 1e-12 * np.abs(dk).max()
+        assert np.abs(dv_ - rv.reshape(B, N, Hkv, G, dv).sum(3)).max() <= 1e-12 * np.abs(dv_).max()
+
+
 ALL_PINS = [
     pin_phi_is_elu_plus_one,
     pin_hand_2x2,
@@ -377,4 +482,8 @@ ALL_PINS = [
     pin_state_split_continuation,
     pin_state_final_equals_decode_chain,
     pin_state_noncausal_prefix,
+    pin_bwd_hand_2x2,
+    pin_bwd_finite_differences,
+    pin_bwd_two_forms_agree,
+    pin_bwd_packed_and_gqa,
 ]

@@ -37,6 +37,17 @@ MUTANTS = [
      "\n        const int64_t jend = i + 1;"),
     ("rows: GQA head mapping h % Hkv", "\n        const int g = h / G;\n        double *pq",
      "\n        const int g = h % Hkv;\n        double *pq"),
+    ("bwd: phi' of a negative input taken as 1", "return x > 0.0 ? 1.0 : exp(x);",
+     "return x > 0.0 ? 1.0 : 1.0;"),
+    ("bwd: normaliser term with the wrong sign (quadratic)", "const double hi = -go / den;",
+     "const double hi = go / den;"),
+    ("bwd: normaliser term dropped (recurrent)", "hs[i] = -go / den;", "hs[i] = 0.0 * go;"),
+    ("bwd: dV weighted by da instead of a", "dv[off(t0 + j, g, Hkv, dvw, c)] += a * gi[c];",
+     "dv[off(t0 + j, g, Hkv, dvw, c)] += da * gi[c];"),
+    ("bwd: the dK/dV recurrence scans forward instead of in reverse",
+     "for (int64_t j = n - 1; j >= 0; --j) {", "for (int64_t j = 0; j < n; ++j) {"),
+    ("bwd: dK of a GQA group from its first query head only", "for (int h = g * G; h < (g + 1) * G; ++h) {\n                /* forward recurrence",
+     "for (int h = g * G; h < g * G + 1; ++h) {\n                /* forward recurrence"),
     ("rows: packed offsets ignored", "\n        seq_range(s, N, cu_seqlens, &t0, &n);\n        if (i < 0",
      "\n        seq_range(s, N, NULL, &t0, &n);\n        if (i < 0"),
 ]
