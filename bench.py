@@ -388,6 +388,37 @@ def measure_decode(L, stream, device, steps=1000, reps=3):
             "note": "1000 steps replayed as one CUDA graph; the 8.4 MB fp32 state is L2-resident"}
 
 
+def measure_backward(L, w, stream, device, peak, reps=5):
+    """lt_linear_attn_bwd on the workload's shape: dQ, dK, dV for a random
+    upstream gradient.  Algorithmic bytes: q, k, v and dO read once, dq, dk,
+    dv written once."""
+    q, k, v, _ = inputs.make(w, seed=w.seed + 700)
+    q, k, v = q.to(device), k.to(device), v.to(device)
+    g = inputs.generator(w.seed + 701)
+    dout = torch.randn(q.shape[:-1] + (w.dv,), generator=g).to(w.dtype).to(device)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            L.linear_attn_bwd(q, k, v, dout, causal=w.causal, eps=w.eps, stream=stream)
+    torch.cuda.synchronize()
+    assert L.get_last_device_error(stream) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            L.linear_attn_bwd(q, k, v, dout, causal=w.causal, eps=w.eps, stream=stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    es = 2 if w.dtype == torch.bfloat16 else 4
+    nbytes = w.B * w.N * (2 * w.Hq * w.d + 2 * w.Hkv * (w.d + w.dv) + w.Hq * w.dv) * es
+    ach = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": w.name + "_backward", "tokens_per_s": w.B * w.Hq * w.N / (ms / 1e3),
+            "ms_per_step": ms, "achieved_gbs": ach, "roofline_frac": ach / peak,
+            "algorithmic_bytes": nbytes,
+            "note": "lt_linear_attn_bwd: two fp32 FMA scans (one CTA per (sequence, head)), "
+                    "eager calls timed with CUDA events"}
+
+
 def measure_e2e(L, w, steps, stream, device):
     q, k, v, cu = inputs.make(w)
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
@@ -535,6 +566,7 @@ def run_lt(args):
                                         device, l2, peak))
         extra.append(measure_decode(L, stream, device))
         extra.append(measure_eager(L, w, stream, device))
+        extra.append(measure_backward(L, w, stream, device, peak))
         line["extra"] = extra
     if rank == 0 and world == 1 and not args.profile:
         line["cpu_baseline"] = cpu_baseline(w)

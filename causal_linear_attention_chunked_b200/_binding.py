@@ -23,7 +23,8 @@ _SCHED = {"auto": LT_SCHED_AUTO, "two_launch": LT_SCHED_TWO_LAUNCH, "general": L
 EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_fwd_noalloc", "lt_linear_attn_fwd_plan",
             "lt_linear_attn_fwd_state", "lt_linear_attn_decode_step", "lt_status_string",
             "lt_get_last_device_error", "lt_abi_version", "lt_selftest_wait_timeout",
-            "lt_debug_set_schedule", "lt_linear_attn_state", "lt_linear_attn_state_carry")
+            "lt_debug_set_schedule", "lt_linear_attn_state", "lt_linear_attn_state_carry",
+            "lt_linear_attn_bwd")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("liblt.so is not built (run `python -m "
@@ -59,6 +60,9 @@ lib.lt_linear_attn_state.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp
 lib.lt_linear_attn_state.restype = _i
 lib.lt_linear_attn_state_carry.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]
 lib.lt_linear_attn_state_carry.restype = _i
+lib.lt_linear_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                   _f, _vp, _vp, _i]
+lib.lt_linear_attn_bwd.restype = _i
 lib.lt_debug_set_schedule.argtypes = [_i, _i]
 lib.lt_debug_set_schedule.restype = _i
 
@@ -158,6 +162,35 @@ def linear_attn_fwd_state(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, S0=No
                                         _ptr(S0), _ptr(z0), _ptr(S), _ptr(z),
                                         _stream_handle(stream, q.device), _dtype_code(q.dtype)))
     return (out, S, z) if return_state else out
+
+
+def linear_attn_bwd(q, k, v, dout, causal=True, eps=1e-6, cu_seqlens=None, dq=None, dk=None,
+                    dv=None, stream=None):
+    """Gradients (dq, dk, dv) of linear attention for the upstream gradient
+    dout (the output's shape and dtype).  See lt_linear_attn_bwd in
+    include/lt_linear_attn.h."""
+    if cu_seqlens is None:
+        B, N, Hq, d = q.shape
+        Hkv, dvw = k.shape[2], v.shape[3]
+    else:
+        N, Hq, d = q.shape
+        Hkv, dvw = k.shape[1], v.shape[2]
+        B = cu_seqlens.numel() - 1
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
+            raise TypeError("cu_seqlens must be a contiguous int32 tensor")
+    for t in (q, k, v, dout):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v, dout must be contiguous")
+    if dout.dtype != q.dtype:
+        raise TypeError("dout must have q's dtype")
+    dq = dq if dq is not None else torch.empty_like(q)
+    dk = dk if dk is not None else torch.empty_like(k)
+    dv = dv if dv is not None else torch.empty_like(v)
+    _check(lib.lt_linear_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), B, Hq, Hkv, N, d, dvw, int(bool(causal)), float(eps),
+                                  _ptr(cu_seqlens), _stream_handle(stream, q.device),
+                                  _dtype_code(q.dtype)))
+    return dq, dk, dv
 
 
 def linear_attn_state(k, v, cu_seqlens=None, S0=None, z0=None, S_out=None, z_out=None,

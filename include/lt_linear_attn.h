@@ -26,7 +26,8 @@
  *     cudaFreeAsync on the same stream before the call returns) for the
  *     per-block partial states; lt_linear_attn_fwd_plan() gives its size.
  *     lt_linear_attn_fwd_state and lt_linear_attn_state with LT_BF16
- *     allocate the same way (always).  No other entry point allocates.
+ *     allocate the same way (always); lt_linear_attn_bwd allocates its
+ *     workspace the same way.  No other entry point allocates.
  *   - Layouts are token-major and dense (row-major, no padding):
  *       dense:   q [B][N][H_q][d],  k [B][N][H_kv][d],  v [B][N][H_kv][dv],
  *                out [B][N][H_q][dv]
@@ -263,6 +264,35 @@ LT_API lt_status_t lt_linear_attn_state_carry(const float *S_all, const float *z
                                               int rank, int causal, int B, int H_kv, int d,
                                               int dv, float *S_out, float *z_out,
                                               lt_stream_t stream);
+
+/*
+ * lt_linear_attn_bwd: backward pass of lt_linear_attn_fwd.  For an upstream
+ * gradient dout = dL/dO it returns dq = dL/dQ, dk = dL/dK, dv = dL/dV (the
+ * lineartile page lists a backward pass, "Project Structure":
+ * core/kernels/backward.py; its formulas follow from the forward definition).
+ * With a_ij = phi(Q_i).phi(K_j) over the kept pairs, den_i = sum_j a_ij + eps:
+ *     g_i = dout_i / den_i,  h_i = -(dout_i . O_i) / den_i,  da_ij = g_i.V_j + h_i,
+ *     dQ_i = phi'(Q_i) * sum_j da_ij phi(K_j),  dK_j = phi'(K_j) * sum_i da_ij phi(Q_i),
+ *     dV_j = sum_i a_ij g_i,   phi'(x) = 1 (x > 0), e^x (x <= 0);
+ * a KV head's dk, dv sum over the query heads of its group.  O is recomputed.
+ *
+ * q, k, v, B .. cu_seqlens, stream, dtype   as for lt_linear_attn_fwd.
+ * dout   the output's layout and element type; must not overlap q, k, v.
+ * dq, dk, dv  q's, k's and v's layouts and element type (16-byte aligned,
+ *        device); written whole; must not overlap any input or each other.
+ * Evaluation: two chunked scans with fp32 FMA arithmetic (32-token chunks):
+ * a forward scan per (sequence, query head) for dq, and a reverse scan per
+ * (sequence, KV head) for dk, dv ("Why Stream Wins at Ultra-Long Context",
+ * section 4.2: the backward recurrence of a linear scan).  Scratch: a
+ * stream-ordered workspace of tokens * H_q * (dv + 1) floats, released
+ * before return.
+ * Returns as lt_linear_attn_fwd.
+ */
+LT_API lt_status_t lt_linear_attn_bwd(const void *q, const void *k, const void *v,
+                                      const void *dout, void *dq, void *dk, void *dv, int B,
+                                      int H_q, int H_kv, int N, int d, int dv_width, int causal,
+                                      float eps, const int32_t *cu_seqlens, lt_stream_t stream,
+                                      lt_dtype_t dtype);
 
 /*
  * One recurrent decode step: the fixed-size state (S, z) plays the role of

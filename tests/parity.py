@@ -47,3 +47,28 @@ def state_rel_err(got, ref):
 # well inside the bf16 rounding of its terms (2^-8)
 TOL_STATE_BF16 = 8e-3
 TOL_STATE_F32 = 1e-4
+
+
+def grad_rel_err(got, ref, cu=None):
+    """Gradient metric: per (sequence, head) slice, the largest error
+    relative to the slice's largest entry; the maximum over slices.
+
+    A row of dQ (or dK) can be a near-exact cancellation whose true value is
+    proportional to eps -- the first token of a causal sequence attends only
+    to itself, so its output moves with Q_0 and K_0 only through eps -- and a
+    per-row relative error is then meaningless; the slice holds the terms'
+    scale.  Dense arrays [B][N][H][w]; packed [T][H][w] with cu_seqlens."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape and np.all(np.isfinite(got))
+    if cu is None:
+        slices = [(got[b, :, h], ref[b, :, h]) for b in range(got.shape[0])
+                  for h in range(got.shape[2])]
+    else:
+        c = [int(x) for x in cu]
+        slices = [(got[c[s]:c[s + 1], h], ref[c[s]:c[s + 1], h]) for s in range(len(c) - 1)
+                  for h in range(got.shape[1]) if c[s + 1] > c[s]]
+    worst = 0.0
+    for g, r in slices:
+        worst = max(worst, float(np.abs(g - r).max() / max(np.abs(r).max(), 1e-30)))
+    return worst

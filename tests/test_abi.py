@@ -181,6 +181,22 @@ def test_state_carry_rejects_invalid_arguments(case, expect):
     assert st == expect
 
 
+@pytest.mark.parametrize("case,expect", [
+    (dict(q=None), 1), (dict(dout=None), 1), (dict(dq=None), 1), (dict(dv=None), 1),
+    (dict(B=0), 1), (dict(Hkv=3, Hq=8), 1), (dict(causal=2), 1), (dict(eps=-1.0), 1),
+    (dict(d=32), 2), (dict(dtype=9), 2),
+])
+def test_bwd_rejects_invalid_arguments(case, expect):
+    from causal_linear_attention_chunked_b200 import _binding as b
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, B=1, Hq=8, Hkv=8,
+             N=16, d=64, dvw=64, causal=1, eps=1e-6, dtype=1)
+    a.update(case)
+    st = b.lib.lt_linear_attn_bwd(a["q"], a["k"], a["v"], a["dout"], a["dq"], a["dk"], a["dv"],
+                                  a["B"], a["Hq"], a["Hkv"], a["N"], a["d"], a["dvw"],
+                                  a["causal"], a["eps"], None, None, a["dtype"])
+    assert st == expect
+
+
 def test_selftest_wait_rejects_invalid_limit():
     from causal_linear_attention_chunked_b200 import _binding as b
     assert b.lib.lt_selftest_wait_timeout(0, None) == 1
