@@ -18,7 +18,8 @@ import numpy as np
 
 from . import build as _build
 
-_F32, _BF16, _F64 = 0, 1, 2
+_F32, _BF16, _F64, _F16 = 0, 1, 2, 3
+PHI_KINDS = {"elu1": 0, "relu": 1, "exp": 2}
 _lib = None
 
 
@@ -44,6 +45,8 @@ def _load():
                     ctypes.c_double, i32p]
         lib.lt_oracle_bwd_quadratic.argtypes = bwd_args
         lib.lt_oracle_bwd_recurrent.argtypes = bwd_args
+        lib.lt_oracle_set_phi.argtypes = [ctypes.c_int]
+        lib.lt_oracle_set_phi.restype = ctypes.c_int
         lib.lt_oracle_phi.argtypes = [ctypes.c_double]
         lib.lt_oracle_phi.restype = ctypes.c_double
         lib.lt_oracle_num_threads.restype = ctypes.c_int
@@ -64,6 +67,8 @@ def _raw(x):
             x = x.detach().cpu().contiguous()
             if x.dtype == torch.bfloat16:
                 return x.view(torch.int16).numpy().view(np.uint16), _BF16
+            if x.dtype == torch.float16:
+                return x.view(torch.int16).numpy().view(np.uint16), _F16
             if x.dtype == torch.float32:
                 return x.numpy(), _F32
             if x.dtype == torch.float64:
@@ -72,6 +77,8 @@ def _raw(x):
     except ImportError:
         pass
     x = np.ascontiguousarray(x)
+    if x.dtype == np.float16:
+        return x.view(np.uint16), _F16
     if x.dtype == np.float32:
         return x, _F32
     if x.dtype == np.float64:
@@ -114,9 +121,27 @@ def _geometry(q, k, v, cu_seqlens):
     return B, Hq, Hkv, N, d, dv, (N, Hq, dv)
 
 
-def phi(x: float) -> float:
-    """phi(x) = ELU(x) + 1 (alpha = 1), in fp64."""
-    return _load().lt_oracle_phi(float(x))
+class feature_map:
+    """Context manager: the oracle's feature map within the block ("elu1",
+    the method's ELU + 1 and the default; "relu"; "exp")."""
+
+    def __init__(self, kind):
+        self.kind = PHI_KINDS[kind]
+
+    def __enter__(self):
+        if _load().lt_oracle_set_phi(self.kind) != 0:
+            raise ValueError("unknown feature map")
+        return self
+
+    def __exit__(self, *exc):
+        _load().lt_oracle_set_phi(0)
+        return False
+
+
+def phi(x: float, kind="elu1") -> float:
+    """The feature map in fp64 (default: phi(x) = ELU(x) + 1, alpha = 1)."""
+    with feature_map(kind):
+        return _load().lt_oracle_phi(float(x))
 
 
 def num_threads() -> int:
@@ -135,14 +160,16 @@ def _fwd(fn, q, k, v, causal, eps, cu_seqlens):
     return out
 
 
-def fwd_quadratic(q, k, v, causal=True, eps=1e-6, cu_seqlens=None):
+def fwd_quadratic(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, phi="elu1"):
     """Masked quadratic form: O_i = sum_j a_ij V_j / (sum_j a_ij + eps)."""
-    return _fwd(_load().lt_oracle_fwd_quadratic, q, k, v, causal, eps, cu_seqlens)
+    with feature_map(phi):
+        return _fwd(_load().lt_oracle_fwd_quadratic, q, k, v, causal, eps, cu_seqlens)
 
 
-def fwd_recurrent(q, k, v, causal=True, eps=1e-6, cu_seqlens=None):
+def fwd_recurrent(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, phi="elu1"):
     """Recurrent (RNN) form over the fixed-size state (S, z)."""
-    return _fwd(_load().lt_oracle_fwd_recurrent, q, k, v, causal, eps, cu_seqlens)
+    with feature_map(phi):
+        return _fwd(_load().lt_oracle_fwd_recurrent, q, k, v, causal, eps, cu_seqlens)
 
 
 def fwd_state(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, S0=None, z0=None):
@@ -166,7 +193,7 @@ def fwd_state(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, S0=None, z0=None)
     return out, S, z
 
 
-def fwd_rows(q, k, v, rows, causal=True, eps=1e-6, cu_seqlens=None):
+def fwd_rows(q, k, v, rows, causal=True, eps=1e-6, cu_seqlens=None, phi="elu1"):
     """Selected output rows by the quadratic definition.
 
     ``rows``: integer array of shape [R, 3] holding (sequence, position
@@ -177,10 +204,11 @@ def fwd_rows(q, k, v, rows, causal=True, eps=1e-6, cu_seqlens=None):
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
     out = np.zeros((rows.shape[0], dv), dtype=np.float64)
     cu, cup = _cu(cu_seqlens)
-    rc = _load().lt_oracle_fwd_rows(_ptr(rq), _ptr(rk), _ptr(rv), t, B, Hq, Hkv, N, d, dv,
-                                    int(bool(causal)), float(eps), cup,
-                                    rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
-                                    rows.shape[0], _dptr(out))
+    with feature_map(phi):
+        rc = _load().lt_oracle_fwd_rows(_ptr(rq), _ptr(rk), _ptr(rv), t, B, Hq, Hkv, N, d, dv,
+                                        int(bool(causal)), float(eps), cup,
+                                        rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                        rows.shape[0], _dptr(out))
     if rc != 0:
         raise ValueError("oracle rejected a row index")
     return out

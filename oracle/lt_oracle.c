@@ -62,11 +62,24 @@
 #define ORC_F32 0
 #define ORC_BF16 1
 #define ORC_F64 2
+#define ORC_F16 3
+
+/* IEEE binary16 bits -> double, exactly: sign, 5-bit exponent (bias 15),
+ * 10-bit fraction; exponent 0 holds the subnormals, 31 infinities and NaN. */
+static double half_to_double(uint16_t h) {
+    const int sign = h >> 15, e = (h >> 10) & 31, m = h & 1023;
+    double x;
+    if (e == 0) x = ldexp((double)m, -24);
+    else if (e == 31) x = m ? NAN : INFINITY;
+    else x = ldexp(1024.0 + m, e - 25);
+    return sign ? -x : x;
+}
 
 /* Read element idx of a raw buffer of the given type, widened to double. */
 static double load_elem(const void *p, int64_t idx, int type) {
     if (type == ORC_F64) return ((const double *)p)[idx];
     if (type == ORC_F32) return (double)((const float *)p)[idx];
+    if (type == ORC_F16) return half_to_double(((const uint16_t *)p)[idx]);
     /* bf16: the 16 stored bits are the high half of an IEEE binary32 */
     uint32_t bits = (uint32_t)((const uint16_t *)p)[idx] << 16;
     float f;
@@ -74,8 +87,27 @@ static double load_elem(const void *p, int64_t idx, int type) {
     return (double)f;
 }
 
-/* phi(x) = ELU(x) + 1 with alpha = 1: x + 1 for x > 0, exp(x) for x <= 0. */
-double lt_oracle_phi(double x) { return x > 0.0 ? x + 1.0 : exp(x); }
+/* The feature map.  Kind 0, the method's: phi(x) = ELU(x) + 1 with alpha =
+ * 1, i.e. x + 1 for x > 0 and exp(x) for x <= 0.  The "lineartile 1.0.0"
+ * page's "Features" list lets the map be replaced; the other maps the CUDA
+ * library offers are kind 1, ReLU: max(x, 0), and kind 2, exp(x).  The kind
+ * in force is set by lt_oracle_set_phi (default 0); the backward forms
+ * support kind 0 only. */
+static int g_phi_kind = 0;
+
+int lt_oracle_set_phi(int kind) {
+    if (kind < 0 || kind > 2) return 1;
+    g_phi_kind = kind;
+    return 0;
+}
+
+static double phi_elu1(double x) { return x > 0.0 ? x + 1.0 : exp(x); }
+
+double lt_oracle_phi(double x) {
+    if (g_phi_kind == 1) return x > 0.0 ? x : 0.0;
+    if (g_phi_kind == 2) return exp(x);
+    return phi_elu1(x);
+}
 
 int lt_oracle_num_threads(void) {
 #ifdef _OPENMP
@@ -407,7 +439,7 @@ int lt_oracle_bwd_quadratic(const void *q, const void *k, const void *v, const v
                             int in_type, double *dq, double *dk, double *dv, int B, int Hq,
                             int Hkv, int N, int d, int dvw, int causal, double eps,
                             const int32_t *cu_seqlens) {
-    if (check_args(B, Hq, Hkv, N, d, dvw, eps)) return 1;
+    if (check_args(B, Hq, Hkv, N, d, dvw, eps) || g_phi_kind != 0) return 1;
     const int G = Hq / Hkv;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
     for (int s = 0; s < B; ++s) {
@@ -485,7 +517,7 @@ int lt_oracle_bwd_recurrent(const void *q, const void *k, const void *v, const v
                             int in_type, double *dq, double *dk, double *dv, int B, int Hq,
                             int Hkv, int N, int d, int dvw, int causal, double eps,
                             const int32_t *cu_seqlens) {
-    if (check_args(B, Hq, Hkv, N, d, dvw, eps)) return 1;
+    if (check_args(B, Hq, Hkv, N, d, dvw, eps) || g_phi_kind != 0) return 1;
     const int G = Hq / Hkv;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
     for (int s = 0; s < B; ++s) {

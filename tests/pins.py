@@ -40,6 +40,64 @@ def pin_phi_is_elu_plus_one():
     assert abs(oracle.phi(-math.log(2.0)) - 0.5) < 1e-16
 
 
+def pin_feature_maps():
+    """The other feature maps against torch: ReLU = max(x, 0), exp; and a
+    forward pass under each map equals the quadratic form written with that
+    map's features (the ELU + 1 pins above hold the forms together)."""
+    xs = np.concatenate([np.linspace(-30, 30, 601), [-1e-12, 0.0, 1e-12]])
+    t = torch.tensor(xs, dtype=torch.float64)
+    for kind, ref in (("relu", torch.relu(t)), ("exp", torch.exp(t))):
+        got = np.array([oracle.phi(x, kind) for x in xs])
+        assert np.allclose(got, ref.numpy(), rtol=1e-15, atol=0), kind
+    assert oracle.phi(-1.0) == math.exp(-1.0)  # the default is back after each call
+    # under map m, phi(Q) phi(K)^T has the same entries as the ELU + 1 form
+    # applied to inputs whose ELU + 1 features are m's features: for ReLU,
+    # x -> x - 1 maps x > 1 onto ELU + 1's linear branch, and zero features
+    # come from very negative inputs (exp underflows to 0)
+    q = np.abs(_rand((1, 9, 2, 4), 150)) + 1.1
+    k = np.abs(_rand((1, 9, 2, 4), 151)) + 1.1
+    k[0, ::3, 0, 1] = -1.0  # relu features 0 here
+    v = _rand((1, 9, 2, 3), 152)
+    kk = np.where(k > 0, k - 1.0, -800.0)
+    for causal in (True, False):
+        a = oracle.fwd_quadratic(q, k, v, causal=causal, eps=1e-6, phi="relu")
+        b = oracle.fwd_quadratic(q - 1.0, kk, v, causal=causal, eps=1e-6)
+        assert np.abs(a - b).max() <= 1e-12 * np.abs(b).max()
+        a = oracle.fwd_recurrent(q, k, v, causal=causal, eps=1e-6, phi="relu")
+        assert np.abs(a - b).max() <= 1e-12 * np.abs(b).max()
+    # exp: phi(x) = e^x for every x equals ELU + 1 on inputs <= 0; shift by a
+    # constant c (e^(x - c) = e^x e^-c cancels between numerator and
+    # denominator when eps = 0)
+    q2, k2 = _rand((1, 7, 2, 3), 153), _rand((1, 7, 2, 3), 154)
+    c = max(q2.max(), k2.max()) + 0.5
+    for causal in (True, False):
+        a = oracle.fwd_recurrent(q2, k2, v[:, :7], causal=causal, eps=0.0, phi="exp")
+        b = oracle.fwd_quadratic(q2 - c, k2 - c, v[:, :7], causal=causal, eps=0.0)
+        assert np.abs(a - b).max() <= 1e-12 * np.abs(b).max()
+
+
+def pin_fp16_inputs_widened_exactly():
+    """fp16 inputs are read as the exact values they hold: the oracle on
+    fp16 tensors equals the oracle on the same values in fp64, subnormals,
+    the largest finite value and signed zero included."""
+    h = torch.tensor([0.0, -0.0, 1.0, -2.5, 65504.0, 6.1e-5, 5.96e-8, -3.0e-6, 0.333],
+                     dtype=torch.float16)
+    assert h.double().tolist() == [float(x) for x in h.double().numpy()]
+    q = (torch.randn(1, 11, 2, 4, generator=torch.Generator().manual_seed(9)) * 0.7).half()
+    k = (torch.randn(1, 11, 2, 4, generator=torch.Generator().manual_seed(10)) * 0.7).half()
+    v = (torch.randn(1, 11, 2, 3, generator=torch.Generator().manual_seed(11))).half()
+    v[0, 3, 0] = h[:3]
+    k[0, 5, 1, :] = h[5:9]
+    for causal in (True, False):
+        a = oracle.fwd_quadratic(q, k, v, causal=causal)
+        b = oracle.fwd_quadratic(q.double(), k.double(), v.double(), causal=causal)
+        assert np.array_equal(a, b)
+    vv = torch.tensor([[[[1.0, 65504.0, 5.96e-8]]]], dtype=torch.float16)
+    o = oracle.fwd_recurrent(torch.zeros(1, 1, 1, 2).half(), torch.zeros(1, 1, 1, 2).half(), vv,
+                             eps=0.0)
+    assert o.tolist() == [[[[1.0, 65504.0, float(torch.tensor(5.96e-8).half().double())]]]]
+
+
 def _hand_2x2_inputs(g):
     q = np.array(g["q"], dtype=np.float64).reshape(1, 2, 1, 2)
     k = np.array([[1.0, 0.0], [0.0, -math.log(2.0)]]).reshape(1, 2, 1, 2)
@@ -466,6 +524,8 @@ def pin_bwd_packed_and_gqa():
 
 ALL_PINS = [
     pin_phi_is_elu_plus_one,
+    pin_feature_maps,
+    pin_fp16_inputs_widened_exactly,
     pin_hand_2x2,
     pin_hand_3tok,
     pin_two_forms_agree,

@@ -15,6 +15,14 @@ import pins
 MUTANTS = [
     ("phi without the +1", "return x > 0.0 ? x + 1.0 : exp(x);", "return x > 0.0 ? x : exp(x);"),
     ("phi with exp(-x)", "return x > 0.0 ? x + 1.0 : exp(x);", "return x > 0.0 ? x + 1.0 : exp(-x);"),
+    ("relu map keeps negative inputs", "if (g_phi_kind == 1) return x > 0.0 ? x : 0.0;",
+     "if (g_phi_kind == 1) return x;"),
+    ("exp map falls back to ELU + 1", "if (g_phi_kind == 2) return exp(x);",
+     "if (g_phi_kind == 2) return phi_elu1(x);"),
+    ("fp16 exponent bias off by one", "else x = ldexp(1024.0 + m, e - 25);",
+     "else x = ldexp(1024.0 + m, e - 24);"),
+    ("fp16 subnormals scaled as normals", "if (e == 0) x = ldexp((double)m, -24);",
+     "if (e == 0) x = ldexp(1024.0 + m, -25);"),
     ("exclusive causal sum", "causal ? i + 1 : n", "causal ? i : n"),
     ("eps dropped", "(den + eps)", "(den)"),
     ("eps dropped (recurrent)", "double den = eps;", "double den = 0.0;"),
