@@ -15,7 +15,8 @@ LIB_PATH = os.path.join(_HERE, "liblt.so")
 
 LT_OK, LT_ERR_INVALID_ARG, LT_ERR_UNSUPPORTED, LT_ERR_CUDA = 0, 1, 2, 3
 LT_ERR_DEVICE_TIMEOUT, LT_ERR_DEVICE_BAD_SEQLENS, LT_ERR_SCRATCH_TOO_SMALL = 4, 5, 6
-LT_F32, LT_BF16 = 0, 1
+LT_F32, LT_BF16, LT_F16 = 0, 1, 2
+FEATURE_MAPS = {"elu1": 0, "relu": 1, "exp": 2}
 LT_SCHED_AUTO, LT_SCHED_TWO_LAUNCH, LT_SCHED_GENERAL = 0, 1, 2
 _SCHED = {"auto": LT_SCHED_AUTO, "two_launch": LT_SCHED_TWO_LAUNCH, "general": LT_SCHED_GENERAL}
 
@@ -24,7 +25,7 @@ EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_fwd_noalloc", "lt_linear_attn_
             "lt_linear_attn_fwd_state", "lt_linear_attn_decode_step", "lt_status_string",
             "lt_get_last_device_error", "lt_abi_version", "lt_selftest_wait_timeout",
             "lt_debug_set_schedule", "lt_linear_attn_state", "lt_linear_attn_state_carry",
-            "lt_linear_attn_bwd")
+            "lt_linear_attn_bwd", "lt_linear_attn_fwd_ex")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("liblt.so is not built (run `python -m "
@@ -35,6 +36,8 @@ _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 lib.lt_linear_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _vp,
                                    _i]
 lib.lt_linear_attn_fwd.restype = _i
+lib.lt_linear_attn_fwd_ex.argtypes = lib.lt_linear_attn_fwd.argtypes + [_i]
+lib.lt_linear_attn_fwd_ex.restype = _i
 lib.lt_linear_attn_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
                                            _vp, _vp]
 lib.lt_linear_attn_fwd_noalloc.restype = _i
@@ -83,7 +86,9 @@ def _dtype_code(t):
         return LT_BF16
     if t == torch.float32:
         return LT_F32
-    raise TypeError("unsupported dtype %s (bfloat16 or float32)" % t)
+    if t == torch.float16:
+        return LT_F16
+    raise TypeError("unsupported dtype %s (bfloat16, float16 or float32)" % t)
 
 
 def _stream_handle(stream, device):
@@ -96,11 +101,14 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
-def linear_attn_fwd(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, out=None, stream=None):
+def linear_attn_fwd(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, out=None, stream=None,
+                    feature_map="elu1"):
     """O = linear attention of (q, k, v); see include/lt_linear_attn.h.
 
     Dense: q [B, N, H_q, d], k [B, N, H_kv, d], v [B, N, H_kv, dv].
     Packed: q [N, H_q, d] ... with cu_seqlens (int32, device, B+1 entries).
+    dtype bfloat16, float16 or float32.  feature_map: "elu1" (ELU + 1, the
+    method's), "relu" or "exp" (lt_linear_attn_fwd_ex).
     Returns out with q's dtype, shape [..., H_q, dv].
     """
     if cu_seqlens is None:
@@ -119,9 +127,12 @@ def linear_attn_fwd(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, out=None, s
             raise ValueError("q, k, v must be contiguous")
     if out is None:
         out = torch.empty(oshape, dtype=q.dtype, device=q.device)
-    _check(lib.lt_linear_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, Hq, Hkv, N, d, dv,
-                                  int(bool(causal)), float(eps), _ptr(cu_seqlens),
-                                  _stream_handle(stream, q.device), _dtype_code(q.dtype)))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, Hq, Hkv, N, d, dv, int(bool(causal)),
+            float(eps), _ptr(cu_seqlens), _stream_handle(stream, q.device), _dtype_code(q.dtype))
+    if feature_map == "elu1":
+        _check(lib.lt_linear_attn_fwd(*args))
+    else:
+        _check(lib.lt_linear_attn_fwd_ex(*args, FEATURE_MAPS[feature_map]))
     return out
 
 

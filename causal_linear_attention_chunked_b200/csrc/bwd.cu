@@ -448,6 +448,7 @@ extern "C" lt_status_t lt_linear_attn_bwd(const void* q, const void* k, const vo
   lt_status_t st = lt::check_fwd(q, k, v, const_cast<void*>(dout), B, H_q, H_kv, N, d, dv_w,
                                  causal, eps, cu_seqlens, dtype, &p);
   if (st != LT_OK) return st;
+  if (dtype == LT_F16) return LT_ERR_UNSUPPORTED;
   if (!dq || !dk || !dv) return LT_ERR_INVALID_ARG;
   const uintptr_t mis = reinterpret_cast<uintptr_t>(dq) | reinterpret_cast<uintptr_t>(dk) |
                         reinterpret_cast<uintptr_t>(dv);

@@ -68,7 +68,7 @@ struct GenArgs : FwdArgs {
 // phi in place over a full [kChunk x (NBOX*64)] bf16 tile by 128 threads, as
 // a loop with four 16-byte pieces in flight per thread (compact code: this
 // kernel's warp roles share each sub-partition's instruction cache)
-template <int NBOX>
+template <int NBOX, class VAR>
 __device__ __forceinline__ void phi_tile_loop(uint8_t* tile, int tid) {
   constexpr int kIt = kChunk * NBOX * 8 / 128;
   static_assert(kIt % 4 == 0, "pieces per thread");
@@ -80,10 +80,10 @@ __device__ __forceinline__ void phi_tile_loop(uint8_t* tile, int tid) {
     for (int u = 0; u < 4; ++u) v[u] = p[(i + u) * 128];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      v[u].x = phi_bf16x2(v[u].x);
-      v[u].y = phi_bf16x2(v[u].y);
-      v[u].z = phi_bf16x2(v[u].z);
-      v[u].w = phi_bf16x2(v[u].w);
+      v[u].x = phi2<VAR>(v[u].x);
+      v[u].y = phi2<VAR>(v[u].y);
+      v[u].z = phi2<VAR>(v[u].z);
+      v[u].w = phi2<VAR>(v[u].w);
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) p[(i + u) * 128] = v[u];
@@ -160,7 +160,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
   return r;
 }
 
-template <int D, int DV>
+template <int D, int DV, class VAR>
 __global__ void __launch_bounds__(kThreads, 1)
     lt_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -382,8 +382,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // V of chunk c is ready as loaded, except in a ragged chunk, whose
         // tail rows the phi warps zero first (only the block's last chunk
         // can be ragged, so its v_xf barrier completes exactly one phase)
+        // (fp16 inputs: every V tile is converted to the bf16 operand, and
+        // v_xf completes one phase per use of the stage)
         auto v_ready = [&](int c) {
           const int vs = c % K::NKV;
+          if (VAR::kIn != kInBf16) return mbar_test(&bars.v_xf[vs], (c / K::NKV) & 1);
           return n - c * kChunk < kChunk ? mbar_test(&bars.v_xf[vs], 0)
                                          : mbar_test(&bars.v_full[vs], (c / K::NKV) & 1);
         };
@@ -468,7 +471,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int st = c % K::NKV;
             const uint32_t par = (c / K::NKV) & 1;
             ok = mbar_wait(&bars.k_xf[st], par, abort_flag, a.err, kWaitLimitNs) &&
-                 (n - c * kChunk < kChunk
+                 (VAR::kIn != kInBf16
+                      ? mbar_wait(&bars.v_xf[st], par, abort_flag, a.err, kWaitLimitNs)
+                  : n - c * kChunk < kChunk
                       ? mbar_wait(&bars.v_xf[st], 0, abort_flag, a.err, kWaitLimitNs)
                       : mbar_wait(&bars.v_full[st], par, abort_flag, a.err, kWaitLimitNs));
             if (!ok) break;
@@ -509,15 +514,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&bars.k_full[st], par, abort_flag, a.err, kWaitLimitNs)) return false;
       const int valid = min(kChunk, n - c * kChunk);
       if (valid >= kChunk)
-        phi_tile_loop<D / 64>(sK + st * K::KT, x);
+        phi_tile_loop<D / 64, VAR>(sK + st * K::KT, x);
       else
-        xf_tile<D / 64, 128>(sK + st * K::KT, valid, true, x);
+        xf_tile<D / 64, 128, VAR>(sK + st * K::KT, valid, true, x);
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
       if (x == 0) mbar_arrive(&bars.k_xf[st]);
-      if (valid < kChunk) {
+      if (valid < kChunk || VAR::kIn != kInBf16) {
         if (!mbar_wait(&bars.v_full[st], par, abort_flag, a.err, kWaitLimitNs)) return false;
-        xf_tile<DV / 64, 128>(sV + st * K::VT, valid, false, x);
+        xf_tile<DV / 64, 128, VAR>(sV + st * K::VT, valid, false, x);
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (x == 0) mbar_arrive(&bars.v_xf[st]);
@@ -529,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = i % K::NQ;
       if (!mbar_wait(&bars.q_full[st], (i / K::NQ) & 1, abort_flag, a.err, kWaitLimitNs))
         return false;
-      phi_tile_loop<D / 64>(sQ + st * K::QT, x);
+      phi_tile_loop<D / 64, VAR>(sQ + st * K::QT, x);
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
       if (x == 0) mbar_arrive(&bars.q_xf[st]);
@@ -764,10 +769,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4)
           *reinterpret_cast<uint4*>(stg + lane * 64 + ((q4 ^ ((lane >> 1) & 3)) << 4)) =
-              make_uint4(pack_bf16x2(r[q4 * 8 + 0] * inv, r[q4 * 8 + 1] * inv),
-                         pack_bf16x2(r[q4 * 8 + 2] * inv, r[q4 * 8 + 3] * inv),
-                         pack_bf16x2(r[q4 * 8 + 4] * inv, r[q4 * 8 + 5] * inv),
-                         pack_bf16x2(r[q4 * 8 + 6] * inv, r[q4 * 8 + 7] * inv));
+              make_uint4(pack_out<VAR>(r[q4 * 8 + 0] * inv, r[q4 * 8 + 1] * inv),
+                         pack_out<VAR>(r[q4 * 8 + 2] * inv, r[q4 * 8 + 3] * inv),
+                         pack_out<VAR>(r[q4 * 8 + 4] * inv, r[q4 * 8 + 5] * inv),
+                         pack_out<VAR>(r[q4 * 8 + 6] * inv, r[q4 * 8 + 7] * inv));
         __syncwarp();
 #pragma unroll
         for (int k8 = 0; k8 < 4; ++k8) {
@@ -816,16 +821,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int DV>
+template <int D, int DV, class VAR = VarDefault>
 cudaError_t launch_fwd(const FwdLaunch& p, int nb, const float* ws, bool carry_pre,
                        cudaStream_t stream) {
   using K = Cfg<D, DV>;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
-      !make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64) ||
-      !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64))
+  const bool f16 = VAR::kIn == kInF16;
+  if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64, f16) ||
+      !make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64, f16) ||
+      !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64, f16))
     return cudaErrorInvalidValue;
-  auto kern = lt_fwd_bf16_kernel<D, DV>;
+  auto kern = lt_fwd_bf16_kernel<D, DV, VAR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
   if (e != cudaSuccess) return e;
   GenArgs a;
@@ -851,8 +857,27 @@ cudaError_t launch_fwd(const FwdLaunch& p, int nb, const float* ws, bool carry_p
 
 }  // namespace
 
+template <int D, int DV>
+static cudaError_t launch_var(const FwdLaunch& p, int nb, const float* ws, bool pre,
+                              cudaStream_t stream) {
+  switch (p.in_f16 * 4 + p.phi) {
+    case 0: return launch_fwd<D, DV, Var<kInBf16, kPhiElu1>>(p, nb, ws, pre, stream);
+    case 1: return launch_fwd<D, DV, Var<kInBf16, kPhiRelu>>(p, nb, ws, pre, stream);
+    case 2: return launch_fwd<D, DV, Var<kInBf16, kPhiExp>>(p, nb, ws, pre, stream);
+    case 4: return launch_fwd<D, DV, Var<kInF16, kPhiElu1>>(p, nb, ws, pre, stream);
+    case 5: return launch_fwd<D, DV, Var<kInF16, kPhiRelu>>(p, nb, ws, pre, stream);
+    case 6: return launch_fwd<D, DV, Var<kInF16, kPhiExp>>(p, nb, ws, pre, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
 static cudaError_t launch_seq(const FwdLaunch& p, int nb, const float* ws, bool pre,
                               cudaStream_t stream) {
+  if (p.in_f16 || p.phi) {  // variants: d = dv = 64 or 128
+    if (p.d == 64 && p.dv == 64) return launch_var<64, 64>(p, nb, ws, pre, stream);
+    if (p.d == 128 && p.dv == 128) return launch_var<128, 128>(p, nb, ws, pre, stream);
+    return cudaErrorInvalidValue;
+  }
   if (p.d == 64 && p.dv == 64) return launch_fwd<64, 64>(p, nb, ws, pre, stream);
   if (p.d == 128 && p.dv == 128) return launch_fwd<128, 128>(p, nb, ws, pre, stream);
   if (p.d == 64 && p.dv == 128) return launch_fwd<64, 128>(p, nb, ws, pre, stream);
@@ -874,7 +899,8 @@ cudaError_t launch_fwd_bf16_seq_pre(const FwdLaunch& p, int nb, const float* ws,
 // block scan where the one-launch path applies, or run the general kernel on
 // d = dv = 64 too (tests and ablations).
 static bool use_block_fused(const FwdLaunch& p, int nb, int num_sms) {
-  return sched_kernel() == LT_SCHED_AUTO && block_fused_supported(p, nb, num_sms);
+  return sched_kernel() == LT_SCHED_AUTO && !p.in_f16 && !p.phi &&
+         block_fused_supported(p, nb, num_sms);
 }
 
 cudaError_t launch_fwd_bf16_ws(const FwdLaunch& p, int nb, float* ws, cudaStream_t stream) {
@@ -885,7 +911,8 @@ cudaError_t launch_fwd_bf16_ws(const FwdLaunch& p, int nb, float* ws, cudaStream
     e = launch_block_state(p, nb, ws, stream);
     if (e != cudaSuccess) return e;
   }
-  if (sched_kernel() != LT_SCHED_GENERAL && block_supported(p))
+  // fp16 inputs and the other feature maps run the general kernel
+  if (sched_kernel() != LT_SCHED_GENERAL && !p.in_f16 && !p.phi && block_supported(p))
     return launch_fwd_bf16_block(p, nb, ws, stream);
   return launch_fwd_bf16_seq(p, nb, ws, stream);
 }

@@ -21,7 +21,9 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 // phi in place over a [kChunk x (NBOX*64)] bf16 tile (rows of 128-byte
 // boxes, swizzled; phi is elementwise so the swizzle does not matter).
 // Rows >= valid are zeroed.  NT threads (tid in [0, NT)).
-template <int NBOX, int NT = 128>
+// Without apply_phi the rows below `valid` are only converted to the bf16
+// operand type (nothing to do for bf16 inputs).
+template <int NBOX, int NT = 128, class VAR = VarDefault>
 __device__ __forceinline__ void xf_tile(uint8_t* tile, int valid, bool apply_phi, int tid) {
   constexpr int kChunks = kChunk * NBOX * 8;  // 16-byte pieces
 #pragma unroll 4
@@ -33,10 +35,15 @@ __device__ __forceinline__ void xf_tile(uint8_t* tile, int valid, bool apply_phi
     if (row >= valid) {
       v = make_uint4(0u, 0u, 0u, 0u);
     } else if (apply_phi) {
-      v.x = phi_bf16x2(v.x);
-      v.y = phi_bf16x2(v.y);
-      v.z = phi_bf16x2(v.z);
-      v.w = phi_bf16x2(v.w);
+      v.x = phi2<VAR>(v.x);
+      v.y = phi2<VAR>(v.y);
+      v.z = phi2<VAR>(v.z);
+      v.w = phi2<VAR>(v.w);
+    } else if (VAR::kIn != kInBf16) {
+      v.x = conv2<VAR>(v.x);
+      v.y = conv2<VAR>(v.y);
+      v.z = conv2<VAR>(v.z);
+      v.w = conv2<VAR>(v.w);
     } else {
       continue;
     }
@@ -47,7 +54,7 @@ __device__ __forceinline__ void xf_tile(uint8_t* tile, int valid, bool apply_phi
 // phi in place over a full [kChunk x (NBOX*64)] bf16 tile (every row
 // valid).  The NBOX boxes are contiguous, so thread t takes the 16-byte
 // pieces t, t + NT, ...; all loads are issued before the arithmetic.
-template <int NBOX, int NT>
+template <int NBOX, int NT, class VAR = VarDefault>
 __device__ __forceinline__ void phi_tile_full(uint8_t* tile, int tid) {
   constexpr int kPieces = kChunk * NBOX * 8;
   constexpr int kIt = (kPieces + NT - 1) / NT;
@@ -60,10 +67,10 @@ __device__ __forceinline__ void phi_tile_full(uint8_t* tile, int tid) {
     if (i < kIt - 1 || last) v[i] = p[i * NT];
 #pragma unroll
   for (int i = 0; i < kIt; ++i) {
-    v[i].x = phi_bf16x2(v[i].x);
-    v[i].y = phi_bf16x2(v[i].y);
-    v[i].z = phi_bf16x2(v[i].z);
-    v[i].w = phi_bf16x2(v[i].w);
+    v[i].x = phi2<VAR>(v[i].x);
+    v[i].y = phi2<VAR>(v[i].y);
+    v[i].z = phi2<VAR>(v[i].z);
+    v[i].w = phi2<VAR>(v[i].w);
   }
 #pragma unroll
   for (int i = 0; i < kIt; ++i)
@@ -72,12 +79,12 @@ __device__ __forceinline__ void phi_tile_full(uint8_t* tile, int tid) {
 
 // phi (apply_phi) and zeroing of the rows >= valid: the fast path for full
 // tiles, the general loop for the ragged last chunk.
-template <int NBOX, int NT>
+template <int NBOX, int NT, class VAR = VarDefault>
 __device__ __forceinline__ void prep_tile(uint8_t* tile, int valid, bool apply_phi, int tid) {
   if (valid >= kChunk) {
-    if (apply_phi) phi_tile_full<NBOX, NT>(tile, tid);
+    if (apply_phi) phi_tile_full<NBOX, NT, VAR>(tile, tid);
   } else {
-    xf_tile<NBOX, NT>(tile, valid, apply_phi, tid);
+    xf_tile<NBOX, NT, VAR>(tile, valid, apply_phi, tid);
   }
 }
 
@@ -113,7 +120,7 @@ __device__ __forceinline__ void init_ones_block(uint8_t* ones, int tid, int nthr
 
 // host side
 inline bool make_tmap_3d(CUtensorMap* m, const void* base, int inner, int heads, long long tokens,
-                  int box_inner) {
+                  int box_inner, bool f16 = false) {
   using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -132,8 +139,9 @@ inline bool make_tmap_3d(CUtensorMap* m, const void* base, int inner, int heads,
   const cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * heads * 2};
   const cuuint32_t box[3] = {(cuuint32_t)box_inner, 1u, (cuuint32_t)kChunk};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
-  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  const CUtensorMapDataType type =
+      f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return encode(m, type, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -23,7 +23,13 @@ namespace {
 constexpr int kC = 32;  // tokens per chunk
 constexpr int kT = 256; // threads
 
-__device__ __forceinline__ float phi_acc(float x) { return x > 0.0f ? x + 1.0f : expf(x); }
+// the feature maps in fp32: ELU + 1 (the method's), ReLU, exp
+template <int PHI>
+__device__ __forceinline__ float phi_acc(float x) {
+  if constexpr (PHI == kPhiElu1) return x > 0.0f ? x + 1.0f : expf(x);
+  else if constexpr (PHI == kPhiRelu) return fmaxf(x, 0.0f);
+  else return expf(x);
+}
 
 struct F32Args {
   const float* q;
@@ -43,7 +49,7 @@ struct F32Args {
   float* z_out;
 };
 
-template <int D, int DV>
+template <int D, int DV, int PHI>
 __global__ void __launch_bounds__(kT) lt_fwd_f32_kernel(const F32Args a) {
   extern __shared__ float sm[];
   float* S = sm;                 // D x DV
@@ -89,7 +95,7 @@ __global__ void __launch_bounds__(kT) lt_fwd_f32_kernel(const F32Args a) {
     const int valid = min(kC, n - c * kC);
     for (int e = tid; e < kC * D; e += kT) {
       const int r = e / D, col = e % D;
-      pk[e] = r < valid ? phi_acc(a.k[((size_t)(t0 + c * kC + r) * a.Hkv + g) * D + col]) : 0.0f;
+      pk[e] = r < valid ? phi_acc<PHI>(a.k[((size_t)(t0 + c * kC + r) * a.Hkv + g) * D + col]) : 0.0f;
     }
     for (int e = tid; e < kC * DV; e += kT) {
       const int r = e / DV, col = e % DV;
@@ -100,7 +106,7 @@ __global__ void __launch_bounds__(kT) lt_fwd_f32_kernel(const F32Args a) {
     const int valid = min(kC, n - c * kC);
     for (int e = tid; e < kC * D; e += kT) {
       const int r = e / D, col = e % D;
-      pq[e] = r < valid ? phi_acc(a.q[((size_t)(t0 + c * kC + r) * a.Hq + h) * D + col]) : 0.0f;
+      pq[e] = r < valid ? phi_acc<PHI>(a.q[((size_t)(t0 + c * kC + r) * a.Hq + h) * D + col]) : 0.0f;
     }
   };
   // S += phi(K_c)^T V_c ; z += sum_rows phi(K_c)
@@ -179,11 +185,11 @@ __global__ void __launch_bounds__(kT) lt_fwd_f32_kernel(const F32Args a) {
   }
 }
 
-template <int D, int DV>
+template <int D, int DV, int PHI>
 cudaError_t launch(const FwdLaunch& p, const float* s0, const float* z0, float* s_out,
                    float* z_out, cudaStream_t stream) {
   const int smem = (D * DV + D + 2 * kC * D + kC * DV + kC * kC + kC) * 4;
-  auto kern = lt_fwd_f32_kernel<D, DV>;
+  auto kern = lt_fwd_f32_kernel<D, DV, PHI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   F32Args a;
@@ -208,14 +214,23 @@ cudaError_t launch(const FwdLaunch& p, const float* s0, const float* z0, float* 
   return cudaGetLastError();
 }
 
+template <int PHI>
+cudaError_t launch_widths(const FwdLaunch& p, const float* s0, const float* z0, float* s_out,
+                          float* z_out, cudaStream_t stream) {
+  if (p.d == 64 && p.dv == 64) return launch<64, 64, PHI>(p, s0, z0, s_out, z_out, stream);
+  if (p.d == 128 && p.dv == 128) return launch<128, 128, PHI>(p, s0, z0, s_out, z_out, stream);
+  if (p.d == 64 && p.dv == 128) return launch<64, 128, PHI>(p, s0, z0, s_out, z_out, stream);
+  if (p.d == 128 && p.dv == 64) return launch<128, 64, PHI>(p, s0, z0, s_out, z_out, stream);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 cudaError_t launch_fwd_f32_state(const FwdLaunch& p, const float* s0, const float* z0,
                                  float* s_out, float* z_out, cudaStream_t stream) {
-  if (p.d == 64 && p.dv == 64) return launch<64, 64>(p, s0, z0, s_out, z_out, stream);
-  if (p.d == 128 && p.dv == 128) return launch<128, 128>(p, s0, z0, s_out, z_out, stream);
-  if (p.d == 64 && p.dv == 128) return launch<64, 128>(p, s0, z0, s_out, z_out, stream);
-  if (p.d == 128 && p.dv == 64) return launch<128, 64>(p, s0, z0, s_out, z_out, stream);
+  if (p.phi == kPhiRelu) return launch_widths<kPhiRelu>(p, s0, z0, s_out, z_out, stream);
+  if (p.phi == kPhiExp) return launch_widths<kPhiExp>(p, s0, z0, s_out, z_out, stream);
+  return launch_widths<kPhiElu1>(p, s0, z0, s_out, z_out, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -64,7 +64,7 @@ bool width_ok(int w) { return w == 64 || w == 128; }
 lt_status_t check_fwd_impl(const void* q, const void* k, const void* v, void* out, int B, int H_q,
                       int H_kv, int N, int d, int dv, int causal, float eps,
                       const int32_t* cu_seqlens, lt_dtype_t dtype, lt::FwdLaunch* p) {
-  if (dtype != LT_F32 && dtype != LT_BF16) return LT_ERR_UNSUPPORTED;
+  if (dtype != LT_F32 && dtype != LT_BF16 && dtype != LT_F16) return LT_ERR_UNSUPPORTED;
   if (!q || !k || !v || !out) return LT_ERR_INVALID_ARG;
   if (B <= 0 || H_q <= 0 || H_kv <= 0 || N <= 0) return LT_ERR_INVALID_ARG;
   if (H_q % H_kv != 0) return LT_ERR_INVALID_ARG;
@@ -80,12 +80,13 @@ lt_status_t check_fwd_impl(const void* q, const void* k, const void* v, void* ou
   if (!is_device_ptr(q) || !is_device_ptr(k) || !is_device_ptr(v) || !is_device_ptr(out) ||
       (cu_seqlens && !is_device_ptr(cu_seqlens)))
     return LT_ERR_INVALID_ARG;
-  const size_t es = dtype == LT_BF16 ? 2 : 4;
+  const size_t es = dtype == LT_F32 ? 4 : 2;
   const size_t nq = (size_t)tokens * H_q * d * es, nk = (size_t)tokens * H_kv * d * es;
   const size_t nv = (size_t)tokens * H_kv * dv * es, no = (size_t)tokens * H_q * dv * es;
   if (overlaps(out, no, q, nq) || overlaps(out, no, k, nk) || overlaps(out, no, v, nv))
     return LT_ERR_INVALID_ARG;
   *p = lt::FwdLaunch{};
+  p->in_f16 = dtype == LT_F16 ? 1 : 0;
   p->q = q;
   p->k = k;
   p->v = v;
@@ -158,21 +159,36 @@ lt_status_t lt_linear_attn_fwd(const void* q, const void* k, const void* v, void
                                int H_q, int H_kv, int N, int d, int dv, int causal, float eps,
                                const int32_t* cu_seqlens, lt_stream_t stream,
                                lt_dtype_t dtype) {
+  return lt_linear_attn_fwd_ex(q, k, v, out, B, H_q, H_kv, N, d, dv, causal, eps, cu_seqlens,
+                               stream, dtype, LT_PHI_ELU1);
+}
+
+lt_status_t lt_linear_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, int B,
+                                  int H_q, int H_kv, int N, int d, int dv, int causal, float eps,
+                                  const int32_t* cu_seqlens, lt_stream_t stream,
+                                  lt_dtype_t dtype, lt_feature_map_t phi) {
+  // the feature map, and the widths of the tensor-core path's variants
+  // (fp16 I/O, the other maps): d = dv = 64 or 128
+  if (phi != LT_PHI_ELU1 && phi != LT_PHI_RELU && phi != LT_PHI_EXP) return LT_ERR_INVALID_ARG;
+  if ((dtype == LT_F16 || (dtype == LT_BF16 && phi != LT_PHI_ELU1)) &&
+      !(d == dv && (d == 64 || d == 128)))
+    return LT_ERR_UNSUPPORTED;
   lt::FwdLaunch p;
   const lt_status_t st =
       check_fwd_impl(q, k, v, out, B, H_q, H_kv, N, d, dv, causal, eps, cu_seqlens, dtype, &p);
   if (st != LT_OK) return st;
+  p.phi = (int)phi;
   p.err = device_error_word();
   if (!p.err) return LT_ERR_CUDA;
-  const cudaError_t e = dtype == LT_BF16 ? lt::launch_fwd_bf16(p, (cudaStream_t)stream)
-                                         : lt::launch_fwd_f32(p, (cudaStream_t)stream);
+  const cudaError_t e = dtype == LT_F32 ? lt::launch_fwd_f32(p, (cudaStream_t)stream)
+                                        : lt::launch_fwd_bf16(p, (cudaStream_t)stream);
   return e == cudaSuccess ? LT_OK : LT_ERR_CUDA;
 }
 
 lt_status_t lt_linear_attn_fwd_plan(int B, int H_q, int H_kv, int N, int d, int dv, int causal,
                                     int packed, lt_dtype_t dtype, int num_sms, int* blocks,
                                     int* launches, size_t* workspace_bytes) {
-  if (dtype != LT_F32 && dtype != LT_BF16) return LT_ERR_UNSUPPORTED;
+  if (dtype != LT_F32 && dtype != LT_BF16 && dtype != LT_F16) return LT_ERR_UNSUPPORTED;
   if (!blocks || !launches || !workspace_bytes) return LT_ERR_INVALID_ARG;
   if (B <= 0 || H_q <= 0 || H_kv <= 0 || N <= 0 || H_q % H_kv != 0) return LT_ERR_INVALID_ARG;
   if (B > 65535 || H_kv > 65535) return LT_ERR_INVALID_ARG;
@@ -201,6 +217,8 @@ lt_status_t lt_linear_attn_fwd_plan(int B, int H_q, int H_kv, int N, int d, int 
   p.dv = dv;
   p.causal = causal;
   p.total_tokens = tokens;
+  p.in_f16 = dtype == LT_F16 ? 1 : 0;
+  if (p.in_f16 && !(d == dv && (d == 64 || d == 128))) return LT_ERR_UNSUPPORTED;
   lt::plan_fwd_bf16(p, num_sms, blocks, launches, workspace_bytes);
   return LT_OK;
 }
@@ -214,6 +232,7 @@ lt_status_t lt_linear_attn_fwd_state(const void* q, const void* k, const void* v
   const lt_status_t st =
       check_fwd_impl(q, k, v, out, B, H_q, H_kv, N, d, dv, causal, eps, cu_seqlens, dtype, &p);
   if (st != LT_OK) return st;
+  if (dtype == LT_F16) return LT_ERR_UNSUPPORTED;
   if ((S0 == nullptr) != (z0 == nullptr) || (S_out == nullptr) != (z_out == nullptr))
     return LT_ERR_INVALID_ARG;
   if ((S0 && (!aligned16(S0) || (reinterpret_cast<uintptr_t>(z0) & 3u))) ||

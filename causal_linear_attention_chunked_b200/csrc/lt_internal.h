@@ -18,6 +18,8 @@ struct FwdLaunch {
   float eps;
   long long total_tokens;  // B*N (dense) or N (packed)
   int* err;                // device error word
+  int in_f16;              // 1: fp16 inputs and output (bf16 tensor-core operands)
+  int phi;                 // feature map (lt_feature_map_t); 0 = ELU + 1
 };
 
 struct DecodeLaunch {

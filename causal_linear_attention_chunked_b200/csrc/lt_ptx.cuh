@@ -8,6 +8,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include <cooperative_groups.h>
@@ -316,6 +317,82 @@ __device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
   const float elo = ex2_approx(lo * 1.4426950408889634f);
   const float ehi = ex2_approx(hi * 1.4426950408889634f);
   return pack_bf16x2(lo > 0.0f ? lo + 1.0f : elo, hi > 0.0f ? hi + 1.0f : ehi);
+}
+
+// ------------------------------------------------ kernel variants
+// Input element type and feature map of a forward kernel, as compile-time
+// parameters.  Var<kInBf16, kPhiElu1> is the method's default (bf16 I/O,
+// phi = ELU + 1) and compiles to the code above.  The tensor-core operands
+// are bf16 for every variant: fp16 inputs are widened exactly to fp32,
+// transformed, and rounded once to bf16 (V included); outputs take the
+// input's type.
+enum : int { kInBf16 = 0, kInF16 = 1 };
+enum : int { kPhiElu1 = 0, kPhiRelu = 1, kPhiExp = 2 };
+
+template <int IN, int PHI>
+struct Var {
+  static constexpr int kIn = IN;
+  static constexpr int kPhi = PHI;
+  static constexpr bool kDefault = IN == kInBf16 && PHI == kPhiElu1;
+};
+using VarDefault = Var<kInBf16, kPhiElu1>;
+
+// two packed 16-bit input elements -> fp32 (the even element in the low half)
+template <int IN>
+__device__ __forceinline__ float2 unpack_in(uint32_t u) {
+  if constexpr (IN == kInBf16) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+  } else {
+    __half2 h = *reinterpret_cast<__half2*>(&u);
+    return __half22float2(h);
+  }
+}
+
+// the feature maps, fp32 in and out: ELU + 1 (x + 1 for x > 0, e^x else),
+// ReLU (max(x, 0)), exp (e^x); e^x as 2^(x log2 e) on the MUFU
+template <int PHI>
+__device__ __forceinline__ float feat(float x) {
+  if constexpr (PHI == kPhiElu1) {
+    const float e = ex2_approx(x * 1.4426950408889634f);
+    return x > 0.0f ? x + 1.0f : e;
+  } else if constexpr (PHI == kPhiRelu) {
+    return fmaxf(x, 0.0f);
+  } else {
+    return ex2_approx(x * 1.4426950408889634f);
+  }
+}
+
+// phi on two packed inputs -> two packed bf16 operands
+template <class V>
+__device__ __forceinline__ uint32_t phi2(uint32_t x) {
+  if constexpr (V::kDefault) {
+    return phi_bf16x2(x);
+  } else {
+    const float2 f = unpack_in<V::kIn>(x);
+    return pack_bf16x2(feat<V::kPhi>(f.x), feat<V::kPhi>(f.y));
+  }
+}
+
+// two packed inputs (V tiles) -> two packed bf16 operands
+template <class V>
+__device__ __forceinline__ uint32_t conv2(uint32_t x) {
+  if constexpr (V::kIn == kInBf16) {
+    return x;
+  } else {
+    const float2 f = unpack_in<V::kIn>(x);
+    return pack_bf16x2(f.x, f.y);
+  }
+}
+
+// two fp32 results -> two packed outputs of the input's type
+template <class V>
+__device__ __forceinline__ uint32_t pack_out(float lo, float hi) {
+  if constexpr (V::kIn == kInBf16) {
+    return pack_bf16x2(lo, hi);
+  } else {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
 }
 
 // Feature map of the method: phi(x) = ELU(x) + 1 = x + 1 (x > 0), e^x (x <= 0).

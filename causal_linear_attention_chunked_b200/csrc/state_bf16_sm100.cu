@@ -52,7 +52,7 @@ struct StateArgs {
   int* err;
 };
 
-template <int D, int DV>
+template <int D, int DV, class VAR>
 __global__ void __launch_bounds__(kThreads, 1)
     lt_block_state_kernel(const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const StateArgs a) {
@@ -177,8 +177,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = mbar_wait(&full[st], (i / K::NS) & 1, abort_flag, a.err, kWaitLimitNs);
       if (!ok) break;
       const int valid = min(kChunk, ntok - c * kChunk);
-      prep_tile<D / 64, kXf>(sK + st * K::KVT, valid, true, x);
-      if (valid < kChunk) xf_tile<DV / 64, kXf>(sV + st * K::KVT, valid, false, x);
+      prep_tile<D / 64, kXf, VAR>(sK + st * K::KVT, valid, true, x);
+      if (valid < kChunk || VAR::kIn != kInBf16)
+        xf_tile<DV / 64, kXf, VAR>(sV + st * K::KVT, valid, false, x);
       fence_proxy_async_smem();
       named_bar_sync(1, kXf);
       if (x == 0) mbar_arrive(&xf[st]);
@@ -218,13 +219,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int DV>
+template <int D, int DV, class VAR = VarDefault>
 cudaError_t launch(const FwdLaunch& p, int nb, int nblocks_launch, float* ws,
                    cudaStream_t stream) {
   using K = SCfg<D, DV>;
   CUtensorMap tk, tv;
-  if (!make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64) ||
-      !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64))
+  const bool f16 = VAR::kIn == kInF16;
+  if (!make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64, f16) ||
+      !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64, f16))
     return cudaErrorInvalidValue;
   StateArgs a;
   a.cu_seqlens = p.cu_seqlens;
@@ -235,11 +237,25 @@ cudaError_t launch(const FwdLaunch& p, int nb, int nblocks_launch, float* ws,
   a.bc = block_chunks(p, nb);
   a.total_tokens = (int)p.total_tokens;
   a.err = p.err;
-  auto kern = lt_block_state_kernel<D, DV>;
+  auto kern = lt_block_state_kernel<D, DV, VAR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<dim3(nblocks_launch, p.Hkv, p.B), kThreads, K::SMEM, stream>>>(tk, tv, a);
   return cudaGetLastError();
+}
+
+// the input type and feature map of p as a compile-time variant
+template <int D, int DV>
+cudaError_t launch_var(const FwdLaunch& p, int nb, int nl, float* ws, cudaStream_t stream) {
+  switch (p.in_f16 * 4 + p.phi) {
+    case 0: return launch<D, DV, Var<kInBf16, kPhiElu1>>(p, nb, nl, ws, stream);
+    case 1: return launch<D, DV, Var<kInBf16, kPhiRelu>>(p, nb, nl, ws, stream);
+    case 2: return launch<D, DV, Var<kInBf16, kPhiExp>>(p, nb, nl, ws, stream);
+    case 4: return launch<D, DV, Var<kInF16, kPhiElu1>>(p, nb, nl, ws, stream);
+    case 5: return launch<D, DV, Var<kInF16, kPhiRelu>>(p, nb, nl, ws, stream);
+    case 6: return launch<D, DV, Var<kInF16, kPhiExp>>(p, nb, nl, ws, stream);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -274,6 +290,11 @@ cudaError_t launch_block_state(const FwdLaunch& p, int nb, float* ws, cudaStream
   // causal: the last block's aggregate is never needed
   const int nl = p.causal ? nb - 1 : nb;
   if (nl <= 0) return cudaSuccess;
+  if (p.in_f16 || p.phi) {  // variants: d = dv = 64 or 128
+    if (p.d == 64 && p.dv == 64) return launch_var<64, 64>(p, nb, nl, ws, stream);
+    if (p.d == 128 && p.dv == 128) return launch_var<128, 128>(p, nb, nl, ws, stream);
+    return cudaErrorInvalidValue;
+  }
   if (p.d == 64 && p.dv == 64) return launch<64, 64>(p, nb, nl, ws, stream);
   if (p.d == 128 && p.dv == 128) return launch<128, 128>(p, nb, nl, ws, stream);
   if (p.d == 64 && p.dv == 128) return launch<64, 128>(p, nb, nl, ws, stream);

@@ -76,8 +76,18 @@ typedef enum {
 
 typedef enum {
   LT_F32 = 0,  /* fp32 inputs/outputs, fp32 FMA arithmetic */
-  LT_BF16 = 1  /* bf16 inputs/outputs, tensor cores, fp32 accumulation */
+  LT_BF16 = 1, /* bf16 inputs/outputs, tensor cores, fp32 accumulation */
+  LT_F16 = 2   /* fp16 inputs/outputs, tensor cores on bf16 operands, fp32
+                  accumulation; lt_linear_attn_fwd and lt_linear_attn_fwd_ex
+                  only, d = dv = 64 or 128 */
 } lt_dtype_t;
+
+/* Feature maps phi of lt_linear_attn_fwd_ex (applied elementwise to Q and K). */
+typedef enum {
+  LT_PHI_ELU1 = 0, /* ELU(x) + 1 (alpha = 1): the method's map, the default */
+  LT_PHI_RELU = 1, /* max(x, 0) */
+  LT_PHI_EXP = 2   /* e^x */
+} lt_feature_map_t;
 
 /*
  * Forward pass of (causal or non-causal) linear attention.
@@ -98,7 +108,9 @@ typedef enum {
  *           Empty sequences are allowed.  An inconsistent array is skipped
  *           by the kernel and reported by lt_get_last_device_error().
  * stream    CUDA stream to enqueue on.
- * dtype     LT_BF16 (tensor-core path) or LT_F32 (fp32 FMA path).
+ * dtype     LT_BF16 (tensor-core path), LT_F16 (fp16 I/O on the same
+ *           tensor-core path with bf16 operands; d = dv = 64 or 128) or
+ *           LT_F32 (fp32 FMA path).
  *
  * Evaluation (bf16): chunks of 128 tokens; the intra-chunk part as masked
  * dense products and the inter-chunk part through the carried state
@@ -117,6 +129,27 @@ LT_API lt_status_t lt_linear_attn_fwd(const void *q, const void *k, const void *
                                int B, int H_q, int H_kv, int N, int d, int dv, int causal,
                                float eps, const int32_t *cu_seqlens, lt_stream_t stream,
                                lt_dtype_t dtype);
+
+/*
+ * lt_linear_attn_fwd_ex: lt_linear_attn_fwd with another feature map phi
+ * (the lineartile page, "Features": "Replace phi kernel freely").  The
+ * library's kernels take the map as a compile-time functor of their tile
+ * transform, so a map is one small device function; the maps compiled in are
+ * lt_feature_map_t.  Same arguments, layouts and results as
+ * lt_linear_attn_fwd otherwise; with LT_PHI_ELU1 it IS lt_linear_attn_fwd.
+ * Every phi here is >= 0, so the denominator stays >= eps (ReLU can make a
+ * row's scores all zero: its output is then 0).
+ *
+ * Other maps and LT_F16 run the general kernel (the state launch plus the
+ * forward launch) and support d = dv = 64 or 128 (LT_ERR_UNSUPPORTED
+ * otherwise); LT_F32 supports every map and width pair.
+ * Returns as lt_linear_attn_fwd; LT_ERR_INVALID_ARG for an unknown phi.
+ */
+LT_API lt_status_t lt_linear_attn_fwd_ex(const void *q, const void *k, const void *v, void *out,
+                                         int B, int H_q, int H_kv, int N, int d, int dv,
+                                         int causal, float eps, const int32_t *cu_seqlens,
+                                         lt_stream_t stream, lt_dtype_t dtype,
+                                         lt_feature_map_t phi);
 
 /*
  * lt_linear_attn_fwd_noalloc: the bf16 forward pass of lt_linear_attn_fwd

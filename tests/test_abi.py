@@ -197,6 +197,40 @@ def test_bwd_rejects_invalid_arguments(case, expect):
     assert st == expect
 
 
+@pytest.mark.parametrize("case,expect", [
+    (dict(phi=3), 1), (dict(phi=-1), 1), (dict(phi=1, d=64, dv=128), 2),
+    (dict(dtype=2, d=128, dv=64), 2), (dict(phi=2, dtype=7), 2), (dict(q=None, phi=1), 1),
+])
+def test_fwd_ex_rejects_invalid_arguments(case, expect):
+    """Unknown feature maps; the tensor-core variants (fp16 I/O, the other
+    maps) take d = dv = 64 or 128 only.  Every case fails before a pointer
+    is examined."""
+    from causal_linear_attention_chunked_b200 import _binding as b
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, B=1, Hq=8, Hkv=8, N=16, d=64, dv=64, causal=1,
+             eps=1e-6, dtype=1, phi=0)
+    a.update(case)
+    st = b.lib.lt_linear_attn_fwd_ex(a["q"], a["k"], a["v"], a["out"], a["B"], a["Hq"],
+                                     a["Hkv"], a["N"], a["d"], a["dv"], a["causal"], a["eps"],
+                                     None, None, a["dtype"], a["phi"])
+    assert st == expect
+
+
+def test_fp16_plan_and_refusals():
+    """fp16 inputs plan the two-launch general path; entry points other than
+    the forward pass refuse LT_F16."""
+    from causal_linear_attention_chunked_b200 import _binding as b
+    nb, nl, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    assert b.lib.lt_linear_attn_fwd_plan(2, 8, 8, 4096, 64, 64, 1, 0, 2, 148, ctypes.byref(nb),
+                                         ctypes.byref(nl), ctypes.byref(ws)) == 0
+    assert (nb.value, nl.value) == (8, 2)
+    assert b.lib.lt_linear_attn_fwd_plan(2, 8, 8, 4096, 64, 128, 1, 0, 2, 148, ctypes.byref(nb),
+                                         ctypes.byref(nl), ctypes.byref(ws)) == 2
+    assert b.lib.lt_linear_attn_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 8, 64, 64,
+                                            1e-6, None, 2) == 2
+    assert b.lib.lt_linear_attn_state(FAKE, FAKE, 1, 8, 16, 64, 64, None, None, None, FAKE, FAKE,
+                                      None, 2) == 2
+
+
 def test_selftest_wait_rejects_invalid_limit():
     from causal_linear_attention_chunked_b200 import _binding as b
     assert b.lib.lt_selftest_wait_timeout(0, None) == 1
