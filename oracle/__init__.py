@@ -45,6 +45,9 @@ def _load():
                     ctypes.c_double, i32p]
         lib.lt_oracle_bwd_quadratic.argtypes = bwd_args
         lib.lt_oracle_bwd_recurrent.argtypes = bwd_args
+        win_args = [vp, vp, vp, ip, dp, ip, ip, ip, ip, ip, ip, ip, ctypes.c_double, i32p]
+        lib.lt_oracle_fwd_window_quadratic.argtypes = win_args
+        lib.lt_oracle_fwd_window_recurrent.argtypes = win_args
         lib.lt_oracle_set_phi.argtypes = [ctypes.c_int]
         lib.lt_oracle_set_phi.restype = ctypes.c_int
         lib.lt_oracle_phi.argtypes = [ctypes.c_double]
@@ -53,7 +56,8 @@ def _load():
         for name in ("lt_oracle_fwd_quadratic", "lt_oracle_fwd_recurrent", "lt_oracle_fwd_rows",
                      "lt_oracle_noncausal_numerator", "lt_oracle_decode_step",
                      "lt_oracle_fwd_state", "lt_oracle_bwd_quadratic",
-                     "lt_oracle_bwd_recurrent"):
+                     "lt_oracle_bwd_recurrent", "lt_oracle_fwd_window_quadratic",
+                     "lt_oracle_fwd_window_recurrent"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -272,3 +276,27 @@ def bwd_quadratic(q, k, v, dout, causal=True, eps=1e-6, cu_seqlens=None):
 def bwd_recurrent(q, k, v, dout, causal=True, eps=1e-6, cu_seqlens=None):
     """Gradients (dQ, dK, dV) by the forward and reverse state recurrences."""
     return _bwd(_load().lt_oracle_bwd_recurrent, q, k, v, dout, causal, eps, cu_seqlens)
+
+
+def _fwd_window(fn, q, k, v, window, eps, cu_seqlens):
+    (rq, rk, rv), t = _same_type(q, k, v)
+    B, Hq, Hkv, N, d, dv, oshape = _geometry(rq, rk, rv, cu_seqlens)
+    out = np.zeros(oshape, dtype=np.float64)
+    cu, cup = _cu(cu_seqlens)
+    rc = fn(_ptr(rq), _ptr(rk), _ptr(rv), t, _dptr(out), B, Hq, Hkv, N, d, dv, int(window),
+            float(eps), cup)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
+
+
+def fwd_window_quadratic(q, k, v, window, eps=1e-6, cu_seqlens=None):
+    """Sliding-window causal attention: keys i - window < j <= i, by the
+    masked quadratic definition."""
+    return _fwd_window(_load().lt_oracle_fwd_window_quadratic, q, k, v, window, eps, cu_seqlens)
+
+
+def fwd_window_recurrent(q, k, v, window, eps=1e-6, cu_seqlens=None):
+    """Sliding-window causal attention as the difference of the prefix state
+    and a prefix state `window` tokens behind."""
+    return _fwd_window(_load().lt_oracle_fwd_window_recurrent, q, k, v, window, eps, cu_seqlens)

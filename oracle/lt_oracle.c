@@ -606,3 +606,93 @@ int lt_oracle_bwd_recurrent(const void *q, const void *k, const void *v, const v
     }
     return 0;
 }
+
+/*
+ * Sliding-window causal attention ("lineartile 1.0.0", "Features": sliding
+ * window attention).  Read plainly for linear attention: row i attends to
+ * the w most recent keys, i - w < j <= i, i.e. the state S_i - S_{i-w}:
+ *     O_i = phi(Q_i) (S_i - S_{i-w}) / (phi(Q_i) . (z_i - z_{i-w}) + eps)
+ * with S_m = z_m = 0 for m < 0.  w >= 1; w >= n is the causal form.
+ *
+ * Form 1 (quadratic): the masked definition with the window.
+ */
+int lt_oracle_fwd_window_quadratic(const void *q, const void *k, const void *v, int in_type,
+                                   double *out, int B, int Hq, int Hkv, int N, int d, int dv,
+                                   int window, double eps, const int32_t *cu_seqlens) {
+    if (check_args(B, Hq, Hkv, N, d, dv, eps) || window < 1) return 1;
+    const int G = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int s = 0; s < B; ++s) {
+        for (int h = 0; h < Hq; ++h) {
+            const int g = h / G;
+            int64_t t0, n;
+            seq_range(s, N, cu_seqlens, &t0, &n);
+            double *pq = malloc(sizeof(double) * d), *num = malloc(sizeof(double) * dv);
+            for (int64_t i = 0; i < n; ++i) {
+                for (int c = 0; c < d; ++c) pq[c] = lt_oracle_phi(load_elem(q, off(t0 + i, h, Hq, d, c), in_type));
+                for (int c = 0; c < dv; ++c) num[c] = 0.0;
+                double den = 0.0;
+                const int64_t jbeg = i - window + 1 > 0 ? i - window + 1 : 0;
+                for (int64_t j = jbeg; j <= i; ++j) {
+                    double a = 0.0;
+                    for (int c = 0; c < d; ++c) a += pq[c] * lt_oracle_phi(load_elem(k, off(t0 + j, g, Hkv, d, c), in_type));
+                    for (int c = 0; c < dv; ++c) num[c] += a * load_elem(v, off(t0 + j, g, Hkv, dv, c), in_type);
+                    den += a;
+                }
+                for (int c = 0; c < dv; ++c) out[off(t0 + i, h, Hq, dv, c)] = num[c] / (den + eps);
+            }
+            free(pq);
+            free(num);
+        }
+    }
+    return 0;
+}
+
+/*
+ * Form 2 (recurrences): the prefix state S, z and a second state S', z'
+ * that follows w tokens behind (token i - w is added to it at step i), so
+ * that S - S' is the window's state:
+ *     S += phi(K_i)^T V_i, z += phi(K_i);   if i >= w: S' += phi(K_{i-w})^T V_{i-w}, ...
+ *     O_i = phi(Q_i)(S - S') / (phi(Q_i).(z - z') + eps).
+ */
+int lt_oracle_fwd_window_recurrent(const void *q, const void *k, const void *v, int in_type,
+                                   double *out, int B, int Hq, int Hkv, int N, int d, int dv,
+                                   int window, double eps, const int32_t *cu_seqlens) {
+    if (check_args(B, Hq, Hkv, N, d, dv, eps) || window < 1) return 1;
+    const int G = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int s = 0; s < B; ++s) {
+        for (int h = 0; h < Hq; ++h) {
+            const int g = h / G;
+            int64_t t0, n;
+            seq_range(s, N, cu_seqlens, &t0, &n);
+            double *S = calloc((size_t)d * dv, sizeof(double)), *z = calloc((size_t)d, sizeof(double));
+            double *Sl = calloc((size_t)d * dv, sizeof(double)), *zl = calloc((size_t)d, sizeof(double));
+            double *pq = malloc(sizeof(double) * d), *pk = malloc(sizeof(double) * d);
+            double *vv = malloc(sizeof(double) * dv);
+            for (int64_t i = 0; i < n; ++i) {
+                for (int lag = 0; lag < 2; ++lag) {
+                    const int64_t t = lag ? i - window : i;
+                    if (t < 0) continue;
+                    double *St = lag ? Sl : S, *zt = lag ? zl : z;
+                    for (int c = 0; c < d; ++c) pk[c] = lt_oracle_phi(load_elem(k, off(t0 + t, g, Hkv, d, c), in_type));
+                    for (int c = 0; c < dv; ++c) vv[c] = load_elem(v, off(t0 + t, g, Hkv, dv, c), in_type);
+                    for (int a = 0; a < d; ++a) {
+                        for (int c = 0; c < dv; ++c) St[a * dv + c] += pk[a] * vv[c];
+                        zt[a] += pk[a];
+                    }
+                }
+                for (int c = 0; c < d; ++c) pq[c] = lt_oracle_phi(load_elem(q, off(t0 + i, h, Hq, d, c), in_type));
+                double den = eps;
+                for (int a = 0; a < d; ++a) den += pq[a] * (z[a] - zl[a]);
+                for (int c = 0; c < dv; ++c) {
+                    double num = 0.0;
+                    for (int a = 0; a < d; ++a) num += pq[a] * (S[a * dv + c] - Sl[a * dv + c]);
+                    out[off(t0 + i, h, Hq, dv, c)] = num / den;
+                }
+            }
+            free(S); free(z); free(Sl); free(zl); free(pq); free(pk); free(vv);
+        }
+    }
+    return 0;
+}

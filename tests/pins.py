@@ -98,6 +98,49 @@ def pin_fp16_inputs_widened_exactly():
     assert o.tolist() == [[[[1.0, 65504.0, float(torch.tensor(5.96e-8).half().double())]]]]
 
 
+def pin_sliding_window():
+    """Sliding window (keys i - w < j <= i): the windowed quadratic form and
+    the difference of two prefix states agree; w >= n is the causal form;
+    w = 1 gives each row its own value (scaled by a/(a+eps)); constant keys
+    give the moving average of the last w values (eps = 0); packed sequences
+    equal independent calls; GQA equals replication."""
+    B, N, Hq, Hkv, d, dv = 2, 29, 4, 2, 5, 3
+    q = _rand((B, N, Hq, d), 160)
+    k = _rand((B, N, Hkv, d), 161)
+    v = _rand((B, N, Hkv, dv), 162)
+    for w in (1, 2, 7, 28, 29, 100):
+        a = oracle.fwd_window_quadratic(q, k, v, w)
+        b = oracle.fwd_window_recurrent(q, k, v, w)
+        assert np.abs(a - b).max() <= 1e-12 * np.abs(a).max(), w
+    full = oracle.fwd_quadratic(q, k, v, causal=True)
+    for w in (29, 100):
+        assert np.abs(oracle.fwd_window_recurrent(q, k, v, w) - full).max() <= 1e-12 * np.abs(full).max()
+    o1 = oracle.fwd_window_quadratic(q, k, v, 1, eps=0.0)
+    assert np.abs(o1 - np.repeat(v, Hq // Hkv, axis=2)).max() <= 1e-14
+    kc = np.broadcast_to(_rand((1, 1, Hkv, d), 163), k.shape).copy()
+    for w in (3, 8):
+        o = oracle.fwd_window_recurrent(q, kc, v, w, eps=0.0)
+        csum = np.concatenate([np.zeros((B, 1, Hkv, dv)), np.cumsum(v, axis=1)], axis=1)
+        idx = np.arange(N)
+        lo = np.maximum(idx - w + 1, 0)
+        mean = (csum[:, idx + 1] - csum[:, lo]) / (idx - lo + 1).reshape(1, N, 1, 1)
+        assert np.abs(o - np.repeat(mean, Hq // Hkv, axis=2)).max() <= 1e-13, w
+    G = Hq // Hkv
+    a = oracle.fwd_window_recurrent(q, k, v, 6)
+    b = oracle.fwd_window_quadratic(q, np.repeat(k, G, axis=2), np.repeat(v, G, axis=2), 6)
+    assert np.abs(a - b).max() <= 1e-12 * np.abs(b).max()
+    lens = [9, 0, 1, 14]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    qp, kp, vp = _rand((T, Hq, d), 164), _rand((T, Hkv, d), 165), _rand((T, Hkv, dv), 166)
+    packed = oracle.fwd_window_recurrent(qp, kp, vp, 4, cu_seqlens=cu)
+    for s_, n in enumerate(lens):
+        if n:
+            x, y = cu[s_], cu[s_ + 1]
+            dense = oracle.fwd_window_quadratic(qp[None, x:y], kp[None, x:y], vp[None, x:y], 4)[0]
+            assert np.abs(packed[x:y] - dense).max() <= 1e-12 * max(1.0, np.abs(dense).max())
+
+
 def _hand_2x2_inputs(g):
     q = np.array(g["q"], dtype=np.float64).reshape(1, 2, 1, 2)
     k = np.array([[1.0, 0.0], [0.0, -math.log(2.0)]]).reshape(1, 2, 1, 2)
@@ -526,6 +569,7 @@ ALL_PINS = [
     pin_phi_is_elu_plus_one,
     pin_feature_maps,
     pin_fp16_inputs_widened_exactly,
+    pin_sliding_window,
     pin_hand_2x2,
     pin_hand_3tok,
     pin_two_forms_agree,

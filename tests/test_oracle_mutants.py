@@ -56,6 +56,10 @@ MUTANTS = [
      "for (int64_t j = n - 1; j >= 0; --j) {", "for (int64_t j = 0; j < n; ++j) {"),
     ("bwd: dK of a GQA group from its first query head only", "for (int h = g * G; h < (g + 1) * G; ++h) {\n                /* forward recurrence",
      "for (int h = g * G; h < g * G + 1; ++h) {\n                /* forward recurrence"),
+    ("window one key too wide", "const int64_t jbeg = i - window + 1 > 0 ? i - window + 1 : 0;",
+     "const int64_t jbeg = i - window > 0 ? i - window : 0;"),
+    ("lagged state one token late", "const int64_t t = lag ? i - window : i;",
+     "const int64_t t = lag ? i - window - 1 : i;"),
     ("rows: packed offsets ignored", "\n        seq_range(s, N, cu_seqlens, &t0, &n);\n        if (i < 0",
      "\n        seq_range(s, N, NULL, &t0, &n);\n        if (i < 0"),
 ]
