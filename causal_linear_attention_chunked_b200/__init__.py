@@ -14,7 +14,7 @@ API names below; a missing library raises ImportError.
 """
 _API = ("linear_attn_fwd", "linear_attn_fwd_state", "linear_attn_fwd_plan",
         "linear_attn_decode_step", "linear_attn_state", "linear_attn_state_carry",
-        "linear_attn_bwd",
+        "linear_attn_bwd", "linear_attn_fwd_window",
         "set_schedule",
         "get_last_device_error",
         "linear_attn_fwd_host", "LtError")

@@ -25,7 +25,7 @@ EXPORTED = ("lt_linear_attn_fwd", "lt_linear_attn_fwd_noalloc", "lt_linear_attn_
             "lt_linear_attn_fwd_state", "lt_linear_attn_decode_step", "lt_status_string",
             "lt_get_last_device_error", "lt_abi_version", "lt_selftest_wait_timeout",
             "lt_debug_set_schedule", "lt_linear_attn_state", "lt_linear_attn_state_carry",
-            "lt_linear_attn_bwd", "lt_linear_attn_fwd_ex")
+            "lt_linear_attn_bwd", "lt_linear_attn_fwd_ex", "lt_linear_attn_fwd_window")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("liblt.so is not built (run `python -m "
@@ -38,6 +38,9 @@ lib.lt_linear_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _
 lib.lt_linear_attn_fwd.restype = _i
 lib.lt_linear_attn_fwd_ex.argtypes = lib.lt_linear_attn_fwd.argtypes + [_i]
 lib.lt_linear_attn_fwd_ex.restype = _i
+lib.lt_linear_attn_fwd_window.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
+                                          _vp, _vp, _i]
+lib.lt_linear_attn_fwd_window.restype = _i
 lib.lt_linear_attn_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
                                            _vp, _vp]
 lib.lt_linear_attn_fwd_noalloc.restype = _i
@@ -133,6 +136,31 @@ def linear_attn_fwd(q, k, v, causal=True, eps=1e-6, cu_seqlens=None, out=None, s
         _check(lib.lt_linear_attn_fwd(*args))
     else:
         _check(lib.lt_linear_attn_fwd_ex(*args, FEATURE_MAPS[feature_map]))
+    return out
+
+
+def linear_attn_fwd_window(q, k, v, window, eps=1e-6, cu_seqlens=None, out=None, stream=None):
+    """Sliding-window causal linear attention: row i attends to keys
+    i - window < j <= i.  See lt_linear_attn_fwd_window."""
+    if cu_seqlens is None:
+        B, N, Hq, d = q.shape
+        Hkv, dv = k.shape[2], v.shape[3]
+        oshape = (B, N, Hq, dv)
+    else:
+        N, Hq, d = q.shape
+        Hkv, dv = k.shape[1], v.shape[2]
+        B = cu_seqlens.numel() - 1
+        oshape = (N, Hq, dv)
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
+            raise TypeError("cu_seqlens must be a contiguous int32 tensor")
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+    if out is None:
+        out = torch.empty(oshape, dtype=q.dtype, device=q.device)
+    _check(lib.lt_linear_attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, Hq, Hkv, N, d,
+                                         dv, int(window), float(eps), _ptr(cu_seqlens),
+                                         _stream_handle(stream, q.device), _dtype_code(q.dtype)))
     return out
 
 

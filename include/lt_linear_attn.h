@@ -152,6 +152,29 @@ LT_API lt_status_t lt_linear_attn_fwd_ex(const void *q, const void *k, const voi
                                          lt_feature_map_t phi);
 
 /*
+ * lt_linear_attn_fwd_window: sliding-window causal linear attention (the
+ * lineartile page, "Features": sliding window attention).  Row i attends to
+ * the `window` most recent keys, i - window < j <= i:
+ *     O_i = phi(Q_i)(S_i - S_{i-w}) / (phi(Q_i).(z_i - z_{i-w}) + eps),
+ * S_m = z_m = 0 for m < 0; window >= N is the causal form.
+ *
+ * q .. cu_seqlens, stream   as for lt_linear_attn_fwd (causal only).
+ * window     >= 1 tokens.
+ * dtype      LT_F32, LT_BF16 or LT_F16 (fp32 arithmetic for all three;
+ *            outputs rounded once to the input's type).
+ * Evaluation: 32-token chunks, one CTA per (sequence, query head); each
+ * row's window split into a window state carried from chunk to chunk
+ * (holding only the window's keys, never a difference of long prefix sums)
+ * and two band-masked tiles.  No scratch memory.
+ * Returns as lt_linear_attn_fwd; LT_ERR_INVALID_ARG for window < 1.
+ */
+LT_API lt_status_t lt_linear_attn_fwd_window(const void *q, const void *k, const void *v,
+                                             void *out, int B, int H_q, int H_kv, int N, int d,
+                                             int dv, int window, float eps,
+                                             const int32_t *cu_seqlens, lt_stream_t stream,
+                                             lt_dtype_t dtype);
+
+/*
  * lt_linear_attn_fwd_noalloc: the bf16 forward pass of lt_linear_attn_fwd
  * (same arguments, dtype fixed to LT_BF16, same kernels and results) for
  * callers that cannot let a library allocate device memory.  The method has

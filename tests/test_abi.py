@@ -231,6 +231,21 @@ def test_fp16_plan_and_refusals():
                                       None, 2) == 2
 
 
+@pytest.mark.parametrize("case,expect", [
+    (dict(window=0), 1), (dict(window=-3), 1), (dict(q=None), 1), (dict(B=0), 1),
+    (dict(d=32), 2), (dict(dtype=9), 2), (dict(Hkv=3, Hq=8), 1),
+])
+def test_window_rejects_invalid_arguments(case, expect):
+    from causal_linear_attention_chunked_b200 import _binding as b
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, B=1, Hq=8, Hkv=8, N=16, d=64, dv=64, window=4,
+             eps=1e-6, dtype=1)
+    a.update(case)
+    st = b.lib.lt_linear_attn_fwd_window(a["q"], a["k"], a["v"], a["out"], a["B"], a["Hq"],
+                                         a["Hkv"], a["N"], a["d"], a["dv"], a["window"],
+                                         a["eps"], None, None, a["dtype"])
+    assert st == expect
+
+
 def test_selftest_wait_rejects_invalid_limit():
     from causal_linear_attention_chunked_b200 import _binding as b
     assert b.lib.lt_selftest_wait_timeout(0, None) == 1
