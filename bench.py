@@ -344,7 +344,8 @@ def measure_from_state(L, w, K, stream, device, l2_bytes, peak):
             "ms_per_step": ms, "achieved_gbs": ach, "roofline_frac": ach / peak,
             "algorithmic_bytes": nbytes,
             "note": "lt_linear_attn_fwd_state: given initial state, final state returned "
-                    "(state launch over every block, prefix kernel, forward launch)"}
+                    "(one cooperative launch: S0 folded into every block's carry, the last "
+                    "block writes the final state)"}
 
 
 def measure_decode(L, stream, device, steps=1000, reps=3):

@@ -80,6 +80,13 @@ struct FusedArgs {
   int bc;           // chunks per block
   float eps;
   int* err;
+  // the forward pass continued from a given state (nullptr: zero) and
+  // returning the final state (nullptr: not returned), per lane:
+  // S [lane][d][dv], z [lane][d] fp32
+  const float* s0;
+  const float* z0;
+  float* s_out;
+  float* z_out;
 };
 
 constexpr int kThreads = 576;
@@ -144,15 +151,31 @@ __device__ __forceinline__ void store_operand_row(uint8_t* op, int row, const fl
   }
 }
 
-// The carry C = sum of the aggregates of blocks [0, nsum) of one lane (base:
-// that lane's first aggregate), fp32 in block order, rounded once to bf16
-// into the K-major operand; rows DV+1 .. OPR-1 zeroed.  Thread u of NT.
+// The carry C = S0 + the aggregates of blocks [0, nsum) of one lane (base:
+// that lane's first aggregate; s0, z0: the lane's given state or nullptr),
+// fp32 in block order, rounded once to bf16 into the K-major operand; rows
+// DV+1 .. OPR-1 zeroed.  With s_out, also the final state C + base[own]
+// (own < 0: C itself) in fp32, in the [d][dv] layout.  Thread u of NT.
 template <int NT>
-__device__ __forceinline__ void gather_carry(const float4* base, int nsum, uint8_t* op, int u) {
+__device__ __forceinline__ void gather_carry(const float4* base, int nsum, uint8_t* op, int u,
+                                             const float* s0, const float* z0, float* s_out,
+                                             float* z_out, int own) {
   constexpr int PER = (E4 + NT - 1) / NT;
   float4 acc[PER];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int e = 0; e < PER; ++e) {
+    const int i = u + e * NT, row = i >> 4, c4 = i & 15;
+    acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (s0 != nullptr && i < E4) {
+      // aggregate row `row`, entries 4*c4 .. 4*c4+3: column `row` of S (rows
+      // 4*c4 .. of the [d][dv] state), or z for row DV
+      if (row < DV)
+        acc[e] = make_float4(s0[(4 * c4) * DV + row], s0[(4 * c4 + 1) * DV + row],
+                             s0[(4 * c4 + 2) * DV + row], s0[(4 * c4 + 3) * DV + row]);
+      else
+        acc[e] = *reinterpret_cast<const float4*>(z0 + 4 * c4);
+    }
+  }
 #pragma unroll 1
   for (int b0 = 0; b0 < nsum; b0 += 4) {  // four blocks' loads in flight
     float4 v[4][PER];
@@ -185,6 +208,24 @@ __device__ __forceinline__ void gather_carry(const float4* base, int nsum, uint8
       const int row = i >> 4, c4 = i & 15;  // 16 float4 per 64-float row
       uint2 w = make_uint2(pack_bf16x2(acc[e].x, acc[e].y), pack_bf16x2(acc[e].z, acc[e].w));
       *reinterpret_cast<uint2*>(op + sw128_off(row, c4 >> 1) + (c4 & 1) * 8) = w;
+      if (s_out != nullptr) {
+        float4 f = acc[e];
+        if (own >= 0) {
+          const float4 a = __ldcg(base + (size_t)own * E4 + i);
+          f.x += a.x;
+          f.y += a.y;
+          f.z += a.z;
+          f.w += a.w;
+        }
+        if (row < DV) {
+          s_out[(4 * c4) * DV + row] = f.x;
+          s_out[(4 * c4 + 1) * DV + row] = f.y;
+          s_out[(4 * c4 + 2) * DV + row] = f.z;
+          s_out[(4 * c4 + 3) * DV + row] = f.w;
+        } else {
+          *reinterpret_cast<float4*>(z_out + 4 * c4) = f;
+        }
+      }
     }
   }
   // zero rows DV+1 .. OPR-1 (15 rows of 8 pieces)
@@ -216,7 +257,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_items = Ri * G;  // item j: chunk j / G, query head g*G + j % G
   // aggregates in the carry: the earlier blocks (causal) or all (non-causal)
   const int nprev = causal ? blk : a.nb;
-  const bool publish = !causal || blk + 1 < a.nb;
+  // the final state: the last block, from its carry plus (causal) its own
+  // aggregate
+  const bool final_state = a.s_out != nullptr && blk + 1 == a.nb;
+  const bool publish = !causal || blk + 1 < a.nb || final_state;
+  // every block with a carry (earlier blocks or a given state) gathers it
+  const bool gath = nprev > 0 || a.s0 != nullptr;
+  const size_t lane_idx = (size_t)s * a.Hkv + g;
   // causal: running sums L_1 .. L_{Ri-1} for the chunks after the first
   const int nlocal = causal ? Ri - 1 : 0;
   const float4* agg_base =
@@ -255,7 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto gather_part = [&](int u) {
     named_bar_sync(5, 384);
     if (!*abort_flag) {
-      gather_carry<384>(agg_base, nprev, sC, u);
+      gather_carry<384>(agg_base, nprev, sC, u,
+                        a.s0 ? a.s0 + lane_idx * D * DV : nullptr,
+                        a.z0 ? a.z0 + lane_idx * D : nullptr,
+                        final_state ? a.s_out + lane_idx * D * DV : nullptr,
+                        final_state ? a.z_out + lane_idx * D : nullptr,
+                        causal ? blk : -1);
       fence_proxy_async_smem();
     }
     named_bar_sync(5, 384);
@@ -362,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_f16_ts(tmem + TM_ACC + j * ACCW, tmem + TM_P + kk * 8, desc_advance(vd, kk * 2048),
                       ID_PV, kk > 0 ? 1u : 0u);
       };
-      const bool has_carry = nprev > 0;
+      const bool has_carry = gath;
       // issued so far: aggregate products (phase A), running-sum products
       // (phase B), scores, P V, phi(Q) L, phi(Q) C; items committed
       int da = 0, db = 0, sc = 0, pv = 0, ql = 0, qc = 0, done = 0;
@@ -475,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_sync(1, kXf);
       if (x == 0 && !*abort_flag) mbar_arrive(is_kv ? &bars.kv_xf[r] : &bars.q_xf[j]);
     }
-    if (nprev > 0) gather_part(x);
+    if (gath) gather_part(x);
     // warps 0-3: the odd items' outputs
     if (warp < 4) {
       bool ok = true;
@@ -582,8 +634,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (y == 0 && !*abort_flag) mbar_arrive(&bars.op_full[r + 1]);
     }
     // 3. the carry, once every CTA has published
-    if (nprev > 0) {
-      if (y == 0 && arrived) grid_wait(grid_old, abort_flag, a.err, kWaitLimitNs);
+    if (gath) {
+      // (a carry of S0 alone needs no other block)
+      if (y == 0 && arrived && (nprev > 0 || final_state))
+        grid_wait(grid_old, abort_flag, a.err, kWaitLimitNs);
       named_bar_sync(3, 128);
       gather_part(256 + y);
     }
@@ -614,6 +668,13 @@ bool block_fused_supported(const FwdLaunch& p, int nb, int num_sms) {
 
 cudaError_t launch_fwd_bf16_block_fused(const FwdLaunch& p, int nb, float* ws,
                                         cudaStream_t stream) {
+  return launch_fwd_bf16_block_fused_state(p, nb, ws, nullptr, nullptr, nullptr, nullptr,
+                                           stream);
+}
+
+cudaError_t launch_fwd_bf16_block_fused_state(const FwdLaunch& p, int nb, float* ws,
+                                              const float* s0, const float* z0, float* s_out,
+                                              float* z_out, cudaStream_t stream) {
   if (ws == nullptr) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
   if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
@@ -632,6 +693,10 @@ cudaError_t launch_fwd_bf16_block_fused(const FwdLaunch& p, int nb, float* ws,
   a.bc = block_chunks(p, nb);
   a.eps = p.eps;
   a.err = p.err;
+  a.s0 = s0;
+  a.z0 = z0;
+  a.s_out = s_out;
+  a.z_out = z_out;
   auto fk = lt_fused_fwd_kernel;
   cudaError_t e =
       cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout::SMEM);

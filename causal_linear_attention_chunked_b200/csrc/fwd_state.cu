@@ -11,7 +11,10 @@
 // result, and the final state feeds the decode step directly.
 //
 // bf16 evaluation reuses the block-parallel scan ("Why Stream Wins at
-// Ultra-Long Context", section 5.3, the second level over blocks):
+// Ultra-Long Context", section 5.3, the second level over blocks).  Short
+// blocks (the one-launch path of lt_linear_attn_fwd) run that single
+// cooperative launch, whose carries start from S0 and whose last block also
+// writes the final state; otherwise three launches:
 //   1. the state launch writes the aggregate A_b of every block;
 //   2. lt_state_prefix_kernel turns them, in block order, into each block's
 //      carry, S0 + sum_{b' < b} A_b' (causal) or S0 + sum_b A_b (non-causal),
@@ -87,6 +90,14 @@ cudaError_t launch_fwd_state(const FwdLaunch& p, bool bf16, const float* s0, con
   if (injected_workspace_alloc_failure()) return cudaErrorMemoryAllocation;
   cudaError_t e = cudaMallocAsync(&ws, bytes, stream);
   if (e != cudaSuccess) return e;
+  if (sched_kernel() == LT_SCHED_AUTO && block_fused_supported(p, nb, sms)) {
+    // short blocks: one cooperative launch that also folds in S0 and writes
+    // the final state (the carries are the same sums in the same order)
+    e = launch_fwd_bf16_block_fused_state(p, nb, static_cast<float*>(ws), s0, z0, s_out, z_out,
+                                          stream);
+    const cudaError_t f = cudaFreeAsync(ws, stream);
+    return e != cudaSuccess ? e : f;
+  }
   float* w = static_cast<float*>(ws);
   // 1. every block's aggregate (the state launch in its all-blocks mode)
   FwdLaunch all = p;

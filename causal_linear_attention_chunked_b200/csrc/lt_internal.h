@@ -66,6 +66,11 @@ cudaError_t launch_fwd_bf16_seq(const FwdLaunch& p, int nb, const float* ws,
 bool block_fused_supported(const FwdLaunch& p, int nb, int num_sms);
 cudaError_t launch_fwd_bf16_block_fused(const FwdLaunch& p, int nb, float* ws,
                                         cudaStream_t stream);
+// the same continued from the state (s0, z0) (nullptr: zero) and writing the
+// final state to (s_out, z_out) (nullptr: not returned)
+cudaError_t launch_fwd_bf16_block_fused_state(const FwdLaunch& p, int nb, float* ws,
+                                              const float* s0, const float* z0, float* s_out,
+                                              float* z_out, cudaStream_t stream);
 // the per-device error word of the current device (looked up once per device)
 int* device_error_word_current();
 // SM count of the current device (queried once per device); 0 on failure

@@ -255,11 +255,13 @@ LT_API lt_status_t lt_linear_attn_fwd_plan(int B, int H_q, int H_kv, int N, int 
  *        overlap S0 or z0.
  * Scratch: LT_BF16 always allocates a stream-ordered workspace (every
  * block's partial state, as lt_linear_attn_fwd; released before return).
- * Evaluation (bf16): a state launch writes every block's partial state; a
- * small kernel turns them, in block order, into each block's starting state
- * S0 + (earlier blocks) and into the final state; the forward launch starts
- * every block from its own.  With S0 = 0 the outputs equal lt_linear_attn_fwd's
- * two-launch path bit for bit.
+ * Evaluation (bf16): where lt_linear_attn_fwd runs one cooperative launch,
+ * so does this call: every block's starting state is S0 + (earlier blocks),
+ * summed in block order, and the last block writes the final state.
+ * Otherwise a state launch writes every block's partial state, a small
+ * kernel turns them, in block order, into each block's starting state and
+ * into the final state, and the forward launch starts every block from its
+ * own.  With S0 = 0 the outputs equal lt_linear_attn_fwd's bit for bit.
  *
  * Returns as lt_linear_attn_fwd.
  */
