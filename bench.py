@@ -416,7 +416,7 @@ def measure_backward(L, w, stream, device, peak, reps=5):
     return {"workload": w.name + "_backward", "tokens_per_s": w.B * w.Hq * w.N / (ms / 1e3),
             "ms_per_step": ms, "achieved_gbs": ach, "roofline_frac": ach / peak,
             "algorithmic_bytes": nbytes,
-            "note": "lt_linear_attn_bwd: two fp32 FMA scans (one CTA per (sequence, head)), "
+            "note": "lt_linear_attn_bwd: a block-sum launch and two fp32 FMA scans, one CTA per (sequence, head, block), "
                     "eager calls timed with CUDA events"}
 
 

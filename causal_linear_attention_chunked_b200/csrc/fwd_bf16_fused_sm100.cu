@@ -415,87 +415,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                       ID_PV, kk > 0 ? 1u : 0u);
       };
       const bool has_carry = gath;
-      // issued so far: aggregate products (phase A), running-sum products
-      // (phase B), scores, P V, phi(Q) L, phi(Q) C; items committed
-      int da = 0, db = 0, sc = 0, pv = 0, ql = 0, qc = 0, done = 0;
-      bool c_ready = false;
-      uint32_t idle = 0;
-      uint64_t idle_t0 = 0;
-      bool ok = true;
-      // item j's local products are issued (P V, and phi(Q) L after the first chunk)
-      auto local_done = [&](int j) { return pv > j && (j / G == 0 || ql > j); };
-      while (done < n_items && ok) {
-        bool did = false;
-        if (da < Ri && mbar_test(&bars.kv_xf[da], 0)) {
-          // phase A first: the aggregate is what the other CTAs wait for
-          tc_fence_after();
-          issue_ds(da, da > 0);
-          ++da;
-          if (da == Ri) umma_commit(bars.agg_full);
-          did = true;
-        } else if (causal && sc < n_items && sc == pv && da > sc / G &&
-                   mbar_test(&bars.q_xf[sc], 0)) {
-          // score of item sc (the single score buffer is free: P V of the
-          // previous item has been issued, and the pipe executes in order)
-          tc_fence_after();
-          issue_score(sc);
-          umma_commit(&bars.p_full[sc]);
-          if (sc % G == G - 1) umma_commit(&bars.k_free[sc / G]);
-          ++sc;
-          did = true;
-        } else if (causal && pv < sc && mbar_test(&bars.pb_full[pv], 0)) {
-          tc_fence_after();
-          issue_pv(pv);
-          if (pv / G == 0 && !has_carry) {
-            umma_commit(&bars.acc_full[pv]);
-            ++done;
-          }
-          ++pv;
-          did = true;
-        } else if (db < nlocal && da == Ri &&
-                   mbar_test(db == 0 ? bars.agg_empty : &bars.s_empty[db - 1], 0)) {
-          // phase B: the state becomes L_{db+1} (the aggregate has been read)
-          tc_fence_after();
-          issue_ds(db, db > 0);
-          umma_commit(&bars.s_full[db]);
-          ++db;
-          did = true;
-        } else if (causal && ql < n_items && (ql / G == 0 || (pv > ql &&
-                   mbar_test(&bars.op_full[ql / G], 0)))) {
-          if (ql / G > 0) {
-            tc_fence_after();
-            issue_qs(ql, sK + (ql / G - 1) * KVT, true);
-            if (!has_carry) {
-              umma_commit(&bars.acc_full[ql]);
-              ++done;
-            }
-            did = true;
-          }
-          ++ql;
-        } else if (has_carry && qc < n_items &&
-                   (c_ready || (c_ready = mbar_test(bars.c_full, 0))) &&
-                   (causal ? local_done(qc) : mbar_test(&bars.q_xf[qc], 0))) {
-          tc_fence_after();
-          issue_qs(qc, sC, causal);
-          umma_commit(&bars.acc_full[qc]);
-          ++qc;
-          ++done;
-          did = true;
+      // A fixed issue order with one blocking (bounded) wait per group: the
+      // tensor pipe executes in issue order, so the single score buffer is
+      // free again once the previous item's P V has been issued.
+      auto W = [&](uint64_t* bar) {
+        const bool ok = mbar_wait(bar, 0, abort_flag, a.err, kWaitLimitNs);
+        if (ok) tc_fence_after();
+        return ok;
+      };
+      do {
+        // 1. the block aggregate (what the other CTAs wait for)
+        bool ok = true;
+        for (int r = 0; r < Ri && ok; ++r) {
+          if ((ok = W(&bars.kv_xf[r]))) issue_ds(r, r > 0);
         }
-        if (did) {
-          idle = 0;
-        } else if ((++idle & 255u) == 0) {
-          if (*abort_flag) {
-            ok = false;
-          } else if (idle == 256) {
-            idle_t0 = global_timer_ns();
-          } else if (global_timer_ns() - idle_t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            report_error(a.err, kDevErrTimeout);
-            ok = false;
+        if (!ok) break;
+        umma_commit(bars.agg_full);
+        // 2. causal: per item its score, the running sum of its chunk (once
+        //    the state has been read), P V and phi(Q) L
+        for (int j = 0; j < n_items && causal && ok; ++j) {
+          const int r = j / G;
+          if (!(ok = W(&bars.q_xf[j]))) break;
+          issue_score(j);
+          umma_commit(&bars.p_full[j]);
+          if (j % G == G - 1) umma_commit(&bars.k_free[r]);
+          if (j % G == 0 && r < nlocal) {
+            // the state becomes L_{r+1}
+            if (!(ok = W(r == 0 ? bars.agg_empty : &bars.s_empty[r - 1]))) break;
+            issue_ds(r, r > 0);
+            umma_commit(&bars.s_full[r]);
           }
+          if (!(ok = W(&bars.pb_full[j]))) break;
+          issue_pv(j);
+          if (r > 0) {
+            if (!(ok = W(&bars.op_full[r]))) break;
+            issue_qs(j, sK + (r - 1) * KVT, true);
+          }
+          if (!has_carry) umma_commit(&bars.acc_full[j]);
         }
-      }
+        if (!ok || !has_carry) break;
+        // 3. phi(Q) [C | c] into every item's accumulator
+        if (!W(bars.c_full)) break;
+        for (int j = 0; j < n_items; ++j) {
+          if (!causal && !W(&bars.q_xf[j])) break;
+          issue_qs(j, sC, causal);
+          umma_commit(&bars.acc_full[j]);
+        }
+      } while (false);
       umma_commit(bars.drain);
       int dummy = 0;
       mbar_wait(bars.drain, 0, &dummy, nullptr, kWaitLimitNs);

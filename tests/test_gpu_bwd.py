@@ -127,3 +127,29 @@ def test_bwd_deterministic():
     torch.cuda.synchronize()
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+FULL = ["bf16_b2h8n4096d64", "bf16_b1h8n65536d64", "bf16_b1h8n65536d64_noncausal",
+        "bf16_gqa_b2hq32hkv8n16384d128", "bf16_varlen64_h8d64"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_bwd_full_size_every_element(name):
+    """Every gradient element of the bf16 workloads at full size (the block
+    count the library picks for them: many blocks per sequence, carried
+    block sums) against the oracle's recurrent backward form."""
+    w = inputs.WORKLOADS[name]
+    q, k, v, cu = inputs.make(w, seed=w.seed + 700)
+    g = inputs.generator(w.seed + 701)
+    dout = torch.randn(q.shape[:-1] + (w.dv,), generator=g).to(w.dtype)
+    cuc = cu.cuda() if cu is not None else None
+    dq, dk, dvv = L().linear_attn_bwd(q.cuda(), k.cuda(), v.cuda(), dout.cuda(),
+                                      causal=w.causal, eps=w.eps, cu_seqlens=cuc)
+    torch.cuda.synchronize()
+    assert L().get_last_device_error() == 0
+    ref = oracle.bwd_recurrent(q, k, v, dout, causal=w.causal, eps=w.eps,
+                               cu_seqlens=cu.numpy() if cu is not None else None)
+    for got, r, nm in zip((dq, dk, dvv), ref, ("dq", "dk", "dv")):
+        err = grad_rel_err(got.float().cpu().numpy(), r,
+                           cu=cu.numpy() if cu is not None else None)
+        assert err <= TOL_BF16, (nm, err)
