@@ -413,11 +413,36 @@ def measure_backward(L, w, stream, device, peak, reps=5):
     es = 2 if w.dtype == torch.bfloat16 else 4
     nbytes = w.B * w.N * (2 * w.Hq * w.d + 2 * w.Hkv * (w.d + w.dv) + w.Hq * w.dv) * es
     ach = nbytes / (ms * 1e-3) / 1e9
+    fma = backward_fma(w)
+    tflops = 2 * fma / (ms * 1e-3) / 1e12
     return {"workload": w.name + "_backward", "tokens_per_s": w.B * w.Hq * w.N / (ms / 1e3),
             "ms_per_step": ms, "achieved_gbs": ach, "roofline_frac": ach / peak,
-            "algorithmic_bytes": nbytes,
-            "note": "lt_linear_attn_bwd: a block-sum launch and two fp32 FMA scans, one CTA per (sequence, head, block), "
-                    "eager calls timed with CUDA events"}
+            "algorithmic_bytes": nbytes, "executed_fma": fma, "achieved_tflops": tflops,
+            "alu_peak_tflops": FP32_ALU_TFLOPS, "alu_frac": tflops / FP32_ALU_TFLOPS,
+            "note": "lt_linear_attn_bwd: a block-sum launch and two fp32 FMA scans, one CTA per "
+                    "(sequence, head, block), eager calls timed with CUDA events; alu_frac: the "
+                    "FMAs the kernels execute (masked tiles whole) against 148 SMs x 128 fp32 "
+                    "lanes x 2 x 1.965 GHz"}
+
+
+# fp32 FMA peak of the B200: 148 SMs x 128 lanes x 2 flops x 1.965 GHz (max SM clock)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def backward_fma(w):
+    """FMAs the backward kernels execute per call (32-token chunks, masked
+    tiles computed whole): the block-sum launch, the dq scan per query head
+    and the dk, dv scan per KV head."""
+    C, d, dv, G = 32, w.d, w.dv, w.Hq // w.Hkv
+    chunks = w.B * ((w.N + C - 1) // C)
+    st = (d * dv + d) * C  # one chunk's phi^T [x | 1]
+    if w.causal:
+        k1 = C * C * d + C * (C + d) + C * dv * (C + d) + C * C * dv + C * d * (C + dv) + 2 * st
+        k2 = 2 * C * d * dv + G * (2 * C * C * d + 2 * C * C * dv + st)
+    else:
+        k1 = C * d + 2 * C * d * dv + st
+        k2 = 2 * C * d * dv
+    return chunks * (w.Hkv * st + w.Hq * k1 + w.Hkv * k2)
 
 
 def measure_e2e(L, w, steps, stream, device):

@@ -23,12 +23,11 @@
 //      and computes per chunk
 //          Acc_r = mask(phi(Q_r) phi(K_r)^T) [V_r | 1] + phi(Q_r) [L_r | l_r]
 //      (numerator columns and the normaliser column);
-//   3. waits at the grid barrier, sums the earlier aggregates (causal) or
-//      all of them (non-causal) in block order into C_b, and adds
-//      phi(Q_r) [C_b | c_b] to every chunk's accumulator;
+//   3. meanwhile waits at the grid barrier, sums the earlier aggregates
+//      (causal) or all of them (non-causal) in block order into C_b, and adds
+//      phi(Q_r) [C_b | c_b] to each chunk's accumulator as soon as both are
+//      ready;
 //   4. normalises and stores.
-// After the barrier only one K = 64 product per chunk and the epilogues
-// remain; the chunk-to-chunk chain runs while the tiles are still landing.
 //
 // The state accumulator is kept transposed, [V | 1]^T phi(K) (M = 128 value
 // columns plus the normaliser row, N = 64 key features), so TMEM lane m holds
@@ -36,14 +35,13 @@
 //
 // Warp roles (576 threads; TMEM sub-partition = warp % 4):
 //   warps 0-7   transform: phi in place on K and Q tiles (tail rows zeroed);
-//               then, with the state warps, the carry sum; warps 0-3 then
-//               store the odd items' outputs
-//   warps 8-11  mask: causal mask of the score tile, bf16 in place in TMEM;
-//               then the even items' outputs
-//   warps 12-15 state: the aggregate to the workspace, the grid barrier, the
-//               running sums -> bf16 operands, the carry sum
+//               then the grid-barrier wait and the carry sum; then the
+//               outputs (warps 0-3 the even items, warps 4-7 the odd ones)
+//   warps 8-11  mask: causal mask of the score tile, bf16 in place in TMEM
+//   warps 12-15 state: the aggregate to the workspace, the grid-barrier
+//               arrival, the running sums -> bf16 operands
 //   warp 16     TMA producer
-//   warp 17     TMEM allocator and MMA issuer
+//   warp 17     TMEM allocator and MMA issuer (a fixed issue order)
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -112,6 +110,7 @@ struct Bars {
   uint64_t *p_full, *pb_full;                  // per item: score ready; masked bf16 ready
   uint64_t *acc_full;                          // per item: accumulator complete
   uint64_t *agg_full, *agg_empty;              // the aggregate is in the state; read
+  uint64_t *g_arr;                             // the grid-barrier arrival is recorded
   uint64_t *c_full;                            // the carry operand is staged
   uint64_t *drain;                             // issued products complete
 };
@@ -132,7 +131,8 @@ __device__ __forceinline__ Bars carve(uint8_t* base) {
   r.acc_full = b; b += NST;
   r.agg_full = b++;
   r.agg_empty = b++;
-  b += NST - 2;  // spare
+  r.g_arr = b++;
+  b += NST - 3;  // spare
   r.c_full = b++;
   r.drain = b++;
   return r;
@@ -156,7 +156,7 @@ __device__ __forceinline__ void store_operand_row(uint8_t* op, int row, const fl
 // fp32 in block order, rounded once to bf16 into the K-major operand; rows
 // DV+1 .. OPR-1 zeroed.  With s_out, also the final state C + base[own]
 // (own < 0: C itself) in fp32, in the [d][dv] layout.  Thread u of NT.
-template <int NT>
+template <int NT, int NF>
 __device__ __forceinline__ void gather_carry(const float4* base, int nsum, uint8_t* op, int u,
                                              const float* s0, const float* z0, float* s_out,
                                              float* z_out, int own) {
@@ -177,10 +177,10 @@ __device__ __forceinline__ void gather_carry(const float4* base, int nsum, uint8
     }
   }
 #pragma unroll 1
-  for (int b0 = 0; b0 < nsum; b0 += 4) {  // four blocks' loads in flight
-    float4 v[4][PER];
+  for (int b0 = 0; b0 < nsum; b0 += NF) {  // NF blocks' loads in flight
+    float4 v[NF][PER];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < NF; ++k) {
       if (b0 + k < nsum) {
         const float4* blk = base + (size_t)(b0 + k) * E4;
 #pragma unroll
@@ -189,7 +189,7 @@ __device__ __forceinline__ void gather_carry(const float4* base, int nsum, uint8
       }
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < NF; ++k) {
       if (b0 + k < nsum) {
 #pragma unroll
         for (int e = 0; e < PER; ++e) {
@@ -244,6 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   using L = Layout;
   __shared__ volatile int s_abort;
+  __shared__ unsigned int s_grid_old;  // the state group's grid-barrier arrival
+  __shared__ int s_grid_arrived;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int blk = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
   const int t0 = s * a.N, ntok = a.N;
@@ -297,12 +299,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (bounded) wait only raises the abort flag, and the work after a barrier
   // is skipped while the flag is up.
 
-  // The carry sum, by the transform and state warps (384 threads) between
-  // two barriers 5.
+  // The carry sum, by the transform warps (256 threads) between two
+  // barriers 5.
   auto gather_part = [&](int u) {
-    named_bar_sync(5, 384);
+    named_bar_sync(5, kXf);
     if (!*abort_flag) {
-      gather_carry<384>(agg_base, nprev, sC, u,
+      gather_carry<kXf, 2>(agg_base, nprev, sC, u,
                         a.s0 ? a.s0 + lane_idx * D * DV : nullptr,
                         a.z0 ? a.z0 + lane_idx * D : nullptr,
                         final_state ? a.s_out + lane_idx * D * DV : nullptr,
@@ -310,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         causal ? blk : -1);
       fence_proxy_async_smem();
     }
-    named_bar_sync(5, 384);
+    named_bar_sync(5, kXf);
     if (u == 0 && !*abort_flag) mbar_arrive(bars.c_full);
   };
 
@@ -432,13 +434,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         umma_commit(bars.agg_full);
         // 2. causal: per item its score, the running sum of its chunk (once
-        //    the state has been read), P V and phi(Q) L
+        //    the state has been read), P V and phi(Q) L; and phi(Q) [C | c]
+        //    for the items whose local products are issued, as soon as the
+        //    carry is staged
+        int qc = 0;
+        bool c_ready = false;
+        auto carry_products = [&](int upto) {
+          if (!c_ready) {
+            if (!mbar_test(bars.c_full, 0)) return;
+            c_ready = true;
+            tc_fence_after();
+          }
+          for (; qc < upto; ++qc) {
+            issue_qs(qc, sC, true);
+            umma_commit(&bars.acc_full[qc]);
+          }
+        };
+        // item j's products that nothing in the score -> mask -> P V chain
+        // waits for: phi(Q) L, then (no carry) the accumulator is complete,
+        // or the carry products that are ready
+        auto finish = [&](int j) {
+          const int r = j / G;
+          if (r > 0) {
+            if (!W(&bars.op_full[r])) return false;
+            issue_qs(j, sK + (r - 1) * KVT, true);
+          }
+          if (!has_carry)
+            umma_commit(&bars.acc_full[j]);
+          else
+            carry_products(j + 1);
+          return true;
+        };
         for (int j = 0; j < n_items && causal && ok; ++j) {
           const int r = j / G;
           if (!(ok = W(&bars.q_xf[j]))) break;
           issue_score(j);
           umma_commit(&bars.p_full[j]);
           if (j % G == G - 1) umma_commit(&bars.k_free[r]);
+          // the previous item's remaining products run during this mask
+          if (j > 0 && !(ok = finish(j - 1))) break;
           if (j % G == 0 && r < nlocal) {
             // the state becomes L_{r+1}
             if (!(ok = W(r == 0 ? bars.agg_empty : &bars.s_empty[r - 1]))) break;
@@ -447,16 +481,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!(ok = W(&bars.pb_full[j]))) break;
           issue_pv(j);
-          if (r > 0) {
-            if (!(ok = W(&bars.op_full[r]))) break;
-            issue_qs(j, sK + (r - 1) * KVT, true);
-          }
-          if (!has_carry) umma_commit(&bars.acc_full[j]);
         }
+        if (ok && causal && n_items > 0) ok = finish(n_items - 1);
         if (!ok || !has_carry) break;
-        // 3. phi(Q) [C | c] into every item's accumulator
-        if (!W(bars.c_full)) break;
-        for (int j = 0; j < n_items; ++j) {
+        // 3. phi(Q) [C | c] into the remaining accumulators
+        if (!c_ready && !W(bars.c_full)) break;
+        for (int j = qc; j < n_items; ++j) {
           if (!causal && !W(&bars.q_xf[j])) break;
           issue_qs(j, sC, causal);
           umma_commit(&bars.acc_full[j]);
@@ -493,12 +523,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_sync(1, kXf);
       if (x == 0 && !*abort_flag) mbar_arrive(is_kv ? &bars.kv_xf[r] : &bars.q_xf[j]);
     }
-    if (gath) gather_part(x);
-    // warps 0-3: the odd items' outputs
-    if (warp < 4) {
-      bool ok = true;
-      for (int j = 1; j < n_items && ok; j += 2) ok = epilogue(j, x);
+    if (gath) {
+      // the grid barrier (after the state group has arrived), then the carry
+      if (x == 0 && mbar_wait(bars.g_arr, 0, abort_flag, a.err, kWaitLimitNs) &&
+          s_grid_arrived && (nprev > 0 || final_state))
+        grid_wait(s_grid_old, abort_flag, a.err, kWaitLimitNs);
+      gather_part(x);
     }
+    // the outputs: warps 0-3 the even items, warps 4-7 the odd ones
+    bool ok = true;
+    for (int j = warp >> 2; j < n_items && ok; j += 2) ok = epilogue(j, x & 127);
   } else if (warp < 12) {
     // ---------------------------------------------------- mask warpgroup
     const int x = tid - 256, sp = warp & 3;
@@ -511,29 +545,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (!*abort_flag) {
         const uint32_t t_p = tmem + TM_P + ((uint32_t)(sp * 32) << 16);
+        // two 32-column blocks per TMEM round trip; fp32 block b becomes
+        // packed bf16 block b (columns [16b, 16b+16)), so every store lands
+        // on columns that are already read
+        auto pack_block = [&](int b, const float (&r)[32], uint32_t (&pk)[16]) {
+          if (b < sp) {  // warp-uniform: a block entirely left of the diagonal
 #pragma unroll
-        for (int b = 0; b < kChunk / 32; ++b) {
-          uint32_t pk[16];
-          if (b <= sp) {  // warp-uniform: blocks right of the diagonal are all zero
-            float r[32];
-            tmem_ld32(t_p + b * 32, r);
-            tmem_wait_ld();
-            if (b < sp) {  // block entirely left of the diagonal
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(r[2 * e], r[2 * e + 1]);
+          } else if (b == sp) {  // the diagonal block
 #pragma unroll
-              for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(r[2 * e], r[2 * e + 1]);
-            } else {  // the diagonal block
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const float lo = (b * 32 + 2 * e > row) ? 0.0f : r[2 * e];
-                const float hi = (b * 32 + 2 * e + 1 > row) ? 0.0f : r[2 * e + 1];
-                pk[e] = pack_bf16x2(lo, hi);
-              }
+            for (int e = 0; e < 16; ++e) {
+              const float lo = (b * 32 + 2 * e > row) ? 0.0f : r[2 * e];
+              const float hi = (b * 32 + 2 * e + 1 > row) ? 0.0f : r[2 * e + 1];
+              pk[e] = pack_bf16x2(lo, hi);
             }
-          } else {
+          } else {  // right of the diagonal: zero
 #pragma unroll
             for (int e = 0; e < 16; ++e) pk[e] = 0u;
           }
-          tmem_st16(t_p + b * 16, pk);
+        };
+#pragma unroll
+        for (int b0 = 0; b0 < kChunk / 32; b0 += 2) {
+          float ra[32], rb[32];
+          uint32_t pk[16];
+          if (b0 <= sp) tmem_ld32(t_p + b0 * 32, ra);
+          if (b0 + 1 <= sp) tmem_ld32(t_p + (b0 + 1) * 32, rb);
+          if (b0 <= sp) tmem_wait_ld();
+          pack_block(b0, ra, pk);
+          tmem_st16(t_p + b0 * 16, pk);
+          pack_block(b0 + 1, rb, pk);
+          tmem_st16(t_p + (b0 + 1) * 16, pk);
         }
         tmem_wait_st();
       }
@@ -541,8 +582,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_sync(2, 128);
       if (x == 0 && !*abort_flag) mbar_arrive(&bars.pb_full[j]);
     }
-    bool ok = true;
-    for (int j = 0; j < n_items && ok; j += 2) ok = epilogue(j, x);
   } else if (warp < 16) {
     // -------------------------------------------------- state warpgroup
     // TMEM state lane m: row m of [S | z]^T (m < 64: column m of S; m = 64:
@@ -582,9 +621,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         dst[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
     }
     named_bar_sync(3, 128);
-    unsigned int grid_old = 0;
-    bool arrived = false;
-    if (y == 0) arrived = grid_arrive(&grid_old, abort_flag, a.err);
+    if (y == 0) {
+      // every CTA arrives exactly once, on every path; the transform group
+      // waits at the barrier
+      unsigned int grid_old = 0;
+      const bool arrived = grid_arrive(&grid_old, abort_flag, a.err);
+      s_grid_old = grid_old;
+      s_grid_arrived = arrived ? 1 : 0;
+      mbar_arrive(bars.g_arr);
+    }
     // 2. causal: the running sums L_1 .. L_{Ri-1}, each staged into the K
     //    slot of the chunk before once that slot's scores are done
     for (int r = 0; r < nlocal; ++r) {
@@ -598,14 +643,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       named_bar_sync(3, 128);
       if (y == 0 && !*abort_flag) mbar_arrive(&bars.op_full[r + 1]);
-    }
-    // 3. the carry, once every CTA has published
-    if (gath) {
-      // (a carry of S0 alone needs no other block)
-      if (y == 0 && arrived && (nprev > 0 || final_state))
-        grid_wait(grid_old, abort_flag, a.err, kWaitLimitNs);
-      named_bar_sync(3, 128);
-      gather_part(256 + y);
     }
   }
 

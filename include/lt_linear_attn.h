@@ -338,12 +338,14 @@ LT_API lt_status_t lt_linear_attn_state_carry(const float *S_all, const float *z
  * dout   the output's layout and element type; must not overlap q, k, v.
  * dq, dk, dv  q's, k's and v's layouts and element type (16-byte aligned,
  *        device); written whole; must not overlap any input or each other.
- * Evaluation: two chunked scans with fp32 FMA arithmetic (32-token chunks):
- * a forward scan per (sequence, query head) for dq, and a reverse scan per
- * (sequence, KV head) for dk, dv ("Why Stream Wins at Ultra-Long Context",
- * section 4.2: the backward recurrence of a linear scan).  Scratch: a
- * stream-ordered workspace of tokens * H_q * (dv + 1) floats, released
- * before return.
+ * Evaluation: two chunked scans with fp32 FMA arithmetic (32-token chunks),
+ * a forward scan for dq and a reverse scan for dk, dv ("Why Stream Wins at
+ * Ultra-Long Context", section 4.2: the backward recurrence of a linear
+ * scan), each sequence cut into blocks of whole chunks that run on their own
+ * CTAs from carried block sums (added in block order: the results do not
+ * depend on scheduling).  Scratch: a stream-ordered workspace of
+ * tokens * H_q * (dv + 1) + B * (H_q + H_kv) * nb * (d * dv + d) floats (nb
+ * blocks per sequence, at most twice the SM count), released before return.
  * Returns as lt_linear_attn_fwd.
  */
 LT_API lt_status_t lt_linear_attn_bwd(const void *q, const void *k, const void *v,
