@@ -52,6 +52,18 @@ __global__ void __launch_bounds__(kT) lt_decode_kernel(const DecodeLaunch a) {
   const int G = a.Hq / a.Hkv;
   const int cg = tid % CG, rg = tid / CG;
   const size_t kv = (size_t)b * a.Hkv + g;
+  float* S = a.S + kv * D * DV;
+  float* z = a.z + kv * D;
+  // this thread's state rows first: their loads are in flight while q, k, v
+  // are staged
+  float4 rows[RPT];
+  float zr[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const int row = rg * RPT + r;
+    rows[r] = *reinterpret_cast<const float4*>(S + (size_t)row * DV + cg * 4);
+    zr[r] = cg == 0 ? z[row] : 0.0f;
+  }
 
   for (int e = tid; e < D; e += kT) s_pk[e] = phi_dec(ld_in<BF16>(a.k, kv * D + e));
   for (int e = tid; e < DV; e += kT) s_v[e] = ld_in<BF16>(a.v, kv * DV + e);
@@ -59,15 +71,11 @@ __global__ void __launch_bounds__(kT) lt_decode_kernel(const DecodeLaunch a) {
     s_pq[e] = phi_dec(ld_in<BF16>(a.q, ((size_t)b * a.Hq + (size_t)g * G) * D + e));
   __syncthreads();
 
-  float* S = a.S + kv * D * DV;
-  float* z = a.z + kv * D;
   const float4 v4 = *reinterpret_cast<const float4*>(&s_v[cg * 4]);
-  float4 rows[RPT];
-  float zr[RPT];
 #pragma unroll
   for (int r = 0; r < RPT; ++r) {
     const int row = rg * RPT + r;
-    float4 x = *reinterpret_cast<const float4*>(S + (size_t)row * DV + cg * 4);
+    float4 x = rows[r];
     const float pk = s_pk[row];
     x.x = fmaf(pk, v4.x, x.x);
     x.y = fmaf(pk, v4.y, x.y);
@@ -75,9 +83,8 @@ __global__ void __launch_bounds__(kT) lt_decode_kernel(const DecodeLaunch a) {
     x.w = fmaf(pk, v4.w, x.w);
     *reinterpret_cast<float4*>(S + (size_t)row * DV + cg * 4) = x;
     rows[r] = x;
-    zr[r] = 0.0f;
     if (cg == 0) {
-      zr[r] = z[row] + pk;
+      zr[r] += pk;
       z[row] = zr[r];
     }
   }
