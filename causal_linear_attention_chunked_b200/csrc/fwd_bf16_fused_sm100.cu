@@ -18,9 +18,10 @@
 //      applies phi; accumulates A_b = sum_r dS_r on the tensor cores as soon
 //      as the K/V tiles are ready, publishes it to the workspace and arrives
 //      at the launch's grid barrier (without waiting);
-//   2. recomputes the running sums L_1 .. L_{R-1} (one more state product
-//      per chunk, K and V are still resident), stages each as a bf16 operand,
-//      and computes per chunk
+//   2. keeps the running sums L_1 .. L_{R-1} that the aggregate passes
+//      through (parked in accumulator columns that are not yet in use),
+//      stages each as a bf16 operand once its K slot is free, and computes
+//      per chunk
 //          Acc_r = mask(phi(Q_r) phi(K_r)^T) [V_r | 1] + phi(Q_r) [L_r | l_r]
 //      (numerator columns and the normaliser column);
 //   3. meanwhile waits at the grid barrier, sums the earlier aggregates
@@ -38,8 +39,9 @@
 //               then the grid-barrier wait and the carry sum; then the
 //               outputs (warps 0-3 the even items, warps 4-7 the odd ones)
 //   warps 8-11  mask: causal mask of the score tile, bf16 in place in TMEM
-//   warps 12-15 state: the aggregate to the workspace, the grid-barrier
-//               arrival, the running sums -> bf16 operands
+//   warps 12-15 state: the running sums parked as they pass, the aggregate
+//               to the workspace, the grid-barrier arrival, the running sums
+//               -> bf16 operands
 //   warp 16     TMA producer
 //   warp 17     TMEM allocator and MMA issuer (a fixed issue order)
 #include <cuda.h>
@@ -104,12 +106,12 @@ struct Layout {
 // Every barrier completes at most once per launch (phase 0).
 struct Bars {
   uint64_t *q_full, *q_xf, *kv_full, *kv_xf;   // per item / chunk: landed, phi applied
-  uint64_t *s_full, *s_empty;                  // per chunk r: L_{r+1} in the state; read
+  uint64_t *s_full, *s_empty;                  // per chunk r: L_{r+1} in the state; parked
   uint64_t *k_free;                            // per chunk: K slot r's scores are done
   uint64_t *op_full;                           // per chunk r >= 1: L_r staged in K slot r-1
   uint64_t *p_full, *pb_full;                  // per item: score ready; masked bf16 ready
   uint64_t *acc_full;                          // per item: accumulator complete
-  uint64_t *agg_full, *agg_empty;              // the aggregate is in the state; read
+  uint64_t *agg_full;                          // the aggregate is in the state
   uint64_t *g_arr;                             // the grid-barrier arrival is recorded
   uint64_t *c_full;                            // the carry operand is staged
   uint64_t *drain;                             // issued products complete
@@ -130,9 +132,8 @@ __device__ __forceinline__ Bars carve(uint8_t* base) {
   r.pb_full = b; b += NST;
   r.acc_full = b; b += NST;
   r.agg_full = b++;
-  r.agg_empty = b++;
   r.g_arr = b++;
-  b += NST - 3;  // spare
+  b += NST - 2;  // spare
   r.c_full = b++;
   r.drain = b++;
   return r;
@@ -266,8 +267,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // every block with a carry (earlier blocks or a given state) gathers it
   const bool gath = nprev > 0 || a.s0 != nullptr;
   const size_t lane_idx = (size_t)s * a.Hkv + g;
-  // causal: running sums L_1 .. L_{Ri-1} for the chunks after the first
-  const int nlocal = causal ? Ri - 1 : 0;
   const float4* agg_base =
       reinterpret_cast<const float4*>(a.ws) + (size_t)(s * a.Hkv + g) * a.nb * E4;
 
@@ -426,17 +425,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         return ok;
       };
       do {
-        // 1. the block aggregate (what the other CTAs wait for)
+        // 1. the state chunk by chunk (causal: after chunk r it holds
+        //    L_{r+1}, which the state warps park before the next product);
+        //    after the last chunk it is the block aggregate (what the other
+        //    CTAs wait for)
         bool ok = true;
         for (int r = 0; r < Ri && ok; ++r) {
-          if ((ok = W(&bars.kv_xf[r]))) issue_ds(r, r > 0);
+          if (!(ok = W(&bars.kv_xf[r]))) break;
+          if (causal && r > 0 && !(ok = W(&bars.s_empty[r - 1]))) break;
+          issue_ds(r, r > 0);
+          if (causal && r + 1 < Ri) umma_commit(&bars.s_full[r]);
         }
         if (!ok) break;
         umma_commit(bars.agg_full);
-        // 2. causal: per item its score, the running sum of its chunk (once
-        //    the state has been read), P V and phi(Q) L; and phi(Q) [C | c]
-        //    for the items whose local products are issued, as soon as the
-        //    carry is staged
+        // 2. causal: per item its score, P V (the first item of a chunk after
+        //    the chunk's running sum has left its accumulator) and phi(Q) L;
+        //    and phi(Q) [C | c] for the items whose local products are
+        //    issued, as soon as the carry is staged
         int qc = 0;
         bool c_ready = false;
         auto carry_products = [&](int upto) {
@@ -473,13 +478,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j % G == G - 1) umma_commit(&bars.k_free[r]);
           // the previous item's remaining products run during this mask
           if (j > 0 && !(ok = finish(j - 1))) break;
-          if (j % G == 0 && r < nlocal) {
-            // the state becomes L_{r+1}
-            if (!(ok = W(r == 0 ? bars.agg_empty : &bars.s_empty[r - 1]))) break;
-            issue_ds(r, r > 0);
-            umma_commit(&bars.s_full[r]);
-          }
           if (!(ok = W(&bars.pb_full[j]))) break;
+          if (r > 0 && j % G == 0 && !(ok = W(&bars.op_full[r]))) break;
           issue_pv(j);
         }
         if (ok && causal && n_items > 0) ok = finish(n_items - 1);
@@ -607,12 +607,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       named_bar_sync(3, 128);
     };
-    // 1. the block aggregate: release the state, publish, arrive at the grid
-    //    barrier (every CTA exactly once, on every path).  The group barrier
-    //    orders every thread's aggregate writes before the arriving thread's
-    //    release at gpu scope (release is cumulative).
+    // 1. causal: the running sums L_1 .. L_{Ri-1} as the state passes
+    //    through them, each parked in the accumulator columns of the first
+    //    item of its chunk (unused until that item's P V)
+    for (int r = 0; r + 1 < Ri && causal; ++r) {
+      read_state(&bars.s_full[r]);
+      if (y == 0 && !*abort_flag) mbar_arrive(&bars.s_empty[r]);
+      if (has_rows && !*abort_flag) {
+        const uint32_t t_park = tmem + TM_ACC + (r + 1) * G * ACCW + ((uint32_t)(sp * 32) << 16);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t bits[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) bits[e] = __float_as_uint(v[16 * q4 + e]);
+          tmem_st16(t_park + 16 * q4, bits);
+        }
+        tmem_wait_st();
+      }
+    }
+    // 2. the block aggregate: publish, arrive at the grid barrier (every CTA
+    //    exactly once, on every path).  The group barrier orders every
+    //    thread's aggregate writes before the arriving thread's release at
+    //    gpu scope (release is cumulative).
     read_state(bars.agg_full);
-    if (y == 0 && !*abort_flag) mbar_arrive(bars.agg_empty);
     if (publish && has_rows && m <= DV && !*abort_flag) {
       float4* dst = reinterpret_cast<float4*>(
           a.ws + (((size_t)(s * a.Hkv + g) * a.nb + blk) * E + (size_t)m * D));
@@ -622,27 +639,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     named_bar_sync(3, 128);
     if (y == 0) {
-      // every CTA arrives exactly once, on every path; the transform group
-      // waits at the barrier
+      // the transform group waits at the barrier
       unsigned int grid_old = 0;
       const bool arrived = grid_arrive(&grid_old, abort_flag, a.err);
       s_grid_old = grid_old;
       s_grid_arrived = arrived ? 1 : 0;
       mbar_arrive(bars.g_arr);
     }
-    // 2. causal: the running sums L_1 .. L_{Ri-1}, each staged into the K
-    //    slot of the chunk before once that slot's scores are done
-    for (int r = 0; r < nlocal; ++r) {
-      read_state(&bars.s_full[r]);
-      if (y == 0) {
-        if (!*abort_flag) mbar_arrive(&bars.s_empty[r]);
-        mbar_wait(&bars.k_free[r], 0, abort_flag, a.err, kWaitLimitNs);
+    // 3. causal: each parked running sum L_r, staged into the K slot of the
+    //    chunk before once that slot's scores are done (this frees its
+    //    accumulator columns for P V)
+    for (int r = 1; r < Ri && causal; ++r) {
+      if (y == 0) mbar_wait(&bars.k_free[r - 1], 0, abort_flag, a.err, kWaitLimitNs);
+      named_bar_sync(3, 128);
+      tc_fence_after();
+      if (has_rows && !*abort_flag) {
+        const uint32_t t_park = tmem + TM_ACC + r * G * ACCW + ((uint32_t)(sp * 32) << 16);
+        tmem_ld32(t_park, *reinterpret_cast<float(*)[32]>(v));
+        tmem_ld32(t_park + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+        tmem_wait_ld();
+        if (m < OPR) store_operand_row(sK + (r - 1) * KVT, m, v);
       }
-      named_bar_sync(3, 128);
-      if (has_rows && m < OPR && !*abort_flag) store_operand_row(sK + r * KVT, m, v);
       fence_proxy_async_smem();
+      tc_fence_before();
       named_bar_sync(3, 128);
-      if (y == 0 && !*abort_flag) mbar_arrive(&bars.op_full[r + 1]);
+      if (y == 0 && !*abort_flag) mbar_arrive(&bars.op_full[r]);
     }
   }
 
