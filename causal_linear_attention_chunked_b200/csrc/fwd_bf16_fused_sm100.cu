@@ -239,7 +239,8 @@ __device__ __forceinline__ void gather_carry(const float4* base, int nsum, uint8
 __global__ void __launch_bounds__(kThreads, 1)
     lt_fused_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const FusedArgs a) {
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_o, const FusedArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -315,35 +316,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (u == 0 && !*abort_flag) mbar_arrive(bars.c_full);
   };
 
-  // Accumulator of item j -> normalised bf16 row -> global, one thread per
-  // row (TMEM lane = chunk row); x in [0, 128).  No group barrier inside.
-  auto epilogue = [&](int j, int x) -> bool {
+  // Accumulator of item j -> normalised bf16 row, one thread per row (TMEM
+  // lane = chunk row); x in [0, 128) of the group of four warps that passes
+  // named barrier `nbar`.  A whole chunk is staged in item j's Q slot (its
+  // last reader, the item's final product, is complete) and written by one
+  // TMA store; the rows of a ragged last chunk are stored directly (a tile
+  // would run into the next sequence).  Returns false once the abort flag is
+  // up (read after the group barrier, so the group agrees).
+  auto epilogue = [&](int j, int x, int nbar) -> bool {
     const int sp = (x >> 5) & 3, row = x;
     const int r = j / G, h = j % G, c = c0 + r;
-    if (!mbar_wait(&bars.acc_full[j], 0, abort_flag, a.err, kWaitLimitNs)) return false;
+    const bool ok = mbar_wait(&bars.acc_full[j], 0, abort_flag, a.err, kWaitLimitNs);
     tc_fence_after();
-    const uint32_t t_acc = tmem + TM_ACC + j * ACCW + ((uint32_t)(sp * 32) << 16);
     uint32_t pk[DV / 2];
-    float n[32];
-    const float den = tmem_ld1(t_acc + DV);
-    tmem_ld32(t_acc, n);
-    tmem_wait_ld();
-    const float inv = 1.0f / (den + a.eps);
+    if (ok) {
+      const uint32_t t_acc = tmem + TM_ACC + j * ACCW + ((uint32_t)(sp * 32) << 16);
+      float n[32];
+      const float den = tmem_ld1(t_acc + DV);
+      tmem_ld32(t_acc, n);
+      tmem_wait_ld();
+      const float inv = 1.0f / (den + a.eps);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(n[2 * e] * inv, n[2 * e + 1] * inv);
-    tmem_ld32(t_acc + 32, n);
-    tmem_wait_ld();
+      for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(n[2 * e] * inv, n[2 * e + 1] * inv);
+      tmem_ld32(t_acc + 32, n);
+      tmem_wait_ld();
 #pragma unroll
-    for (int e = 0; e < 16; ++e) pk[16 + e] = pack_bf16x2(n[2 * e] * inv, n[2 * e + 1] * inv);
+      for (int e = 0; e < 16; ++e) pk[16 + e] = pack_bf16x2(n[2 * e] * inv, n[2 * e + 1] * inv);
+    }
     const int valid = min(kChunk, ntok - c * kChunk);
-    if (row < valid) {
+    if (valid == kChunk) {  // uniform over the group
+      uint8_t* tile = sQ + j * QT;
+      if (ok) {
+#pragma unroll
+        for (int q = 0; q < DV / 8; ++q)
+          *reinterpret_cast<uint4*>(tile + sw128_off(row, q)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(nbar, 128);
+      if (x == 0 && !*abort_flag) {
+        tma_store_3d(&tm_o, tile, 0, g * G + h, t0 + c * kChunk);
+        bulk_commit_group();
+      }
+      return !*abort_flag;
+    }
+    if (ok && row < valid) {
       uint4* orow = reinterpret_cast<uint4*>(
           a.out + ((size_t)(t0 + c * kChunk + row) * a.Hq + (size_t)(g * G + h)) * DV);
 #pragma unroll
       for (int q = 0; q < DV / 8; ++q)
         orow[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
     }
-    return true;
+    return ok;
   };
 
   if (warp == 16) {
@@ -354,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_o);
       for (int r = 0; r < Ri; ++r) {
         const int c = c0 + r;
         mbar_arrive_expect_tx(&bars.kv_full[r], KT + VT);
@@ -530,9 +555,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         grid_wait(s_grid_old, abort_flag, a.err, kWaitLimitNs);
       gather_part(x);
     }
-    // the outputs: warps 0-3 the even items, warps 4-7 the odd ones
+    // the outputs: warps 0-3 the even items, warps 4-7 the odd ones (named
+    // barriers 6 and 7); the issuing thread waits for its TMA stores
     bool ok = true;
-    for (int j = warp >> 2; j < n_items && ok; j += 2) ok = epilogue(j, x & 127);
+    for (int j = warp >> 2; j < n_items && ok; j += 2) ok = epilogue(j, x & 127, 6 + (warp >> 2));
+    if ((x & 127) == 0) bulk_wait_all();
   } else if (warp < 12) {
     // ---------------------------------------------------- mask warpgroup
     const int x = tid - 256, sp = warp & 3;
@@ -700,10 +727,11 @@ cudaError_t launch_fwd_bf16_block_fused_state(const FwdLaunch& p, int nb, float*
                                               const float* s0, const float* z0, float* s_out,
                                               float* z_out, cudaStream_t stream) {
   if (ws == nullptr) return cudaErrorInvalidValue;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
       !make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64) ||
-      !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64))
+      !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64) ||
+      !make_tmap_3d(&to, p.out, DV, p.Hq, p.total_tokens, 64))
     return cudaErrorInvalidValue;
   FusedArgs a;
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
@@ -735,7 +763,7 @@ cudaError_t launch_fwd_bf16_block_fused_state(const FwdLaunch& p, int nb, float*
   at[0].val.cooperative = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fk, tq, tk, tv, a);
+  return cudaLaunchKernelEx(&cfg, fk, tq, tk, tv, to, a);
 }
 
 }  // namespace lt
