@@ -174,11 +174,14 @@ __device__ __forceinline__ void sum_aggregates(const float4* base, int nsum, flo
 // each from the aggregates of the state launch.  Without it (one block per
 // sequence, e.g. packed inputs) the carry code is left out of the image: the
 // instruction working set of the warp roles matters to this kernel's speed.
-template <bool kCarry>
+// kTmaOut (non-causal launches): whole output tiles are staged in their Q
+// slot and written by TMA stores; the causal image has only the row stores.
+template <bool kCarry, bool kTmaOut>
 __global__ void __launch_bounds__(kThreads, 1)
     lt_block_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const BlockArgs a) {
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_o, const BlockArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -263,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
+      if (kTmaOut) prefetch_tmap(&tm_o);
       int q_issued = 0, kv_issued = 0;
       bool ok = true;
       auto load_kv = [&](int r) -> bool {
@@ -429,7 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           issue_qs(tmem + TM_ACC + as * ACCW, qs, false);
           umma_commit(&bars.acc_full[as]);
-          umma_commit(&bars.q_empty[qs]);
+          // (with TMA output the epilogue releases the Q slot: it stages the
+          // output tile there)
+          if (!kTmaOut) umma_commit(&bars.q_empty[qs]);
         }
       }
       umma_commit(bars.drain);
@@ -525,6 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (x == 0) mbar_arrive(&bars.pb_full[as]);
       return true;
     };
+    int q_pend = -1;  // thread 0: the item whose stored tile still holds its Q slot
     auto epilogue = [&](int j) -> bool {
       const int r = j / G, h = j % G, as = j & 1, c = c0 + r;
       if (!mbar_wait(&bars.acc_full[as], (j >> 1) & 1, abort_flag, a.err, kWaitLimitNs))
@@ -556,13 +563,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       named_bar_sync(2, 128);
       if (x == 0) mbar_arrive(&bars.acc_empty[as]);
+      // Non-causal: the item's Q slot is free (its last reader, phi(Q)
+      // [S|z], is complete), so a whole chunk is staged there (128-byte
+      // swizzle) and written by one TMA store; the slot is released at the
+      // next item's epilogue, when the store has long read it.  Causal: the
+      // Q slots stay with the producer (the chunk chain paces the Q stream
+      // and a slot held by an epilogue stalls it), rows are stored directly,
+      // as are the rows of a ragged last chunk (a tile would run into the
+      // next sequence).
       const int valid = min(kChunk, ntok - c * kChunk);
-      if (row < valid) {
-        uint4* orow = reinterpret_cast<uint4*>(
-            a.out + ((size_t)(t0 + c * kChunk + row) * a.Hq + (size_t)(g * G + h)) * DV);
+      const int qs = j % NQ;
+      auto release_pending = [&]() {
+        if (q_pend >= 0) {
+          bulk_wait_read_all();
+          mbar_arrive(&bars.q_empty[q_pend % NQ]);
+          q_pend = -1;
+        }
+      };
+      if (kTmaOut && valid == kChunk) {
+        uint8_t* tile = sQ + qs * QT;
 #pragma unroll
         for (int q = 0; q < DV / 8; ++q)
-          orow[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          *reinterpret_cast<uint4*>(tile + sw128_off(row, q)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(2, 128);
+        if (x == 0) {
+          release_pending();
+          tma_store_3d(&tm_o, tile, 0, g * G + h, t0 + c * kChunk);
+          bulk_commit_group();
+          q_pend = j;
+        }
+      } else {
+        if (row < valid) {
+          uint4* orow = reinterpret_cast<uint4*>(
+              a.out + ((size_t)(t0 + c * kChunk + row) * a.Hq + (size_t)(g * G + h)) * DV);
+#pragma unroll
+          for (int q = 0; q < DV / 8; ++q)
+            orow[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+        if (kTmaOut && x == 0) {
+          release_pending();
+          mbar_arrive(&bars.q_empty[qs]);
+        }
       }
       return true;
     };
@@ -571,6 +614,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t <= n_items && ok; ++t) {
       if (causal && t < n_items) ok = mask_p(t);
       if (ok && t > 0) ok = epilogue(t - 1);
+    }
+    if (kTmaOut && x == 0) {
+      if (q_pend >= 0) {
+        bulk_wait_read_all();
+        mbar_arrive(&bars.q_empty[q_pend % NQ]);
+      }
+      bulk_wait_all();  // every output store has landed
     }
   } else if (warp < 16) {
     // -------------------------------------------------- state warpgroup
@@ -673,10 +723,11 @@ bool block_supported(const FwdLaunch& p) { return p.d == 64 && p.dv == 64; }
 namespace {
 cudaError_t launch_block(const FwdLaunch& p, int nb, const float* ws, bool carry_pre,
                          cudaStream_t stream) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
       !make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64) ||
-      !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64))
+      !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64) ||
+      !make_tmap_3d(&to, p.out, DV, p.Hq, p.total_tokens, 64))
     return cudaErrorInvalidValue;
   BlockArgs a;
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
@@ -693,10 +744,13 @@ cudaError_t launch_block(const FwdLaunch& p, int nb, const float* ws, bool carry
   a.eps = p.eps;
   a.total_tokens = (int)p.total_tokens;
   a.err = p.err;
-  auto fk = a.ws != nullptr ? lt_block_fwd_kernel<true> : lt_block_fwd_kernel<false>;
+  const bool tma_out = p.causal == 0;
+  auto fk = a.ws != nullptr
+                ? (tma_out ? lt_block_fwd_kernel<true, true> : lt_block_fwd_kernel<true, false>)
+                : (tma_out ? lt_block_fwd_kernel<false, true> : lt_block_fwd_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  fk<<<dim3(nb, p.Hkv, p.B), kThreads, SMEM, stream>>>(tq, tk, tv, a);
+  fk<<<dim3(nb, p.Hkv, p.B), kThreads, SMEM, stream>>>(tq, tk, tv, to, a);
   return cudaGetLastError();
 }
 }  // namespace

@@ -42,7 +42,7 @@
 //   warps 12-15 state: the running sums parked as they pass, the aggregate
 //               to the workspace, the grid-barrier arrival, the running sums
 //               -> bf16 operands
-//   warp 16     TMA producer
+//   warp 16     TMA producer (every load issued at kernel entry)
 //   warp 17     TMEM allocator and MMA issuer (a fixed issue order)
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -279,11 +279,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   Bars bars = carve(smem + L::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_BAR + L::NBARS * 8);
 
-  if (tid == 0) {
+  if (tid == 16 * 32) {
+    // the producer thread initialises the barriers and issues every tile
+    // load before the CTA-wide setup (every tile has its own slot: K/V of
+    // every chunk first, the state products need them, then every Q tile);
+    // the other threads use the barriers after the barrier below
     s_abort = 0;
     uint64_t* b = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
     for (int i = 0; i < L::NBARS; ++i) mbar_init(&b[i], 1);
     fence_mbar_init();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_o);
+    for (int r = 0; r < Ri; ++r) {
+      const int c = c0 + r;
+      mbar_arrive_expect_tx(&bars.kv_full[r], KT + VT);
+      tma_load_3d(sK + r * KVT, &tm_k, &bars.kv_full[r], 0, g, t0 + c * kChunk);
+      tma_load_3d(sV + r * KVT, &tm_v, &bars.kv_full[r], 0, g, t0 + c * kChunk);
+    }
+    for (int j = 0; j < n_items; ++j) {
+      const int r = j / G, h = j % G, c = c0 + r;
+      mbar_arrive_expect_tx(&bars.q_full[j], QT);
+      tma_load_3d(sQ + j * QT, &tm_q, &bars.q_full[j], 0, g * G + h, t0 + c * kChunk);
+    }
   }
   init_ones_block(sOnes, tid, kThreads);
   fence_proxy_async_smem();
@@ -371,26 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp == 16) {
-    // ------------------------------------------------------------ producer
-    // Every tile has its own slot: K/V of every chunk first (the state
-    // products need them), then every Q tile.
-    if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      prefetch_tmap(&tm_o);
-      for (int r = 0; r < Ri; ++r) {
-        const int c = c0 + r;
-        mbar_arrive_expect_tx(&bars.kv_full[r], KT + VT);
-        tma_load_3d(sK + r * KVT, &tm_k, &bars.kv_full[r], 0, g, t0 + c * kChunk);
-        tma_load_3d(sV + r * KVT, &tm_v, &bars.kv_full[r], 0, g, t0 + c * kChunk);
-      }
-      for (int j = 0; j < n_items; ++j) {
-        const int r = j / G, h = j % G, c = c0 + r;
-        mbar_arrive_expect_tx(&bars.q_full[j], QT);
-        tma_load_3d(sQ + j * QT, &tm_q, &bars.q_full[j], 0, g * G + h, t0 + c * kChunk);
-      }
-    }
+    // producer: its loads were issued before the setup barrier
     __syncwarp();
   } else if (warp == 17) {
     // ---------------------------------------------------------- MMA issuer
