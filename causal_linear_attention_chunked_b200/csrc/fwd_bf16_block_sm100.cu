@@ -85,19 +85,27 @@ __device__ __forceinline__ bool seq_bounds(const BlockArgs& a, int s, int& t0, i
 // ========================================================================
 constexpr int kThreads = 576;
 constexpr int kXf = 256;  // transform threads (warps 0-7, two per SM sub-partition)
-constexpr int NQ = 4, NKV = 4;
+constexpr int NQ = 4;
+constexpr int OSTT = kChunk * DV * 2;  // one output staging tile
 // two score tiles (item j uses j & 1), two accumulators, the running state
 constexpr int TM_P = 0, TM_ACC = 2 * kChunk, TM_S = TM_ACC + 2 * ACCW, TM_COLS = 512;
 static_assert(TM_S + ACCW <= TM_COLS, "TMEM budget");
-constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + NQ * QT;  // stage st: [K][V] at st*KVT
-constexpr int OFF_ONES = OFF_KV + NKV * KVT;
-constexpr int OFF_SOP = OFF_ONES + ONEST;
-constexpr int OFF_Z = OFF_SOP + SOPT;
-constexpr int OFF_BAR = OFF_Z + D * 4;
-constexpr int NBARS = 3 * NQ + 3 * NKV + 2 * 2 + 2 + 2 + 2 * 2 + 1;
-constexpr int SMEM = OFF_BAR + NBARS * 8 + 16 + 1024;
-static_assert(SMEM <= 232448, "shared memory budget");
+// Shared-memory layout.  kTma (the TMA-store image) trades one of the four
+// K/V stages for two output staging tiles.
+template <bool kTma>
+struct BL {
+  static constexpr int NKV = kTma ? 3 : 4;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KV = OFF_Q + NQ * QT;  // stage st: [K][V] at st*KVT
+  static constexpr int OFF_ONES = OFF_KV + NKV * KVT;
+  static constexpr int OFF_SOP = OFF_ONES + ONEST;
+  static constexpr int OFF_Z = OFF_SOP + SOPT;
+  static constexpr int OFF_OST = (OFF_Z + D * 4 + 1023) & ~1023;  // kTma: two staging tiles
+  static constexpr int OFF_BAR = kTma ? OFF_OST + 2 * OSTT : OFF_Z + D * 4;
+  static constexpr int NBARS = 3 * NQ + 3 * NKV + 2 * 2 + 2 + 2 + 2 * 2 + 1;
+  static constexpr int SMEM = OFF_BAR + NBARS * 8 + 16 + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
 
 struct Bars {
   uint64_t *q_full, *q_empty, *q_xf, *kv_full, *kv_empty, *kv_xf;
@@ -105,6 +113,7 @@ struct Bars {
   uint64_t *s_full, *s_empty, *acc_full, *acc_empty, *drain;
 };
 
+template <int NKV>
 __device__ __forceinline__ Bars carve(uint8_t* base) {
   uint64_t* b = reinterpret_cast<uint64_t*>(base);
   Bars r;
@@ -174,8 +183,10 @@ __device__ __forceinline__ void sum_aggregates(const float4* base, int nsum, flo
 // each from the aggregates of the state launch.  Without it (one block per
 // sequence, e.g. packed inputs) the carry code is left out of the image: the
 // instruction working set of the warp roles matters to this kernel's speed.
-// kTmaOut (non-causal launches): whole output tiles are staged in their Q
-// slot and written by TMA stores; the causal image has only the row stores.
+// kTmaOut (dense non-causal launches): whole output tiles are staged in one
+// of two staging tiles and written by TMA stores through a 4-D map (d, head,
+// token, sequence) that clips a ragged last chunk at the sequence end; the
+// other images have only the row stores.
 template <bool kCarry, bool kTmaOut>
 __global__ void __launch_bounds__(kThreads, 1)
     lt_block_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -185,6 +196,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
+  using Lo = BL<kTmaOut>;
+  constexpr int NKV = Lo::NKV;
   __shared__ volatile int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int blk = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
@@ -204,12 +217,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // CTA reads only Q
   const bool nc_from_ws = !causal && a.ws != nullptr;
 
-  uint8_t* sQ = smem + OFF_Q;
-  uint8_t* sK = smem + OFF_KV;
-  uint8_t* sV = smem + OFF_KV + KT;
-  uint8_t* sSOP = smem + OFF_SOP;
-  Bars bars = carve(smem + OFF_BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + NBARS * 8);
+  uint8_t* sQ = smem + Lo::OFF_Q;
+  uint8_t* sK = smem + Lo::OFF_KV;
+  uint8_t* sV = smem + Lo::OFF_KV + KT;
+  uint8_t* sSOP = smem + Lo::OFF_SOP;
+  Bars bars = carve<NKV>(smem + Lo::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lo::OFF_BAR + Lo::NBARS * 8);
 
   if (tid == 0) {
     s_abort = 0;
@@ -236,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bars.drain, 1);
     fence_mbar_init();
   }
-  init_ones_block(smem + OFF_ONES, tid, kThreads);
+  init_ones_block(smem + Lo::OFF_ONES, tid, kThreads);
   fence_proxy_async_smem();
   if (warp == 17) tmem_alloc(tmem_slot, TM_COLS);
   tc_fence_before();
@@ -251,8 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (with a precomputed carry, slot blk alone)
   const int nprev =
       (!kCarry || a.ws == nullptr) ? 0 : (a.carry_pre ? 1 : (causal ? blk : a.nb));
-  float* carry_s = reinterpret_cast<float*>(smem + OFF_SOP);
-  float* carry_z = reinterpret_cast<float*>(smem + OFF_Z);
+  float* carry_s = reinterpret_cast<float*>(smem + Lo::OFF_SOP);
+  float* carry_z = reinterpret_cast<float*>(smem + Lo::OFF_Z);
   if (kCarry && nprev > 0 && warp < 16) {
     sum_aggregates<512>(reinterpret_cast<const float4*>(a.ws) +
                             ((size_t)(s * a.Hkv + g) * a.nb + (a.carry_pre ? blk : 0)) * (E / 4),
@@ -319,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dKk = smem_desc_sw128(smem_u32(sK), 16, 1024);      // K-major
       const uint64_t dKmn = smem_desc_sw128(smem_u32(sK), kBox, 1024);   // MN-major
       const uint64_t dVmn = smem_desc_sw128(smem_u32(sV), kBox, 1024);   // MN-major V
-      const uint32_t ones = smem_u32(smem + OFF_ONES);
+      const uint32_t ones = smem_u32(smem + Lo::OFF_ONES);
       const uint64_t dSop = smem_desc_sw128(smem_u32(sSOP), D * kRowBytes, 1024);
       bool ok = true;
       // dS (or the running S for the non-causal state pass) = phi(K)^T [V | 1]
@@ -433,9 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           issue_qs(tmem + TM_ACC + as * ACCW, qs, false);
           umma_commit(&bars.acc_full[as]);
-          // (with TMA output the epilogue releases the Q slot: it stages the
-          // output tile there)
-          if (!kTmaOut) umma_commit(&bars.q_empty[qs]);
+          umma_commit(&bars.q_empty[qs]);
         }
       }
       umma_commit(bars.drain);
@@ -531,7 +542,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (x == 0) mbar_arrive(&bars.pb_full[as]);
       return true;
     };
-    int q_pend = -1;  // thread 0: the item whose stored tile still holds its Q slot
     auto epilogue = [&](int j) -> bool {
       const int r = j / G, h = j % G, as = j & 1, c = c0 + r;
       if (!mbar_wait(&bars.acc_full[as], (j >> 1) & 1, abort_flag, a.err, kWaitLimitNs))
@@ -560,28 +570,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 16; ++e)
           pk[cb * 16 + e] = pack_bf16x2(n[2 * e] * inv, n[2 * e + 1] * inv);
       }
+      if (kTmaOut) {
+        // staging tile j & 1 was last stored from by item j-2: its reads are
+        // done once at most one bulk group (item j-1's) is pending
+        if (x == 0 && j >= 2) bulk_wait_read_but_last();
+      }
       tc_fence_before();
       named_bar_sync(2, 128);
       if (x == 0) mbar_arrive(&bars.acc_empty[as]);
-      // Non-causal: the item's Q slot is free (its last reader, phi(Q)
-      // [S|z], is complete), so a whole chunk is staged there (128-byte
-      // swizzle) and written by one TMA store; the slot is released at the
-      // next item's epilogue, when the store has long read it.  Causal: the
-      // Q slots stay with the producer (the chunk chain paces the Q stream
-      // and a slot held by an epilogue stalls it), rows are stored directly,
-      // as are the rows of a ragged last chunk (a tile would run into the
-      // next sequence).
-      const int valid = min(kChunk, ntok - c * kChunk);
-      const int qs = j % NQ;
-      auto release_pending = [&]() {
-        if (q_pend >= 0) {
-          bulk_wait_read_all();
-          mbar_arrive(&bars.q_empty[q_pend % NQ]);
-          q_pend = -1;
-        }
-      };
-      if (kTmaOut && valid == kChunk) {
-        uint8_t* tile = sQ + qs * QT;
+      if (kTmaOut) {
+        uint8_t* tile = smem + Lo::OFF_OST + (j & 1) * OSTT;
 #pragma unroll
         for (int q = 0; q < DV / 8; ++q)
           *reinterpret_cast<uint4*>(tile + sw128_off(row, q)) =
@@ -589,22 +587,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         named_bar_sync(2, 128);
         if (x == 0) {
-          release_pending();
-          tma_store_3d(&tm_o, tile, 0, g * G + h, t0 + c * kChunk);
+          tma_store_4d(&tm_o, tile, 0, g * G + h, c * kChunk, s);
           bulk_commit_group();
-          q_pend = j;
         }
       } else {
+        const int valid = min(kChunk, ntok - c * kChunk);
         if (row < valid) {
           uint4* orow = reinterpret_cast<uint4*>(
               a.out + ((size_t)(t0 + c * kChunk + row) * a.Hq + (size_t)(g * G + h)) * DV);
 #pragma unroll
           for (int q = 0; q < DV / 8; ++q)
             orow[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
-        if (kTmaOut && x == 0) {
-          release_pending();
-          mbar_arrive(&bars.q_empty[qs]);
         }
       }
       return true;
@@ -615,13 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (causal && t < n_items) ok = mask_p(t);
       if (ok && t > 0) ok = epilogue(t - 1);
     }
-    if (kTmaOut && x == 0) {
-      if (q_pend >= 0) {
-        bulk_wait_read_all();
-        mbar_arrive(&bars.q_empty[q_pend % NQ]);
-      }
-      bulk_wait_all();  // every output store has landed
-    }
+    if (kTmaOut && x == 0) bulk_wait_all();  // every output store has landed
   } else if (warp < 16) {
     // -------------------------------------------------- state warpgroup
     // The running [S | z] is an fp32 M=64 accumulator in TMEM (S_acc): state
@@ -724,10 +711,15 @@ namespace {
 cudaError_t launch_block(const FwdLaunch& p, int nb, const float* ws, bool carry_pre,
                          cudaStream_t stream) {
   CUtensorMap tq, tk, tv, to;
+  // TMA stores for dense non-causal launches: in causal mode the epilogue
+  // shares warps with the mask, which is on the chunk chain, and the fourth
+  // K/V stage matters to packed inputs
+  const bool tma_out = p.cu_seqlens == nullptr && p.causal == 0;
   if (!make_tmap_3d(&tq, p.q, D, p.Hq, p.total_tokens, 64) ||
       !make_tmap_3d(&tk, p.k, D, p.Hkv, p.total_tokens, 64) ||
       !make_tmap_3d(&tv, p.v, DV, p.Hkv, p.total_tokens, 64) ||
-      !make_tmap_3d(&to, p.out, DV, p.Hq, p.total_tokens, 64))
+      (tma_out ? !make_tmap_4d_dense(&to, p.out, DV, p.Hq, p.N, p.B, 64)
+               : !make_tmap_3d(&to, p.out, DV, p.Hq, p.total_tokens, 64)))
     return cudaErrorInvalidValue;
   BlockArgs a;
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
@@ -744,13 +736,13 @@ cudaError_t launch_block(const FwdLaunch& p, int nb, const float* ws, bool carry
   a.eps = p.eps;
   a.total_tokens = (int)p.total_tokens;
   a.err = p.err;
-  const bool tma_out = p.causal == 0;
   auto fk = a.ws != nullptr
                 ? (tma_out ? lt_block_fwd_kernel<true, true> : lt_block_fwd_kernel<true, false>)
                 : (tma_out ? lt_block_fwd_kernel<false, true> : lt_block_fwd_kernel<false, false>);
-  cudaError_t e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  const int smem = tma_out ? BL<true>::SMEM : BL<false>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  fk<<<dim3(nb, p.Hkv, p.B), kThreads, SMEM, stream>>>(tq, tk, tv, to, a);
+  fk<<<dim3(nb, p.Hkv, p.B), kThreads, smem, stream>>>(tq, tk, tv, to, a);
   return cudaGetLastError();
 }
 }  // namespace

@@ -146,5 +146,36 @@ inline bool make_tmap_3d(CUtensorMap* m, const void* base, int inner, int heads,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Dense [B][N][heads][inner] bf16 tensor as a 4-D map (inner, head, token in
+// the sequence, sequence) with a {box_inner, 1, kChunk, 1} box: a tile
+// stored at the end of a sequence is clipped at N instead of running into
+// the next sequence.
+inline bool make_tmap_4d_dense(CUtensorMap* m, const void* base, int inner, int heads, long long n,
+                               long long b, int box_inner) {
+  using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static EncodeFn encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return false;
+    encode = reinterpret_cast<EncodeFn>(fn);
+  }
+  const cuuint64_t row = (cuuint64_t)inner * heads * 2;
+  const cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)heads, (cuuint64_t)n, (cuuint64_t)b};
+  const cuuint64_t strides[3] = {(cuuint64_t)inner * 2, row, row * (cuuint64_t)n};
+  const cuuint32_t box[4] = {(cuuint32_t)box_inner, 1u, (cuuint32_t)kChunk, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 }  // namespace fwd
 }  // namespace lt
