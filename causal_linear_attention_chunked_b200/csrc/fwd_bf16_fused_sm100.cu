@@ -154,15 +154,16 @@ __device__ __forceinline__ void store_operand_row(uint8_t* op, int row, const fl
 
 // The carry C = S0 + the aggregates of blocks [0, nsum) of one lane (base:
 // that lane's first aggregate; s0, z0: the lane's given state or nullptr),
-// fp32 in block order, rounded once to bf16 into the K-major operand; rows
-// DV+1 .. OPR-1 zeroed.  With s_out, also the final state C + base[own]
-// (own < 0: C itself) in fp32, in the [d][dv] layout.  Thread u of NT.
+// fp32 in block order into acc (PER float4 per thread), rounded once to bf16
+// into the K-major operand; rows DV+1 .. OPR-1 zeroed.  Thread u of NT.
+template <int NT>
+constexpr int gather_per() { return (E4 + NT - 1) / NT; }
+
 template <int NT, int NF>
-__device__ __forceinline__ void gather_carry(const float4* base, int nsum, uint8_t* op, int u,
-                                             const float* s0, const float* z0, float* s_out,
-                                             float* z_out, int own) {
-  constexpr int PER = (E4 + NT - 1) / NT;
-  float4 acc[PER];
+__device__ __forceinline__ void gather_carry(float4 (&acc)[gather_per<NT>()], const float4* base,
+                                             int nsum, uint8_t* op, int u, const float* s0,
+                                             const float* z0) {
+  constexpr int PER = gather_per<NT>();
 #pragma unroll
   for (int e = 0; e < PER; ++e) {
     const int i = u + e * NT, row = i >> 4, c4 = i & 15;
@@ -209,30 +210,44 @@ __device__ __forceinline__ void gather_carry(const float4* base, int nsum, uint8
       const int row = i >> 4, c4 = i & 15;  // 16 float4 per 64-float row
       uint2 w = make_uint2(pack_bf16x2(acc[e].x, acc[e].y), pack_bf16x2(acc[e].z, acc[e].w));
       *reinterpret_cast<uint2*>(op + sw128_off(row, c4 >> 1) + (c4 & 1) * 8) = w;
-      if (s_out != nullptr) {
-        float4 f = acc[e];
-        if (own >= 0) {
-          const float4 a = __ldcg(base + (size_t)own * E4 + i);
-          f.x += a.x;
-          f.y += a.y;
-          f.z += a.z;
-          f.w += a.w;
-        }
-        if (row < DV) {
-          s_out[(4 * c4) * DV + row] = f.x;
-          s_out[(4 * c4 + 1) * DV + row] = f.y;
-          s_out[(4 * c4 + 2) * DV + row] = f.z;
-          s_out[(4 * c4 + 3) * DV + row] = f.w;
-        } else {
-          *reinterpret_cast<float4*>(z_out + 4 * c4) = f;
-        }
-      }
     }
   }
   // zero rows DV+1 .. OPR-1 (15 rows of 8 pieces)
   for (int i = u; i < (OPR - DV - 1) * 8; i += NT) {
     const int row = DV + 1 + (i >> 3);
     *reinterpret_cast<uint4*>(op + sw128_off(row, i & 7)) = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// The final state C + base[own] (own < 0: C itself) in fp32, in the [d][dv]
+// layout, from gather_carry's acc.
+template <int NT>
+__device__ __forceinline__ void write_final_state(const float4 (&acc)[gather_per<NT>()],
+                                                  const float4* base, int u, float* s_out,
+                                                  float* z_out, int own) {
+  constexpr int PER = gather_per<NT>();
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    const int i = u + e * NT;
+    if (i < E4) {
+      const int row = i >> 4, c4 = i & 15;
+      float4 f = acc[e];
+      if (own >= 0) {
+        const float4 a = __ldcg(base + (size_t)own * E4 + i);
+        f.x += a.x;
+        f.y += a.y;
+        f.z += a.z;
+        f.w += a.w;
+      }
+      if (row < DV) {
+        s_out[(4 * c4) * DV + row] = f.x;
+        s_out[(4 * c4 + 1) * DV + row] = f.y;
+        s_out[(4 * c4 + 2) * DV + row] = f.z;
+        s_out[(4 * c4 + 3) * DV + row] = f.w;
+      } else {
+        *reinterpret_cast<float4*>(z_out + 4 * c4) = f;
+      }
+    }
   }
 }
 
@@ -321,18 +336,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The carry sum, by the transform warps (256 threads) between two
   // barriers 5.
   auto gather_part = [&](int u) {
+    float4 acc[gather_per<kXf>()];
     named_bar_sync(5, kXf);
     if (!*abort_flag) {
-      gather_carry<kXf, 2>(agg_base, nprev, sC, u,
-                        a.s0 ? a.s0 + lane_idx * D * DV : nullptr,
-                        a.z0 ? a.z0 + lane_idx * D : nullptr,
-                        final_state ? a.s_out + lane_idx * D * DV : nullptr,
-                        final_state ? a.z_out + lane_idx * D : nullptr,
-                        causal ? blk : -1);
+      gather_carry<kXf, 2>(acc, agg_base, nprev, sC, u,
+                           a.s0 ? a.s0 + lane_idx * D * DV : nullptr,
+                           a.z0 ? a.z0 + lane_idx * D : nullptr);
       fence_proxy_async_smem();
     }
     named_bar_sync(5, kXf);
     if (u == 0 && !*abort_flag) mbar_arrive(bars.c_full);
+    // the final state after the carry is released: off the path to the
+    // carry products
+    if (final_state && !*abort_flag)
+      write_final_state<kXf>(acc, agg_base, u, a.s_out + lane_idx * D * DV,
+                             a.z_out + lane_idx * D, causal ? blk : -1);
   };
 
   // Accumulator of item j -> normalised bf16 row, one thread per row (TMEM
