@@ -746,12 +746,13 @@ extern "C" lt_status_t lt_linear_attn_bwd(const void* q, const void* k, const vo
   int* err = lt::device_error_word_current();
   if (!err) return LT_ERR_CUDA;
   if (lt::injected_workspace_alloc_failure()) return LT_ERR_CUDA;
-  // blocks per sequence: about two CTAs per SM in the KV-head launches
+  // blocks per sequence: about four CTAs per SM in the KV-head launches (two
+  // and eight measured slower at the headline, GQA and long shapes)
   const int sms = lt::device_sm_count();
   if (sms <= 0) return LT_ERR_CUDA;
   const long long lanes = (long long)B * H_kv;
   const long long nch = (N + 31) / 32;  // chunks of the longest possible sequence
-  long long nb = (2LL * sms + lanes - 1) / lanes;
+  long long nb = (4LL * sms + lanes - 1) / lanes;
   if (nb > nch) nb = nch;
   if (nb < 1) nb = 1;
   const long long lb = ((N + nb - 1) / nb + 31) / 32 * 32;

@@ -14,11 +14,11 @@
 #include <cooperative_groups.h>
 #include <cuda_runtime_api.h>  // CUDART_VERSION
 
-// grid_barrier (below) uses the barrier word of the cooperative-groups grid
+// grid_arrive / grid_wait (below) use the barrier word of the cooperative-groups grid
 // workspace and its arrive protocol as the CUDA 12.8 / 12.9 headers define
 // them; another toolkit may change either, so it must be re-checked there.
 static_assert(CUDART_VERSION >= 12080 && CUDART_VERSION < 12100,
-              "grid_barrier follows the cooperative-groups grid workspace of CUDA 12.8-12.9");
+              "grid_arrive / grid_wait follow the cooperative-groups grid workspace of CUDA 12.8-12.9");
 
 namespace lt {
 
@@ -162,11 +162,8 @@ __device__ __forceinline__ void bulk_commit_group() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-// wait until every committed bulk store of this thread has read its source
-__device__ __forceinline__ void bulk_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// ... every one but the most recently committed
+// wait until every committed bulk store of this thread but the most recent
+// one has read its source
 __device__ __forceinline__ void bulk_wait_read_but_last() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
@@ -260,10 +257,6 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
   return __uint_as_float(u);
 }
 
-__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
-}
-
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -327,11 +320,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
-}
-
-__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
-  __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
-  return __bfloat1622float2(h);
 }
 
 // Hardware base-2 exponential (MUFU), fp32 in and out.
@@ -429,164 +417,17 @@ __device__ __forceinline__ uint32_t pack_out(float lo, float hi) {
   }
 }
 
-// Feature map of the method: phi(x) = ELU(x) + 1 = x + 1 (x > 0), e^x (x <= 0).
-__device__ __forceinline__ float phi_f(float x) {
-  const float e = __expf(fminf(x, 0.0f));
-  return x > 0.0f ? x + 1.0f : e;
-}
-
-}  // namespace lt
-
-// ------------------------------------------------------------- clusters
-namespace lt {
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-// All threads of all CTAs of the cluster (release/acquire at cluster scope).
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Address of the same shared-memory variable in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
-  return r;
-}
-
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void st_cluster_f4(uint32_t addr, float4 v) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x),
-               "f"(v.y), "f"(v.z), "f"(v.w)
-               : "memory");
-}
-
-// Asynchronous 16-byte store into the shared memory of a CTA of the
-// cluster; completes 16 transaction bytes on that CTA's mbarrier (both
-// addresses cluster-mapped, same target CTA).
-__device__ __forceinline__ void st_async_f4(uint32_t cluster_addr, float4 v,
-                                            uint32_t cluster_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, "
-      "[%5];" ::"r"(cluster_addr),
-      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(cluster_bar)
-      : "memory");
-}
-
-// Bulk copy (TMA engine) from this CTA's shared memory into the shared
-// memory of a CTA of the cluster, completing `bytes` on that CTA's mbarrier.
-// Addresses 16-byte aligned, size a multiple of 16.
-__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint32_t src_cta,
-                                                     uint32_t bytes, uint32_t bar_cluster) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
-      "[%3];" ::"r"(dst_cluster),
-      "r"(src_cta), "r"(bytes), "r"(bar_cluster)
-      : "memory");
-}
-
-__device__ __forceinline__ void fence_acq_rel_cluster() {
-  asm volatile("fence.acq_rel.cluster;" ::: "memory");
-}
-
-// Arrive on an mbarrier of CTA-in-cluster (cluster-mapped address), with
-// release semantics at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait with cluster-scope acquire (see mbar_wait).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort, int* err,
-                                                  uint64_t limit_ns) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (global_timer_ns() - t0 > limit_ns) {
-        *abort = 1;
-        report_error(err, kDevErrTimeout);
-        return false;
-      }
-    }
-  }
-}
-
 // ------------------------------------------------------------ grid barrier
 // Grid-wide barrier of a cooperative launch, on the barrier word the driver
 // provides to such a launch (the word and the flip-bit protocol of the
 // cooperative-groups grid synchronisation: every CTA adds 1 and block
 // (0,0,0) adds 2^31 - (ctas - 1), so the top bit flips once every CTA has
-// arrived and the low bits return to their former value).  One thread per
-// CTA, exactly once per CTA and launch, on every path.  wait = false:
-// arrive only.  The wait is bounded like mbar_wait.
-__device__ __forceinline__ bool grid_barrier(bool wait, volatile int* abort, int* err,
-                                             uint64_t limit_ns) {
-  cooperative_groups::details::grid_workspace* gw =
-      cooperative_groups::details::get_grid_workspace();
-  if (gw == nullptr) {  // not a cooperative launch
-    *abort = 1;
-    report_error(err, kDevErrTimeout);
-    return false;
-  }
-  unsigned int* bar = &gw->barrier;
-  const unsigned int ctas = gridDim.x * gridDim.y * gridDim.z;
-  const bool master = (blockIdx.x | blockIdx.y | blockIdx.z) == 0;
-  const unsigned int inc = master ? 0x80000000u - (ctas - 1u) : 1u;
-  unsigned int old;
-  asm volatile("atom.add.release.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(bar), "r"(inc)
-               : "memory");
-  if (!wait) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (;;) {
-    unsigned int cur;
-    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(bar) : "memory");
-    if ((cur ^ old) & 0x80000000u) return true;
-    if (*abort) return false;
-    if (global_timer_ns() - t0 > limit_ns) {
-      *abort = 1;
-      report_error(err, kDevErrTimeout);
-      return false;
-    }
-    __nanosleep(128);  // one poller per CTA on one word: keep its line cool
-  }
-}
-
-
-// The grid barrier above split in two, for a CTA that arrives early and
-// waits later.  grid_arrive: one thread per CTA, exactly once per CTA and
-// launch, on every path; it stores the barrier word's value before the
-// arrival in *old and returns false (after recording an error) when the
-// launch is not cooperative.  grid_wait(old): wait, bounded like mbar_wait,
-// until every CTA has arrived.
+// arrived and the low bits return to their former value), in two parts for a
+// CTA that arrives early and waits later.  grid_arrive: one thread per CTA,
+// exactly once per CTA and launch, on every path; it stores the barrier
+// word's value before the arrival in *old and returns false (after recording
+// an error) when the launch is not cooperative.  grid_wait(old): wait,
+// bounded like mbar_wait, until every CTA has arrived.
 __device__ __forceinline__ bool grid_arrive(unsigned int* old, volatile int* abort, int* err) {
   cooperative_groups::details::grid_workspace* gw =
       cooperative_groups::details::get_grid_workspace();

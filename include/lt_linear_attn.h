@@ -345,7 +345,7 @@ LT_API lt_status_t lt_linear_attn_state_carry(const float *S_all, const float *z
  * CTAs from carried block sums (added in block order: the results do not
  * depend on scheduling).  Scratch: a stream-ordered workspace of
  * tokens * H_q * (dv + 1) + B * (H_q + H_kv) * nb * (d * dv + d) floats (nb
- * blocks per sequence, at most twice the SM count), released before return.
+ * blocks per sequence, at most four times the SM count), released before return.
  * Returns as lt_linear_attn_fwd.
  */
 LT_API lt_status_t lt_linear_attn_bwd(const void *q, const void *k, const void *v,
