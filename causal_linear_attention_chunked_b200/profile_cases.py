@@ -3,13 +3,12 @@
     python -m causal_linear_attention_chunked_b200.profile_cases CASE
 
 CASE is one of:
-  fused    the headline forward pass (bf16, B=2, H=8, N=4096, d=dv=64, causal):
+  fused    the forward pass at bf16, B=2, H=8, N=4096, d=dv=64, causal:
            six calls over eight seeded input sets, so a capture can skip the
            first launches and still see a launch with cold inputs
   decode   eight decode steps of the decode workload (B=64, H=8, d=dv=64) from
            a zero state
-  bwd      one backward call at the headline shape with a random upstream
-           gradient
+  bwd      one backward call at that shape with a random upstream gradient
   gqa      four forward passes of the GQA workload cut to one sequence
            (B=1, Hq=32, Hkv=8, N=16384, d=dv=128)
 

@@ -197,7 +197,7 @@ def test_block_kernel_block_counts(sched, nb, case, mode):
 FUSED_CASES = [
     # (B, Hq, Hkv, N, causal, forced block count or 0): one cooperative launch
     # in which the blocks publish and gather the aggregates themselves
-    (2, 8, 8, 4096, True, 0),        # the headline shape: 8 blocks of 4 chunks
+    (2, 8, 8, 4096, True, 0),        # B2 H8 N4096: 8 blocks of 4 chunks
     (4, 8, 8, 2000, True, 0),        # 4 blocks of 4 chunks, ragged last chunk
     (1, 4, 4, 7 * 128 + 117, True, 0),  # 8 blocks of 1 chunk
     (2, 4, 1, 1000, True, 0),        # 4 query heads per KV head: 8 blocks of 1 chunk
